@@ -1,0 +1,447 @@
+"""Benchmark of the cached causal Conv3D call on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ccv3d|reference]
+                    [--workload NAME]
+
+One step is one ccv3d_forward call (the whole hot path: per-call validation,
+tensor-map encode, one launch that computes the implicit GEMM with the bias
+epilogue and writes new_cache) on the decoder-bottleneck signature
+bf16 384->384, 3x3x3, 90x160, 2-frame cache + 1 frame.  Plans are made once
+per signature, as a decoder does; the planner's own cost is reported apart.
+
+Metric: effective TFLOP/s = 2*N*Cout*H_o*W_o*Cin*kh*kw*sum_k(o_h-o_l) per
+call (active temporal taps only) / time.  Inputs are resident in HBM; the
+timed loop rotates over enough independent input/weight/output sets to exceed
+the 126 MB L2, so no call finds its operands in L2 from the previous use.
+Under torchrun (N > 1) every rank runs an independent replica (weak scaling,
+no collective on the data path); time is the max over ranks.
+
+`--impl reference` times the FP64 CPU oracle on the host cores instead, on a
+bounded sample of output points of the same call.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_conv3d_video_b200 import synth, workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algorithmic(conv, intervals):
+    """FLOPs and bytes of one call (active taps only; Z read once, W once,
+    out and new_cache written once)."""
+    T_o, H_o, W_o = intervals["T_o"], intervals["H_o"], intervals["W_o"]
+    tap_frames = sum(intervals["o_h"][k] - intervals["o_l"][k] for k in range(conv.kt))
+    flops = 2.0 * conv.N * conv.Cout * H_o * W_o * conv.Cin * conv.kh * conv.kw * tap_frames
+    e = 2 if conv.dtype == "bf16" else 4
+    z = conv.cache_len + conv.T_x
+    keep = min(conv.cache_keep, z)
+    nbytes = e * (z * conv.N * conv.H * conv.W * conv.Cin
+                  + conv.Cout * conv.Cin * conv.kt * conv.kh * conv.kw
+                  + conv.N * T_o * H_o * W_o * conv.Cout
+                  + conv.N * keep * conv.H * conv.W * conv.Cin
+                  + (conv.Cout if conv.has_bias else 0))
+    return flops, nbytes
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_conv3d_video_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(workload_name):
+    """DRAM bytes per launch from profiles/traffic.tsv, only if that row was
+    captured with the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.tsv")
+    if not os.path.exists(path):
+        return None
+    digest = kernel_source_digest()
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = line.split("\t")
+        if len(parts) >= 3 and parts[0] == workload_name and parts[1] == digest:
+            return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from causal_conv3d_video_b200 import ccv3d
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    conv = workloads.WORKLOADS[args.workload]
+    t0 = time.perf_counter()
+    plan = ccv3d.Plan(ccv3d.desc_for(conv))
+    plan_us = (time.perf_counter() - t0) * 1e6
+    flops, nbytes = algorithmic(conv, plan.intervals)
+    dt = torch.bfloat16 if conv.dtype == "bf16" else torch.float32
+
+    # independent operand sets, enough to exceed L2 between two uses of one set
+    n_sets = max(2, int(np.ceil(2.0 * L2_BYTES / nbytes)) + 1)
+    sets = []
+    for i in range(n_sets):
+        inp = synth.conv_inputs(**conv.synth_kwargs(), stream_base=16 * i)
+        to = lambda a: None if a is None else torch.from_numpy(a).to(dt).to(dev)
+        out, nc = plan.alloc_outputs(dev)
+        sets.append((to(inp["x"]), to(inp["cache"]), to(inp["w"]), to(inp["bias"]), out, nc))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        x, c, w, b, out, nc = sets[i % n_sets]
+        plan.forward(x, c, w, b, out, nc, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if plan.status() != 0:
+        raise RuntimeError("device status after warm-up: %d" % plan.status())
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+    calls0 = plan.stats()
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clocks:
+        if dist:
+            tdist.barrier()
+        torch.cuda.synchronize()
+        events[0].record(stream)
+        for i in range(args.steps):
+            step(i)
+            events[i + 1].record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            tdist.barrier()
+    per = [events[i].elapsed_time(events[i + 1]) for i in range(args.steps)]
+    total_ms = events[0].elapsed_time(events[-1])
+    calls1 = plan.stats()
+    launches = (calls1["tc_path"] + calls1["simt_path"]) - (calls0["tc_path"] + calls0["simt_path"])
+    status = plan.status()
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {status}")
+
+    # ---- end to end through the C ABI with host buffers -------------------
+    x, c, w, b, out, nc = sets[0]
+    hx = torch.empty(x.shape, dtype=dt, pin_memory=True).copy_(x)
+    hc = torch.empty(c.shape, dtype=dt, pin_memory=True).copy_(c) if c is not None else None
+    ho = torch.empty(out.shape, dtype=dt, pin_memory=True)
+    hn = torch.empty(nc.shape, dtype=dt, pin_memory=True) if nc is not None else None
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    h2d = hx.numel() * hx.element_size() + (hc.numel() * hc.element_size() if hc is not None else 0)
+    d2h = ho.numel() * ho.element_size() + (hn.numel() * hn.element_size() if hn is not None else 0)
+
+    def e2e_step():
+        x.copy_(hx, non_blocking=True)
+        if hc is not None:
+            c.copy_(hc, non_blocking=True)
+        plan.forward(x, c, w, b, out, nc, stream)
+        ho.copy_(out, non_blocking=True)
+        if hn is not None:
+            hn.copy_(nc, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb)
+
+    if dist:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    avg_launch_s = (sum(per) / len(per)) / 1e3
+    achieved = flops / avg_launch_s / 1e12
+    peak = peaks["bf16_tflops"]
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+    csum = clocks.summary()
+    line = {
+        "metric": "cached causal Conv3D effective TFLOP/s (bf16), 1 GPU",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": conv.dtype,
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/(Cin*27)) weights)",
+        "config": {
+            "workload": conv.name, "N": conv.N, "Cin": conv.Cin, "Cout": conv.Cout,
+            "kernel": [conv.kt, conv.kh, conv.kw], "H": conv.H, "W": conv.W,
+            "T_x": conv.T_x, "cache_len": conv.cache_len, "stride": list(conv.stride),
+            "pad": list(conv.pad), "dilation": list(conv.dilation),
+            "gflop_per_call": round(flops / 1e9, 3), "mb_per_call": round(nbytes / 1e6, 2),
+            "l2": f"rotating {n_sets} operand sets of {nbytes / 1e6:.1f} MB "
+                  f"({n_sets * nbytes / 1e6:.0f} MB > 126 MB L2)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "plan": "one plan per signature, made before timing",
+            "planner_us": round(plan_us, 1),
+            "path": "tcgen05" if plan.path["tc"] else "simt",
+            "tile": [plan.path["tile_m"], plan.path["tile_n"]],
+        },
+        "us_per_call_median": round(statistics.median(per) * 1e3, 2),
+        "roofline": {
+            "bound": "tensor" if conv.dtype == "bf16" else "alu",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic_from_profiles(conv.name),
+            "peak_source": f"{peaks['source']} (bf16 burst)",
+            "hbm_frac_of_measured": round(nbytes / avg_launch_s / 1e9 / peaks["hbm_gbs"], 4),
+            "t_star_us": round(max(flops / (peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e6, 2),
+        },
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "steps": e2e_steps,
+                "what": "pinned host x+cache -> device, ccv3d_forward, out+new_cache -> "
+                        "pinned host; weights resident"},
+        "gpu_launches": int(launches),
+        "clocks": csum,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(conv, args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------------- CPU oracle
+class OracleSampler:
+    """The FP64 oracle evaluated on random output points of one call: a
+    bounded sample of the workload for the CPU baseline."""
+
+    def __init__(self, conv):
+        import oracle
+
+        self.oracle = oracle
+        self.conv = conv
+        self.op = oracle.params(conv.N, conv.Cin, conv.Cout, conv.H, conv.W, conv.T_x,
+                                conv.cache_len, kt=conv.kt, kh=conv.kh, kw=conv.kw,
+                                pad_t_base=conv.pad_t_base, cache_keep=conv.cache_keep,
+                                stride=conv.stride, pad=conv.pad, dilation=conv.dilation)
+        inp = synth.conv_inputs(**conv.synth_kwargs())
+        f64 = lambda a: None if a is None else a.astype(np.float64)
+        self.x, self.cache, self.w, self.b = (f64(inp["x"]), f64(inp["cache"]),
+                                              f64(inp["w"]), f64(inp["bias"]))
+        T_o, H_o, W_o, _ = oracle.shape(self.op)
+        _, _, o_l, o_h, _ = oracle.tap_scan(self.op)
+        self.intervals = {"T_o": T_o, "H_o": H_o, "W_o": W_o, "o_l": o_l, "o_h": o_h}
+        self.flops, self.nbytes = algorithmic(conv, self.intervals)
+        self.out_shape = (conv.N, T_o, H_o, W_o, conv.Cout)
+        self.n_out = int(np.prod(self.out_shape))
+        self.cores = oracle.threads()
+        self.rng = np.random.default_rng(0)
+
+    def sample(self, n):
+        return np.stack([self.rng.integers(0, s, n) for s in self.out_shape], axis=1)
+
+    def run(self, n):
+        """Evaluate n random points; returns seconds taken."""
+        idx = self.sample(n)
+        t = time.perf_counter()
+        self.oracle.points(self.op, self.x, self.cache, self.w, self.b, idx)
+        return time.perf_counter() - t
+
+    def points_per_s(self):
+        self.run(256)
+        n = 2048
+        return n / max(self.run(n), 1e-6)
+
+    def tflops(self, n, seconds):
+        return n * (self.flops / self.n_out) / seconds / 1e12
+
+    def describe(self, n, seconds):
+        return (f"{n} random output points of the {self.conv.name} call "
+                f"({n / self.n_out:.2%} of its outputs), FP64 direct definition, "
+                f"{seconds:.1f} s")
+
+
+def cpu_baseline(conv, seconds):
+    smp = OracleSampler(conv)
+    n = int(max(256, min(smp.n_out, smp.points_per_s() * seconds)))
+    dt = smp.run(n)
+    return {"value": round(smp.tflops(n, dt), 6), "unit": "TFLOP/s", "cores": smp.cores,
+            "kind": "oracle", "sample": smp.describe(n, dt)}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands, on the host cores."""
+    if rank != 0:
+        return None
+    conv = workloads.WORKLOADS[args.workload]
+    smp = OracleSampler(conv)
+    rate = smp.points_per_s()
+    budget_s = 150.0  # whole warm-up + timed run
+    n = int(max(16, rate * budget_s / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        smp.run(n)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        smp.run(n)
+    total = time.perf_counter() - t
+    value = round(smp.tflops(n * args.steps, total), 6)
+    return {
+        "impl": "reference",
+        "metric": "cached causal Conv3D effective TFLOP/s (bf16), 1 GPU",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": conv.name, "gflop_per_call": round(smp.flops / 1e9, 3),
+                   "points_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": smp.cores,
+                         "kind": "oracle", "sample": smp.describe(n * args.steps, total)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ccv3d", choices=["ccv3d", "reference"])
+    ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD.name,
+                    choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,54 @@
+// cache_copy.cuh -- the new_cache write: the last `keep` frames of
+// Z = [cache; x] are copied to new_cache without ever forming Z.  Frame t of
+// Z is cache[t] when t < |C|, else x[t - |C|] (the paper's cache-augmented
+// input, Sec. 4; the cache carries Z's trailing frames to the next call).
+#pragma once
+#include "params.h"
+
+namespace ccv3d {
+
+__device__ __forceinline__ const uint8_t* z_frame(const CopyJob& c, int n, int t) {
+    return t < c.cache_len
+               ? c.cache + ((long long)n * c.cache_len + t) * c.frame_bytes
+               : c.x + ((long long)n * c.T_x + (t - c.cache_len)) * c.frame_bytes;
+}
+
+// Copy part `part` of `parts` equal slices of the job with `nthreads`
+// threads (thread index `tid`).  Uses 16-byte vectors when every frame is a
+// multiple of 16 bytes (all pointers are 16-byte aligned by contract), else
+// 4-byte, else 2-byte words.
+__device__ __forceinline__ void copy_new_cache(const CopyJob& c, long long part,
+                                               long long parts, int tid,
+                                               int nthreads) {
+    if (c.keep <= 0) return;
+    const int vb = (c.frame_bytes % 16 == 0) ? 16 : ((c.frame_bytes % 4 == 0) ? 4 : 2);
+    const long long per_frame = c.frame_bytes / vb;
+    const long long frames = (long long)c.N * c.keep;
+    const long long total = per_frame * frames;
+    const long long slice = (total + parts - 1) / parts;
+    const long long begin = part * slice;
+    const long long end = begin + slice < total ? begin + slice : total;
+    if (begin >= end) return;
+    for (long long f = begin / per_frame; f < frames && f * per_frame < end; ++f) {
+        const long long lo = begin > f * per_frame ? begin - f * per_frame : 0;
+        const long long hi = end < (f + 1) * per_frame ? end - f * per_frame : per_frame;
+        const int n = (int)(f / c.keep), j = (int)(f % c.keep);
+        const uint8_t* src = z_frame(c, n, c.z_len - c.keep + j);
+        uint8_t* dst = c.dst + f * c.frame_bytes;
+        if (vb == 16) {
+            const int4* s = reinterpret_cast<const int4*>(src);
+            int4* d = reinterpret_cast<int4*>(dst);
+            for (long long v = lo + tid; v < hi; v += nthreads) d[v] = __ldg(s + v);
+        } else if (vb == 4) {
+            const int* s = reinterpret_cast<const int*>(src);
+            int* d = reinterpret_cast<int*>(dst);
+            for (long long v = lo + tid; v < hi; v += nthreads) d[v] = __ldg(s + v);
+        } else {
+            const unsigned short* s = reinterpret_cast<const unsigned short*>(src);
+            unsigned short* d = reinterpret_cast<unsigned short*>(dst);
+            for (long long v = lo + tid; v < hi; v += nthreads) d[v] = __ldg(s + v);
+        }
+    }
+}
+
+}  // namespace ccv3d

@@ -1,0 +1,483 @@
+// ccv3d.cu -- C ABI of libccv3d: planner, tensor-map builder and launches.
+//
+// The planner computes the temporal bookkeeping of "Cache-Aware Conv3D
+// Lowering Across Embedded World-Model Decoders" (Sec. 4) in integer
+// arithmetic: |Z| = |C| + T_x, p_l = p_l^base - |C|,
+// T_o = |Z| + p_l - d_t (k_t - 1), delta_k = k d_t - p_l and the valid output
+// interval [o_l, o_h) = [max(0, -delta_k), min(T_o, |Z| - delta_k)) of every
+// tap (the intersection of 0 <= o < T_o and 0 <= o + delta_k < |Z|).  Nothing
+// concatenates C and X: the kernels pick each source frame from one or the
+// other.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "ccv3d.h"
+#include "conv_simt.cuh"
+#include "conv_tc.cuh"
+#include "params.h"
+
+using namespace ccv3d;
+
+struct ccv3d_plan_s {
+    ccv3d_desc d;
+    int T_o, H_o, W_o, z_len, p_l, keep;
+    int delta[kMaxTaps], o_l[kMaxTaps], o_h[kMaxTaps];
+    int path_tc;  // 1: tcgen05 implicit GEMM, 0: SIMT
+    int BK, BN, box_h, box_w, tiles_x, tiles_y, tiles_n, stages, tmem_cols;
+    size_t smem_bytes;
+    int device;
+    int* d_status;
+    std::atomic<uint64_t> calls{0}, tc{0}, simt{0}, unsupported{0}, errors{0};
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Planner: the paper's closed forms.  Returns CCV3D_OK or the refusal code.
+ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    if (d.N < 0 || d.Cin <= 0 || d.Cout <= 0 || d.kt <= 0 || d.kh <= 0 || d.kw <= 0 ||
+        d.H <= 0 || d.W <= 0 || d.T_x < 1 || d.cache_len < 0 || d.pad_t_base < 0 ||
+        d.cache_keep < 0 || d.stride_t <= 0 || d.stride_h <= 0 || d.stride_w <= 0 ||
+        d.pad_h < 0 || d.pad_w < 0 || d.dil_t <= 0 || d.dil_h <= 0 || d.dil_w <= 0 ||
+        d.groups <= 0)
+        return CCV3D_ERR_INVALID;
+    if (d.stride_t != 1 || d.groups != 1 || d.kt != 3 ||
+        (d.dtype != CCV3D_BF16 && d.dtype != CCV3D_FP32))
+        return CCV3D_ERR_UNSUPPORTED;
+    p->z_len = d.cache_len + d.T_x;
+    p->p_l = d.pad_t_base - d.cache_len;
+    p->T_o = p->z_len + p->p_l - d.dil_t * (d.kt - 1);
+    const long long hn = (long long)d.H + 2LL * d.pad_h - (long long)d.dil_h * (d.kh - 1) - 1;
+    const long long wn = (long long)d.W + 2LL * d.pad_w - (long long)d.dil_w * (d.kw - 1) - 1;
+    p->H_o = hn < 0 ? 0 : (int)(hn / d.stride_h + 1);
+    p->W_o = wn < 0 ? 0 : (int)(wn / d.stride_w + 1);
+    p->keep = std::min(d.cache_keep, p->z_len);
+    for (int k = 0; k < kMaxTaps; ++k) {
+        p->delta[k] = p->o_l[k] = p->o_h[k] = 0;
+        if (k >= d.kt) continue;
+        const int delta = k * d.dil_t - p->p_l;
+        const int lo = std::max(0, -delta);
+        const int hi = std::min(p->T_o, p->z_len - delta);
+        p->delta[k] = delta;
+        if (hi > lo) {
+            p->o_l[k] = lo;
+            p->o_h[k] = hi;
+        }
+    }
+    if (d.N == 0 || p->T_o <= 0 || p->H_o <= 0 || p->W_o <= 0) return CCV3D_ERR_EMPTY_OUTPUT;
+    return CCV3D_OK;
+}
+
+constexpr size_t kSmemBudget = 200 * 1024;
+
+template <int BK>
+int pick_stages(int bn) {
+    int s = 8;
+    while (s > 2 && tc_smem_bytes<BK>(bn, s) > kSmemBudget) --s;
+    return s;
+}
+
+bool force_simt() {
+    const char* e = std::getenv("CCV3D_FORCE_PATH");
+    return e != nullptr && std::strcmp(e, "simt") == 0;
+}
+
+// Kernel choice and tiling.
+void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    p->path_tc = 0;
+    const bool tc_ok = d.dtype == CCV3D_BF16 && d.Cin % 16 == 0 && d.Cout % 16 == 0 &&
+                       d.stride_h <= 2 && d.stride_w <= 2 && !force_simt();
+    if (!tc_ok) return;
+    // spatial box of 128 output pixels: fewest tiles, then widest rows
+    int best_w = 0, best_tiles = 0;
+    for (int bw = 128; bw >= 8; bw /= 2) {
+        const int bh = kTileM / bw;
+        if (bw * d.stride_w > 256 || bh * d.stride_h > 256) continue;
+        const int tiles = ceil_div(p->H_o, bh) * ceil_div(p->W_o, bw);
+        if (best_w == 0 || tiles < best_tiles) {
+            best_w = bw;
+            best_tiles = tiles;
+        }
+    }
+    if (best_w == 0) return;
+    p->box_w = best_w;
+    p->box_h = kTileM / best_w;
+    p->tiles_x = ceil_div(p->W_o, p->box_w);
+    p->tiles_y = ceil_div(p->H_o, p->box_h);
+    p->tiles_n = ceil_div(d.Cout, 256);
+    p->BN = ((ceil_div(d.Cout, p->tiles_n) + 15) / 16) * 16;
+    p->BK = d.Cin % 64 == 0 ? 64 : (d.Cin % 32 == 0 ? 32 : 16);
+    switch (p->BK) {
+        case 64: p->stages = pick_stages<64>(p->BN); p->smem_bytes = tc_smem_bytes<64>(p->BN, p->stages); break;
+        case 32: p->stages = pick_stages<32>(p->BN); p->smem_bytes = tc_smem_bytes<32>(p->BN, p->stages); break;
+        default: p->stages = pick_stages<16>(p->BN); p->smem_bytes = tc_smem_bytes<16>(p->BN, p->stages); break;
+    }
+    p->tmem_cols = 32;
+    while (p->tmem_cols < p->BN) p->tmem_cols *= 2;
+    p->path_tc = 1;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+    if (a == nullptr || b == nullptr || an == 0 || bn == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+size_t elt(const ccv3d_desc& d) { return d.dtype == CCV3D_BF16 ? 2 : 4; }
+
+ccv3d_status encode_act(CUtensorMap* m, const void* base, int frames, const ccv3d_desc& d,
+                        const ccv3d_plan_s* p) {
+    const cuuint64_t dims[4] = {(cuuint64_t)d.Cin, (cuuint64_t)d.W, (cuuint64_t)d.H,
+                                (cuuint64_t)frames};
+    const cuuint64_t strides[3] = {(cuuint64_t)d.Cin * 2, (cuuint64_t)d.W * d.Cin * 2,
+                                   (cuuint64_t)d.H * d.W * d.Cin * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)p->BK, (cuuint32_t)(p->box_w * d.stride_w),
+                               (cuuint32_t)(p->box_h * d.stride_h), 1};
+    const cuuint32_t estr[4] = {1, (cuuint32_t)d.stride_w, (cuuint32_t)d.stride_h, 1};
+    const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+ccv3d_status encode_w(CUtensorMap* m, const void* base, const ccv3d_desc& d,
+                      const ccv3d_plan_s* p) {
+    const int taps = d.kt * d.kh * d.kw;
+    const cuuint64_t dims[3] = {(cuuint64_t)d.Cin, (cuuint64_t)taps, (cuuint64_t)d.Cout};
+    const cuuint64_t strides[2] = {(cuuint64_t)d.Cin * 2, (cuuint64_t)taps * d.Cin * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)p->BK, 1, (cuuint32_t)p->BN};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+CopyJob make_copy(const ccv3d_plan_s* p, const void* x, const void* cache, void* nc) {
+    CopyJob c;
+    c.x = static_cast<const uint8_t*>(x);
+    c.cache = static_cast<const uint8_t*>(cache);
+    c.dst = static_cast<uint8_t*>(nc);
+    c.frame_bytes = (long long)p->d.H * p->d.W * p->d.Cin * (long long)elt(p->d);
+    c.keep = nc != nullptr ? p->keep : 0;
+    c.cache_len = p->d.cache_len;
+    c.T_x = p->d.T_x;
+    c.z_len = p->z_len;
+    c.N = p->d.N;
+    return c;
+}
+
+Taps make_taps(const ccv3d_plan_s* p) {
+    Taps t;
+    t.kt = p->d.kt;
+    for (int k = 0; k < kMaxTaps; ++k) {
+        t.delta[k] = p->delta[k];
+        t.o_l[k] = p->o_l[k];
+        t.o_h[k] = p->o_h[k];
+    }
+    return t;
+}
+
+template <int BK>
+cudaError_t launch_tc(const TcParams& prm, int grid, size_t smem, cudaStream_t s) {
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [] {
+        attr = cudaFuncSetAttribute(conv_tc_kernel<BK>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)(227 * 1024));
+    });
+    if (attr != cudaSuccess) return attr;
+    conv_tc_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
+    return cudaGetLastError();
+}
+
+ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const void* w,
+                    const void* bias, void* out, void* nc, cudaStream_t stream) {
+    if (encode_fn() == nullptr) return CCV3D_ERR_CUDA;
+    const ccv3d_desc& d = p->d;
+    TcParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    ccv3d_status st = encode_act(&prm.tmap_x, x, d.N * d.T_x, d, p);
+    if (st == CCV3D_OK && d.cache_len > 0) st = encode_act(&prm.tmap_c, cache, d.N * d.cache_len, d, p);
+    if (st == CCV3D_OK) st = encode_w(&prm.tmap_w, w, d, p);
+    if (st != CCV3D_OK) return st;
+    prm.bias = d.has_bias ? static_cast<const uint16_t*>(bias) : nullptr;
+    prm.out = static_cast<uint16_t*>(out);
+    prm.status = p->d_status;
+    prm.copy = make_copy(p, x, cache, nc);
+    prm.taps = make_taps(p);
+    prm.N = d.N; prm.T_o = p->T_o; prm.H_o = p->H_o; prm.W_o = p->W_o;
+    prm.Cin = d.Cin; prm.Cout = d.Cout; prm.kh = d.kh; prm.kw = d.kw;
+    prm.s_h = d.stride_h; prm.s_w = d.stride_w; prm.p_h = d.pad_h; prm.p_w = d.pad_w;
+    prm.d_h = d.dil_h; prm.d_w = d.dil_w;
+    prm.cache_len = d.cache_len; prm.T_x = d.T_x;
+    prm.box_h = p->box_h; prm.box_w = p->box_w;
+    prm.tiles_x = p->tiles_x; prm.tiles_y = p->tiles_y; prm.tiles_n = p->tiles_n;
+    prm.BN = p->BN; prm.n_cb = ceil_div(d.Cin, p->BK); prm.stages = p->stages;
+    prm.tmem_cols = p->tmem_cols;
+    prm.wait_limit_ns = kWaitLimitNs;
+    const long long grid = (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
+    if (grid > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
+    cudaError_t e;
+    switch (p->BK) {
+        case 64: e = launch_tc<64>(prm, (int)grid, p->smem_bytes, stream); break;
+        case 32: e = launch_tc<32>(prm, (int)grid, p->smem_bytes, stream); break;
+        default: e = launch_tc<16>(prm, (int)grid, p->smem_bytes, stream); break;
+    }
+    return e == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const void* cache, const void* w,
+                      const void* bias, void* out, void* nc, cudaStream_t stream) {
+    const ccv3d_desc& d = p->d;
+    SimtParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.x = x; prm.cache = cache; prm.w = w;
+    prm.bias = d.has_bias ? bias : nullptr;
+    prm.out = out;
+    prm.copy = make_copy(p, x, cache, nc);
+    prm.taps = make_taps(p);
+    prm.N = d.N; prm.T_o = p->T_o; prm.H_o = p->H_o; prm.W_o = p->W_o;
+    prm.Cin = d.Cin; prm.Cout = d.Cout; prm.H = d.H; prm.W = d.W; prm.kh = d.kh; prm.kw = d.kw;
+    prm.s_h = d.stride_h; prm.s_w = d.stride_w; prm.p_h = d.pad_h; prm.p_w = d.pad_w;
+    prm.d_h = d.dil_h; prm.d_w = d.dil_w;
+    prm.cache_len = d.cache_len; prm.T_x = d.T_x;
+    prm.co_groups = ceil_div(d.Cout, kSimtCoT);
+    prm.conv_threads = (long long)d.N * p->T_o * p->H_o * p->W_o * prm.co_groups;
+    const long long cb = (prm.conv_threads + kSimtThreads - 1) / kSimtThreads;
+    const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
+    const long long kb = copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 32767) / 32768) : 0;
+    if (cb + kb > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
+    prm.conv_blocks = (int)cb;
+    prm.copy_blocks = (int)kb;
+    const int grid = (int)(cb + kb);
+    if (d.dtype == CCV3D_FP32)
+        conv_simt_kernel<float><<<grid, kSimtThreads, 0, stream>>>(prm);
+    else
+        conv_simt_kernel<__nv_bfloat16><<<grid, kSimtThreads, 0, stream>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+__global__ void wait_selftest_kernel(int* status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        // Nothing ever arrives on `bar`: the bounded wait must give up.
+        if (mbar_wait(smem_u32(&bar), 0, status, limit_ns)) atomicExch(status, -1);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+ccv3d_status ccv3d_plan(ccv3d_plan_t* out, const ccv3d_desc* desc) {
+    if (out == nullptr) return CCV3D_ERR_INVALID;
+    *out = nullptr;
+    if (desc == nullptr) return CCV3D_ERR_INVALID;
+    ccv3d_plan_s* p = new (std::nothrow) ccv3d_plan_s();
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    p->d = *desc;
+    ccv3d_status st = compute_intervals(*desc, p);
+    if (st != CCV3D_OK) {
+        delete p;
+        return st;
+    }
+    choose_path(*desc, p);
+    // The status block lives on the current device.  Without any CUDA device
+    // the plan still serves inspection (intervals, sizes, path) and
+    // ccv3d_forward refuses with CCV3D_ERR_CUDA.
+    p->device = -1;
+    p->d_status = nullptr;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
+        if (cudaGetDevice(&p->device) != cudaSuccess ||
+            cudaMalloc(&p->d_status, 256) != cudaSuccess ||
+            cudaMemset(p->d_status, 0, 256) != cudaSuccess) {
+            cudaGetLastError();
+            if (p->d_status) cudaFree(p->d_status);
+            delete p;
+            return CCV3D_ERR_CUDA;
+        }
+    } else {
+        cudaGetLastError();
+    }
+    *out = p;
+    return CCV3D_OK;
+}
+
+ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t p, int* T_o, int* H_o, int* W_o,
+                                  int delta[CCV3D_MAX_KT], int o_l[CCV3D_MAX_KT],
+                                  int o_h[CCV3D_MAX_KT]) {
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    if (T_o) *T_o = p->T_o;
+    if (H_o) *H_o = p->H_o;
+    if (W_o) *W_o = p->W_o;
+    for (int k = 0; k < CCV3D_MAX_KT; ++k) {
+        if (delta) delta[k] = p->delta[k];
+        if (o_l) o_l[k] = p->o_l[k];
+        if (o_h) o_h[k] = p->o_h[k];
+    }
+    return CCV3D_OK;
+}
+
+int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
+    if (p == nullptr) return -1;
+    if (tile_m) *tile_m = p->path_tc ? kTileM : 0;
+    if (tile_n) *tile_n = p->path_tc ? p->BN : 0;
+    return p->path_tc;
+}
+
+ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t p, size_t* out_bytes, size_t* nc_bytes,
+                              int* nc_frames) {
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    const ccv3d_desc& d = p->d;
+    if (out_bytes) *out_bytes = (size_t)d.N * p->T_o * p->H_o * p->W_o * d.Cout * elt(d);
+    if (nc_bytes) *nc_bytes = (size_t)d.N * p->keep * d.H * d.W * d.Cin * elt(d);
+    if (nc_frames) *nc_frames = p->keep;
+    return CCV3D_OK;
+}
+
+ccv3d_status ccv3d_forward(ccv3d_plan_t p, const void* x, const void* cache, const void* w,
+                           const void* bias, void* out, void* nc, const int stride[2],
+                           const int pad[2], const int dilation[3], cudaStream_t stream) {
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    const ccv3d_desc& d = p->d;
+    auto refuse = [&](ccv3d_status s) {
+        p->errors.fetch_add(1, std::memory_order_relaxed);
+        return s;
+    };
+    if (stride == nullptr || pad == nullptr || dilation == nullptr) return refuse(CCV3D_ERR_INVALID);
+    if (stride[0] != d.stride_h || stride[1] != d.stride_w || pad[0] != d.pad_h ||
+        pad[1] != d.pad_w || dilation[0] != d.dil_t || dilation[1] != d.dil_h ||
+        dilation[2] != d.dil_w)
+        return refuse(CCV3D_ERR_INVALID);
+    if (x == nullptr || w == nullptr || out == nullptr || (d.cache_len > 0 && cache == nullptr) ||
+        (d.has_bias && bias == nullptr) || (p->keep > 0 && nc == nullptr))
+        return refuse(CCV3D_ERR_INVALID);
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out) ||
+        (d.cache_len > 0 && !aligned16(cache)) || (nc != nullptr && !aligned16(nc)) ||
+        (d.has_bias && (reinterpret_cast<uintptr_t>(bias) % elt(d)) != 0))
+        return refuse(CCV3D_ERR_ALIGNMENT);
+    const size_t e = elt(d);
+    const size_t frame = (size_t)d.H * d.W * d.Cin * e;
+    const size_t x_bytes = (size_t)d.N * d.T_x * frame;
+    const size_t c_bytes = d.cache_len > 0 ? (size_t)d.N * d.cache_len * frame : 0;
+    const size_t nc_bytes = nc != nullptr ? (size_t)d.N * p->keep * frame : 0;
+    const size_t o_bytes = (size_t)d.N * p->T_o * p->H_o * p->W_o * d.Cout * e;
+    const size_t w_bytes = (size_t)d.Cout * d.kt * d.kh * d.kw * d.Cin * e;
+    if (overlaps(nc, nc_bytes, x, x_bytes) || overlaps(nc, nc_bytes, cache, c_bytes) ||
+        overlaps(out, o_bytes, x, x_bytes) || overlaps(out, o_bytes, cache, c_bytes) ||
+        overlaps(out, o_bytes, w, w_bytes) || overlaps(out, o_bytes, nc, nc_bytes))
+        return refuse(CCV3D_ERR_ALIAS);
+    if (p->d_status == nullptr) return refuse(CCV3D_ERR_CUDA);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return refuse(CCV3D_ERR_INVALID);
+    ccv3d_status st = p->path_tc ? run_tc(p, x, cache, w, bias, out, nc, stream)
+                                 : run_simt(p, x, cache, w, bias, out, nc, stream);
+    if (st != CCV3D_OK) return refuse(st);
+    p->calls.fetch_add(1, std::memory_order_relaxed);
+    (p->path_tc ? p->tc : p->simt).fetch_add(1, std::memory_order_relaxed);
+    return CCV3D_OK;
+}
+
+ccv3d_status ccv3d_get_stats(ccv3d_plan_t p, ccv3d_stats* s) {
+    if (p == nullptr || s == nullptr) return CCV3D_ERR_INVALID;
+    s->calls = p->calls.load();
+    s->tc_path = p->tc.load();
+    s->simt_path = p->simt.load();
+    s->unsupported = p->unsupported.load();
+    s->errors = p->errors.load();
+    s->workspace_bytes = 0;
+    return CCV3D_OK;
+}
+
+ccv3d_status ccv3d_get_status(ccv3d_plan_t p) {
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    if (p->d_status == nullptr) return CCV3D_ERR_CUDA;
+    int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return CCV3D_ERR_CUDA;
+    if (cudaMemcpy(&v, p->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return CCV3D_ERR_CUDA;
+    if (v != 0 && cudaMemset(p->d_status, 0, sizeof(int)) != cudaSuccess) return CCV3D_ERR_CUDA;
+    return v == 0 ? CCV3D_OK : (ccv3d_status)v;
+}
+
+void ccv3d_destroy(ccv3d_plan_t p) {
+    if (p == nullptr) return;
+    if (p->d_status) cudaFree(p->d_status);
+    delete p;
+}
+
+const char* ccv3d_strerror(ccv3d_status s) {
+    switch (s) {
+        case CCV3D_OK: return "ok";
+        case CCV3D_ERR_INVALID: return "invalid argument";
+        case CCV3D_ERR_UNSUPPORTED: return "unsupported call (outside the cached causal Conv3D contract)";
+        case CCV3D_ERR_EMPTY_OUTPUT: return "empty output";
+        case CCV3D_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case CCV3D_ERR_ALIAS: return "output buffer overlaps an input";
+        case CCV3D_ERR_CUDA: return "CUDA error";
+        case CCV3D_ERR_TIMEOUT: return "bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+    int* d = nullptr;
+    if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) return CCV3D_ERR_CUDA;
+    int v = 0;
+    cudaError_t e = cudaMemsetAsync(d, 0, sizeof(int), stream);
+    if (e == cudaSuccess) {
+        wait_selftest_kernel<<<1, 32, 0, stream>>>(d, limit_ns);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&v, d, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    cudaFree(d);
+    if (e != cudaSuccess) return CCV3D_ERR_CUDA;
+    if (v == kStatusTimeout) return CCV3D_ERR_TIMEOUT;
+    return v == 0 ? CCV3D_ERR_CUDA : CCV3D_OK;
+}
+
+}  // extern "C"

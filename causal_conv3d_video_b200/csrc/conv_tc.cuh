@@ -1,0 +1,225 @@
+// conv_tc.cuh -- bf16 cached causal Conv3D as one implicit GEMM on the
+// sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// GEMM view of the paper's per-tap sum (Sec. 4): rows = output pixels
+// (n, o, y, x) of one output frame, columns = Cout, reduction over
+// (active tap k, r, s, ci).  A tile of 128 output pixels is a box_h x box_w
+// spatial box of frame o.  For every active tap k the source frame
+// t = o + delta_k is picked from the cache or the input tensor map (no
+// concatenation), and for every spatial tap (r, s) one TMA box load brings the
+// shifted, strided box of BK input channels, zero-filled outside the image.
+// Weights W[co, k, r, s, ci] are read in place (K-major rows).
+//
+// Warp roles (192 threads, one CTA per output tile):
+//   warp 0     TMA producer (one lane): A box + B box per pipeline stage
+//   warp 1     TMEM owner; one lane issues tcgen05.mma (M=128, N=BN, K=16)
+//   warps 2-5  copy a slice of new_cache while the GEMM runs, then the
+//              epilogue: tcgen05.ld -> + bias (fp32) -> bf16 (RNE) -> global
+// Every mbarrier wait is bounded (mbar_wait); a timeout is recorded in the
+// status block and the roles drain and exit instead of hanging.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "cache_copy.cuh"
+#include "params.h"
+#include "ptx.cuh"
+
+namespace ccv3d {
+
+template <int BK>
+struct TcSmem {
+    static constexpr int kRowBytes = BK * 2;            // one swizzle span
+    static constexpr int kABytes = kTileM * kRowBytes;  // one A stage
+};
+
+// Dynamic shared memory needed for `stages` stages of an N=BN tile.
+template <int BK>
+__host__ __device__ constexpr size_t tc_smem_bytes(int bn, int stages) {
+    return 1024 /* alignment slack */ +
+           (size_t)stages * (TcSmem<BK>::kABytes + (size_t)bn * TcSmem<BK>::kRowBytes) +
+           (size_t)(2 * stages + 1) * 8 /* mbarriers */ + 16 /* tmem slot */ +
+           (size_t)bn * 4 /* bias */;
+}
+
+template <int BK>
+__global__ void __launch_bounds__(kTcThreads, 1)
+conv_tc_kernel(const __grid_constant__ TcParams p) {
+    constexpr int kRow = TcSmem<BK>::kRowBytes;
+    constexpr int kA = TcSmem<BK>::kABytes;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int stages = p.stages;
+    const int BN = p.BN;
+    const int kB = BN * kRow;
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + (size_t)stages * kA;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kB);
+    uint64_t* empty_bar = full_bar + stages;
+    uint64_t* acc_bar = empty_bar + stages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+    float* bias_s = reinterpret_cast<float*>(tmem_slot + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- tile coordinates: (n, o, ty, tx) x n_tile, n_tile fastest so that
+    // neighbouring CTAs share the A operand in L2.
+    const int n_tile = blockIdx.x % p.tiles_n;
+    int m_tile = blockIdx.x / p.tiles_n;
+    const int tx = m_tile % p.tiles_x;
+    m_tile /= p.tiles_x;
+    const int ty = m_tile % p.tiles_y;
+    m_tile /= p.tiles_y;
+    const int o = m_tile % p.T_o;
+    const int n = m_tile / p.T_o;
+
+    int n_active = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxTaps; ++k)
+        if (k < p.taps.kt && o >= p.taps.o_l[k] && o < p.taps.o_h[k]) ++n_active;
+    const int iters = n_active * p.kh * p.kw * p.n_cb;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        mbar_init(smem_u32(acc_bar), 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&p.tmap_x);
+        if (p.cache_len > 0) tma_prefetch_desc(&p.tmap_c);
+        tma_prefetch_desc(&p.tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+        tmem_relinquish();
+    }
+    if (warp >= 2) {
+        for (int i = threadIdx.x - 64; i < BN; i += 128) {
+            const int co = n_tile * BN + i;
+            float b = 0.f;
+            if (p.bias != nullptr && co < p.Cout)
+                b = __bfloat162float(__ushort_as_bfloat16(p.bias[co]));
+            bias_s[i] = b;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int it = 0;
+            bool ok = true;
+            const uint32_t stage_bytes = (uint32_t)(kA + kB);
+            for (int k = 0; k < p.taps.kt && ok; ++k) {
+                if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
+                const int t = o + p.taps.delta[k];  // frame of Z
+                const CUtensorMap* src;
+                int f;
+                if (t < p.cache_len) {
+                    src = &p.tmap_c;
+                    f = n * p.cache_len + t;
+                } else {
+                    src = &p.tmap_x;
+                    f = n * p.T_x + (t - p.cache_len);
+                }
+                for (int r = 0; r < p.kh && ok; ++r) {
+                    const int y0 = ty * p.box_h * p.s_h + r * p.d_h - p.p_h;
+                    for (int s = 0; s < p.kw && ok; ++s) {
+                        const int x0 = tx * p.box_w * p.s_w + s * p.d_w - p.p_w;
+                        const int wrow = (k * p.kh + r) * p.kw + s;
+                        for (int cb = 0; cb < p.n_cb; ++cb, ++it) {
+                            const int st = it % stages;
+                            if (it >= stages &&
+                                !mbar_wait(smem_u32(&empty_bar[st]), ((it / stages) & 1) ^ 1,
+                                           p.status, p.wait_limit_ns)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t fb = smem_u32(&full_bar[st]);
+                            mbar_arrive_expect_tx(fb, stage_bytes);
+                            tma_load_4d(smem_u32(sA + (size_t)st * kA), src, fb, cb * BK, x0,
+                                        y0, f);
+                            tma_load_3d(smem_u32(sB + (size_t)st * kB), &p.tmap_w, fb,
+                                        cb * BK, wrow, n_tile * BN);
+                        }
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------- MMA issuer
+            const uint32_t idesc = idesc_bf16_m128((uint32_t)BN);
+            for (int it = 0; it < iters; ++it) {
+                const int st = it % stages;
+                if (!mbar_wait(smem_u32(&full_bar[st]), (it / stages) & 1, p.status,
+                               p.wait_limit_ns))
+                    break;
+                tc_fence_after();
+                const uint64_t a_desc = smem_desc_kmajor(smem_u32(sA + (size_t)st * kA), kRow);
+                const uint64_t b_desc = smem_desc_kmajor(smem_u32(sB + (size_t)st * kB), kRow);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    // +32 bytes of K per step inside the swizzle span
+                    umma_bf16(tmem_base, a_desc + 2u * kk, b_desc + 2u * kk, idesc,
+                              (it | kk) != 0 ? 1u : 0u);
+                umma_commit(smem_u32(&empty_bar[st]));
+            }
+            umma_commit(smem_u32(acc_bar));
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- new_cache slice, then epilogue
+        const int etid = threadIdx.x - 64;
+        copy_new_cache(p.copy, blockIdx.x, gridDim.x, etid, 128);
+
+        const bool ok = mbar_wait(smem_u32(acc_bar), 0, p.status, p.wait_limit_ns);
+        tc_fence_after();
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;
+        const int y = ty * p.box_h + row / p.box_w;
+        const int x = tx * p.box_w + row % p.box_w;
+        const bool valid = ok && y < p.H_o && x < p.W_o;
+        uint16_t* orow = p.out + ((((long long)n * p.T_o + o) * p.H_o + y) * p.W_o + x) *
+                                     (long long)p.Cout;
+        const bool have_acc = iters > 0;
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+            tmem_ld_wait();
+            const int co = n_tile * BN + c0;
+            if (!valid || co >= p.Cout) continue;
+            uint32_t packed[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float a0 = (have_acc ? __uint_as_float(v[2 * j]) : 0.f) + bias_s[c0 + 2 * j];
+                const float a1 =
+                    (have_acc ? __uint_as_float(v[2 * j + 1]) : 0.f) + bias_s[c0 + 2 * j + 1];
+                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+                packed[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            if (co + 16 <= p.Cout) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + co);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            } else {
+                for (int j = 0; j < 16 && co + j < p.Cout; ++j)
+                    orow[co + j] = (uint16_t)(packed[j >> 1] >> ((j & 1) * 16));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
+    }
+}
+
+}  // namespace ccv3d

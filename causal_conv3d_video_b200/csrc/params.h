@@ -1,0 +1,65 @@
+// params.h -- kernel parameter blocks shared by the host launcher and the
+// kernels of libccv3d.  Passed by value as __grid_constant__ parameters.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+namespace ccv3d {
+
+constexpr int kMaxTaps = 3;
+constexpr int kTileM = 128;          // output pixels per GEMM tile (UMMA M)
+constexpr int kTcThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
+
+// new_cache = last `keep` frames of Z = [cache; x], copied frame by frame.
+struct CopyJob {
+    const uint8_t* x;       // [N, T_x, frame_bytes]
+    const uint8_t* cache;   // [N, cache_len, frame_bytes]
+    uint8_t* dst;           // [N, keep, frame_bytes]
+    long long frame_bytes;
+    int keep, cache_len, T_x, z_len, N;
+};
+
+// Temporal bookkeeping of one call (paper, Sec. 4): tap k of output frame o
+// reads frame o + delta[k] of Z, and is active iff o_l[k] <= o < o_h[k].
+struct Taps {
+    int kt;
+    int delta[kMaxTaps];
+    int o_l[kMaxTaps];
+    int o_h[kMaxTaps];
+};
+
+struct __align__(64) TcParams {
+    CUtensorMap tmap_x;      // x      as [N*T_x, H, W, Cin], box [BK, bw*s_w, bh*s_h, 1]
+    CUtensorMap tmap_c;      // cache  as [N*|C|, H, W, Cin] (unused when |C| = 0)
+    CUtensorMap tmap_w;      // weight as [Cout, kt*kh*kw, Cin], box [BK, 1, BN]
+    const uint16_t* bias;    // bf16 [Cout] or null
+    uint16_t* out;           // bf16 [N, T_o, H_o, W_o, Cout]
+    int* status;
+    CopyJob copy;
+    Taps taps;
+    int N, T_o, H_o, W_o, Cin, Cout, kh, kw;
+    int s_h, s_w, p_h, p_w, d_h, d_w;
+    int cache_len, T_x;
+    int box_h, box_w, tiles_x, tiles_y, tiles_n;
+    int BN, n_cb, stages, tmem_cols;
+    uint64_t wait_limit_ns;
+};
+
+struct SimtParams {
+    const void* x;
+    const void* cache;
+    const void* w;
+    const void* bias;
+    void* out;
+    CopyJob copy;
+    Taps taps;
+    int N, T_o, H_o, W_o, Cin, Cout, H, W, kh, kw;
+    int s_h, s_w, p_h, p_w, d_h, d_w;
+    int cache_len, T_x;
+    int co_groups;
+    long long conv_threads;  // N*T_o*H_o*W_o*co_groups
+    int conv_blocks, copy_blocks;
+};
+
+}  // namespace ccv3d

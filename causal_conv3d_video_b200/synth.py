@@ -13,6 +13,9 @@ Generator (one counter-based stream per tensor):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 _GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -37,38 +40,49 @@ def stream_key(seed: int, stream: int) -> np.uint64:
         return _mix(np.array([k], np.uint64))[0]
 
 
-def normal(shape, sigma: float, seed: int, stream: int) -> np.ndarray:
+def _fill(out, lo, hi, key, sigma, bf16=False):
+    with np.errstate(over="ignore"):
+        i = np.arange(lo, hi, dtype=np.uint64)
+        c1 = key + (np.uint64(2) * i + np.uint64(1)) * _GAMMA
+        c2 = key + (np.uint64(2) * i + np.uint64(2)) * _GAMMA
+        u1 = ((_mix(c1) >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0**-53
+        u2 = (_mix(c2) >> np.uint64(11)).astype(np.float64) * 2.0**-53
+        z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+        out[lo:hi] = (z * sigma).astype(np.float32)
+        if bf16:
+            out[lo:hi] = round_to_bf16(out[lo:hi])
+
+
+def normal(shape, sigma: float, seed: int, stream: int, bf16: bool = False) -> np.ndarray:
     """N(0, sigma^2) samples as float32, element i of the C-order array drawn
-    from counters 2i+1 and 2i+2 of the (seed, stream) key."""
+    from counters 2i+1 and 2i+2 of the (seed, stream) key.  Large arrays are
+    filled chunk by chunk on a thread pool (the values do not depend on it)."""
     n = int(np.prod(shape)) if len(shape) else 1
     out = np.empty(n, np.float32)
     key = stream_key(seed, stream)
-    two_pi = 2.0 * np.pi
-    with np.errstate(over="ignore"):
-        for lo in range(0, n, _CHUNK):
-            hi = min(n, lo + _CHUNK)
-            i = np.arange(lo, hi, dtype=np.uint64)
-            c1 = key + (np.uint64(2) * i + np.uint64(1)) * _GAMMA
-            c2 = key + (np.uint64(2) * i + np.uint64(2)) * _GAMMA
-            u1 = ((_mix(c1) >> np.uint64(11)).astype(np.float64) + 1.0) * 2.0**-53
-            u2 = (_mix(c2) >> np.uint64(11)).astype(np.float64) * 2.0**-53
-            z = np.sqrt(-2.0 * np.log(u1)) * np.cos(two_pi * u2)
-            out[lo:hi] = (z * sigma).astype(np.float32)
+    chunks = [(lo, min(n, lo + _CHUNK)) for lo in range(0, n, _CHUNK)]
+    if len(chunks) <= 1:
+        for lo, hi in chunks:
+            _fill(out, lo, hi, key, sigma, bf16)
+    else:
+        workers = min(len(chunks), max(1, (os.cpu_count() or 1)))
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(lambda c: _fill(out, c[0], c[1], key, sigma, bf16), chunks))
     return out.reshape(shape)
 
 
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); returned
-    as float32 holding bf16-representable values.  Inputs are finite."""
+    as float32 holding bf16-representable values.  Inputs are finite (their
+    bit patterns plus the rounding increment stay below 2**32)."""
     a = np.ascontiguousarray(a, np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    u = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) & np.uint64(0xFFFF0000)
-    return u.astype(np.uint32).view(np.float32).reshape(a.shape)
+    u = a.view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32).reshape(a.shape)
 
 
 def tensor(shape, sigma, seed, stream, dtype: str) -> np.ndarray:
-    a = normal(shape, sigma, seed, stream)
-    return round_to_bf16(a) if dtype == "bf16" else a
+    return normal(shape, sigma, seed, stream, bf16=(dtype == "bf16"))
 
 
 def conv_inputs(*, N, Cin, Cout, H, W, T_x, cache_len, kt=3, kh=3, kw=3,

@@ -1,0 +1,168 @@
+/*
+ * ccv3d.h -- cache-aware causal Conv3D for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operator ("Cache-Aware Conv3D Lowering Across Embedded World-Model
+ * Decoders", Sec. 4): a temporal cache C and the current frames X form the
+ * cache-augmented input Z = [C; X]_T.  With unit temporal stride, one group,
+ * temporal kernel k_t = 3 and effective left pad p_l = p_l^base - |C|_T,
+ * output frame o of tap k reads frame o + delta_k of Z, delta_k = k*d_t - p_l;
+ * frames outside Z contribute zero.  The output is the sum over taps of a
+ * spatial cross-correlation with W_k = W[:, :, k, :, :] (PyTorch convention,
+ * spatial stride s, padding p, dilation d), plus the bias exactly once.
+ * Tap k is active on the output interval [o_l, o_h) where
+ *   o_l = max(0, -delta_k),  o_h = min(T_o, |Z|_T - delta_k),
+ * and reads the equally long source interval [o_l + delta_k, o_h + delta_k).
+ * Each call also writes new_cache = the last min(cache_keep, |Z|_T) frames of
+ * Z, ready to be passed as the next call's cache.
+ *
+ * Memory layout (every tensor dense, row-major, channels innermost -- the
+ * physical order of PyTorch's channels_last_3d):
+ *   x          [N, T_x,  H,   W,   Cin ]
+ *   cache      [N, |C|,  H,   W,   Cin ]   NULL allowed iff cache_len == 0
+ *   w          [Cout, k_t, k_h, k_w, Cin]   a channels_last_3d Conv3d weight
+ *   bias       [Cout]                       NULL iff has_bias == 0
+ *   out        [N, T_o,  H_o, W_o, Cout]
+ *   new_cache  [N, K',   H,   W,   Cin ]   K' = min(cache_keep, |C| + T_x);
+ *                                           NULL allowed iff K' == 0
+ * Element type: CCV3D_BF16 (bf16 in, fp32 accumulate, fp32 bias add, one
+ * round-to-nearest-even to bf16 out) or CCV3D_FP32 (IEEE fp32 FMA, no TF32).
+ * bias has the element type of the activations.
+ *
+ * Ownership: the caller owns every device buffer.  A plan owns host state and
+ * one small device status block; ccv3d_forward allocates nothing, never
+ * synchronises the host, and runs asynchronously on the given stream.
+ * new_cache must not overlap x or cache (ping-pong two buffers across calls).
+ *
+ * Errors: functions return a ccv3d_status; nothing throws, exits or traps.
+ * Device-side waits are bounded: a wait that runs out records
+ * CCV3D_ERR_TIMEOUT in the plan's status block, which ccv3d_get_status reads.
+ */
+#ifndef CCV3D_H
+#define CCV3D_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define CCV3D_API __attribute__((visibility("default")))
+#else
+#define CCV3D_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CCV3D_ABI_VERSION 1
+#define CCV3D_MAX_KT 3 /* the contract's temporal kernel size */
+
+typedef enum { CCV3D_BF16 = 0, CCV3D_FP32 = 1 } ccv3d_dtype;
+
+typedef enum {
+    CCV3D_OK = 0,
+    CCV3D_ERR_INVALID = 1,      /* bad or inconsistent argument (NULL plan or
+                                   pointer, negative size, forward's
+                                   stride/pad/dilation differ from the plan) */
+    CCV3D_ERR_UNSUPPORTED = 2,  /* outside the contract: stride_t != 1,
+                                   groups != 1, k_t != 3, unknown dtype */
+    CCV3D_ERR_EMPTY_OUTPUT = 3, /* T_o, H_o or W_o would be <= 0, or N == 0 */
+    CCV3D_ERR_ALIGNMENT = 4,    /* a pointer is not 16-byte aligned */
+    CCV3D_ERR_ALIAS = 5,        /* new_cache overlaps x or cache, or out
+                                   overlaps an input */
+    CCV3D_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
+    CCV3D_ERR_TIMEOUT = 7       /* a bounded device-side wait ran out */
+} ccv3d_status;
+
+/* Conv3D call signature.  Sizes are in elements/frames. */
+typedef struct {
+    int N, Cin, Cout;
+    int kt, kh, kw;       /* kernel extent (k_t must be 3) */
+    int H, W;             /* spatial size of x and cache */
+    int T_x;              /* frames in x, >= 1 */
+    int cache_len;        /* |C|_T, frames in cache, >= 0 */
+    int pad_t_base;       /* p_l^base, causal left pad with an empty cache */
+    int cache_keep;       /* frames of Z kept in new_cache (usually p_l^base) */
+    int stride_t;         /* must be 1 */
+    int stride_h, stride_w;
+    int pad_h, pad_w;     /* symmetric zero padding */
+    int dil_t, dil_h, dil_w;
+    int groups;           /* must be 1 */
+    ccv3d_dtype dtype;
+    int has_bias;
+} ccv3d_desc;
+
+typedef struct {
+    uint64_t calls;       /* successful ccv3d_forward calls */
+    uint64_t tc_path;     /* of which ran the tcgen05 implicit-GEMM kernel */
+    uint64_t simt_path;   /* of which ran the FP32 / thin-channel kernel */
+    uint64_t unsupported; /* forward calls refused as outside the contract */
+    uint64_t errors;      /* forward calls refused for any other reason */
+    uint64_t workspace_bytes; /* device scratch used per call (0) */
+} ccv3d_stats;
+
+typedef struct ccv3d_plan_s* ccv3d_plan_t;
+
+/* Validate the signature, compute the output shape and the per-tap intervals
+ * (integer arithmetic), choose the kernel and its tiling, and allocate the
+ * plan's 256-byte device status block on the current device.  On a host with
+ * no CUDA device the plan is still made, for inspection only (intervals,
+ * sizes, path); ccv3d_forward then returns CCV3D_ERR_CUDA.  *out is set to
+ * NULL on failure.  Errors: INVALID, UNSUPPORTED, EMPTY_OUTPUT, CUDA. */
+CCV3D_API ccv3d_status ccv3d_plan(ccv3d_plan_t* out, const ccv3d_desc* desc);
+
+/* The planner's temporal bookkeeping, for inspection and testing.
+ * T_o/H_o/W_o: output extents.  For k < k_t: delta[k] = k*d_t - p_l,
+ * [o_l[k], o_h[k]) the output frames on which tap k is active; an inactive
+ * tap reports o_l = o_h = 0.  Any output pointer may be NULL. */
+CCV3D_API ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t plan, int* T_o, int* H_o,
+                                  int* W_o, int delta[CCV3D_MAX_KT],
+                                  int o_l[CCV3D_MAX_KT],
+                                  int o_h[CCV3D_MAX_KT]);
+
+/* 1 when the plan runs the tcgen05 tensor-core kernel, 0 for the SIMT kernel;
+ * tile_m/tile_n receive the GEMM tile (may be NULL). */
+CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
+
+/* Run one cached causal Conv3D call on `stream` (device pointers, layouts as
+ * above).  stride = {s_h, s_w}, pad = {p_h, p_w}, dilation = {d_t, d_h, d_w}
+ * must equal the plan's (the call signature of the paper's patched module).
+ * Pointers must be 16-byte aligned.  out and new_cache are written in the
+ * same launch.  Errors: INVALID, ALIGNMENT, ALIAS, CUDA. */
+CCV3D_API ccv3d_status ccv3d_forward(ccv3d_plan_t plan, const void* x, const void* cache,
+                           const void* w, const void* bias, void* out,
+                           void* new_cache, const int stride[2],
+                           const int pad[2], const int dilation[3],
+                           cudaStream_t stream);
+
+/* Counters since the plan was made (route counters of the paper's acceptance
+ * criteria: fast-path hits, refusals). */
+CCV3D_API ccv3d_status ccv3d_get_stats(ccv3d_plan_t plan, ccv3d_stats* stats);
+
+/* Synchronise the device, then return and clear the status recorded by the
+ * plan's kernels: CCV3D_OK, or CCV3D_ERR_TIMEOUT after a bounded wait ran out.
+ * CCV3D_ERR_CUDA when the device reports an error. */
+CCV3D_API ccv3d_status ccv3d_get_status(ccv3d_plan_t plan);
+
+/* Free the plan and its device status block.  NULL is ignored. */
+CCV3D_API void ccv3d_destroy(ccv3d_plan_t plan);
+
+/* Static description of a status code. */
+CCV3D_API const char* ccv3d_strerror(ccv3d_status status);
+
+/* Bytes of output and new_cache for a plan (sizes for the caller's
+ * allocation).  Any pointer may be NULL. */
+CCV3D_API ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t plan, size_t* out_bytes,
+                              size_t* new_cache_bytes, int* new_cache_frames);
+
+/* Self-test of the bounded device wait: launches one block that waits on an
+ * mbarrier nothing will complete, with a limit of `limit_ns` nanoseconds.
+ * Returns CCV3D_ERR_TIMEOUT (the expected outcome: the wait gave up and
+ * reported it, and the context stays usable), CCV3D_OK if the wait completed
+ * (a defect), or CCV3D_ERR_CUDA. */
+CCV3D_API ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CCV3D_H */

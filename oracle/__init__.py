@@ -73,6 +73,8 @@ def _bind(lib):
                                   ctypes.POINTER(ctypes.c_longlong),
                                   ctypes.c_longlong, dp]
     lib.oracle_tap_scan.argtypes = [P, ip, ip, ip, ip, ip]
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = ctypes.c_int
     for f in (lib.oracle_shape, lib.oracle_forward, lib.oracle_points,
               lib.oracle_tap_scan):
         f.restype = ctypes.c_int
@@ -176,6 +178,11 @@ def _check(p, x, cache, w, bias):
         raise ValueError(f"w shape {w.shape}")
     if bias is not None and bias.shape != (p.Cout,):
         raise ValueError("bias shape")
+
+
+def threads(lib=None) -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int((lib or load()).oracle_threads())
 
 
 def metrics(got, ref):

@@ -261,3 +261,15 @@ int oracle_tap_scan(const oracle_params* p, int* T_o_out, int* delta, int* o_l,
     }
     return 0;
 }
+
+/* Threads an OpenMP region of this library uses (1 without OpenMP). */
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

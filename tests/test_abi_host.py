@@ -1,0 +1,164 @@
+"""Host-side checks of libccv3d (no GPU needed): exported symbols, the
+planner against the oracle's brute-force tap scan, validation and error codes."""
+import itertools
+import os
+import re
+import subprocess
+
+import pytest
+
+import oracle
+from causal_conv3d_video_b200 import ccv3d, workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    hdr = open(os.path.join(ROOT, "include", "ccv3d.h")).read()
+    return set(re.findall(r"CCV3D_API\s+[\w\s\*]*?\b(ccv3d_\w+)\s*\(", hdr))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_symbols()
+    assert declared == set(ccv3d.EXPORTED)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", ccv3d.LIB_PATH]).decode()
+    exported = set(re.findall(r"\bT (ccv3d_\w+)", out))
+    assert declared <= exported, declared - exported
+    for name in declared:
+        assert hasattr(ccv3d.lib, name)
+
+
+def test_no_oracle_in_product():
+    # the product library must not link or name the oracle
+    out = subprocess.check_output(["nm", "-D", ccv3d.LIB_PATH]).decode()
+    assert "oracle" not in out
+    deps = subprocess.check_output(["ldd", ccv3d.LIB_PATH]).decode()
+    assert "oracle" not in deps
+
+
+def _plan(**kw):
+    return ccv3d.ccv3d_plan(ccv3d.make_desc(**kw))
+
+
+@pytest.mark.parametrize("d_t", [1, 2, 3])
+def test_planner_matches_oracle_scan_exhaustive(d_t):
+    """Intervals of the closed forms == brute-force scan, bit for bit."""
+    for cl, T_x, pb in itertools.product(range(0, 7), range(1, 7), range(0, 7)):
+        kw = dict(N=1, Cin=16, Cout=16, H=4, W=4, T_x=T_x, cache_len=cl,
+                  dilation=(d_t, 1, 1), pad_t_base=pb)
+        op = oracle.params(1, 16, 16, 4, 4, T_x, cl, dilation=(d_t, 1, 1), pad_t_base=pb)
+        T_o, H_o, W_o, keep = oracle.shape(op)
+        if T_o <= 0:
+            with pytest.raises(ccv3d.CCV3DError) as e:
+                _plan(**kw)
+            assert e.value.status == ccv3d.CCV3D_ERR_EMPTY_OUTPUT
+            continue
+        h = _plan(**kw)
+        try:
+            iv = ccv3d.ccv3d_plan_intervals(h)
+            T_s, delta, o_l, o_h, active = oracle.tap_scan(op)
+            assert (iv["T_o"], iv["H_o"], iv["W_o"]) == (T_o, H_o, W_o)
+            assert iv["delta"] == delta
+            assert iv["o_l"] == o_l and iv["o_h"] == o_h, (cl, T_x, pb, iv, o_l, o_h)
+            assert ccv3d.ccv3d_plan_sizes(h)["new_cache_frames"] == keep
+        finally:
+            ccv3d.ccv3d_destroy(h)
+
+
+@pytest.mark.parametrize("name", sorted(workloads.WORKLOADS))
+def test_planner_shapes_match_oracle_on_workloads(name):
+    c = workloads.WORKLOADS[name]
+    op = oracle.params(c.N, c.Cin, c.Cout, c.H, c.W, c.T_x, c.cache_len, kt=c.kt,
+                       kh=c.kh, kw=c.kw, pad_t_base=c.pad_t_base, cache_keep=c.cache_keep,
+                       stride=c.stride, pad=c.pad, dilation=c.dilation)
+    plan = ccv3d.Plan(ccv3d.desc_for(c))
+    T_o, H_o, W_o, keep = oracle.shape(op)
+    _, delta, o_l, o_h, _ = oracle.tap_scan(op)
+    iv = plan.intervals
+    assert (iv["T_o"], iv["H_o"], iv["W_o"]) == (T_o, H_o, W_o)
+    assert (iv["delta"], iv["o_l"], iv["o_h"]) == (delta, o_l, o_h)
+    assert plan.sizes["new_cache_frames"] == keep
+    # bf16 workloads take the tensor-core path; fp32 the SIMT path
+    assert plan.path["tc"] == (c.dtype == "bf16")
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kt=2), ccv3d.CCV3D_ERR_UNSUPPORTED),
+    (dict(stride_t=2), ccv3d.CCV3D_ERR_UNSUPPORTED),
+    (dict(groups=2), ccv3d.CCV3D_ERR_UNSUPPORTED),
+    (dict(Cin=0), ccv3d.CCV3D_ERR_INVALID),
+    (dict(T_x=0), ccv3d.CCV3D_ERR_INVALID),
+    (dict(cache_len=-1), ccv3d.CCV3D_ERR_INVALID),
+    (dict(stride=(0, 1)), ccv3d.CCV3D_ERR_INVALID),
+    (dict(N=0), ccv3d.CCV3D_ERR_EMPTY_OUTPUT),
+    (dict(H=1, pad=(0, 1)), ccv3d.CCV3D_ERR_EMPTY_OUTPUT),
+    (dict(pad_t_base=0, cache_len=0, T_x=1), ccv3d.CCV3D_ERR_EMPTY_OUTPUT),
+])
+def test_plan_refusals(kw, status):
+    base = dict(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2)
+    base.update(kw)
+    with pytest.raises(ccv3d.CCV3DError) as e:
+        _plan(**base)
+    assert e.value.status == status
+
+
+def test_bad_dtype_refused():
+    d = ccv3d.make_desc(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2)
+    d.dtype = 7
+    with pytest.raises(ccv3d.CCV3DError) as e:
+        ccv3d.ccv3d_plan(d)
+    assert e.value.status == ccv3d.CCV3D_ERR_UNSUPPORTED
+
+
+def test_null_arguments():
+    assert ccv3d.lib.ccv3d_plan(None, None) == ccv3d.CCV3D_ERR_INVALID
+    assert ccv3d.lib.ccv3d_plan_intervals(None, None, None, None, None, None, None) == \
+        ccv3d.CCV3D_ERR_INVALID
+    assert ccv3d.ccv3d_plan_path(None)["tc"] is False
+    ccv3d.ccv3d_destroy(None)  # ignored
+    for s in range(8):
+        assert ccv3d.ccv3d_strerror(s)
+
+
+def test_forward_validation_order_without_gpu():
+    """Argument checks run before any device work; with no GPU a well-formed
+    call is refused with CCV3D_ERR_CUDA, never executed on the host."""
+    plan = ccv3d.Plan(ccv3d.make_desc(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2))
+    A = 1 << 20
+    args = dict(x=A, cache=2 * A, w=3 * A, bias=4 * A, out=5 * A, new_cache=6 * A)
+
+    def call(**over):
+        a = dict(args)
+        a.update(over)
+        st = dict(stride=plan.stride, pad=plan.pad, dilation=plan.dilation)
+        st.update({k: over.pop(k) for k in list(over) if k in st})
+        a = {k: v for k, v in a.items() if k not in st}
+        return ccv3d.ccv3d_forward(plan.handle, a["x"], a["cache"], a["w"], a["bias"],
+                                   a["out"], a["new_cache"], st["stride"], st["pad"],
+                                   st["dilation"], stream=0, check=False)
+
+    assert call(stride=(2, 1)) == ccv3d.CCV3D_ERR_INVALID
+    assert call(dilation=(2, 1, 1)) == ccv3d.CCV3D_ERR_INVALID
+    assert call(x=None) == ccv3d.CCV3D_ERR_INVALID
+    assert call(cache=None) == ccv3d.CCV3D_ERR_INVALID
+    assert call(bias=None) == ccv3d.CCV3D_ERR_INVALID
+    assert call(new_cache=None) == ccv3d.CCV3D_ERR_INVALID
+    assert call(x=A + 8) == ccv3d.CCV3D_ERR_ALIGNMENT
+    assert call(new_cache=A + 64) == ccv3d.CCV3D_ERR_ALIAS      # inside x
+    assert call(out=2 * A + 16) == ccv3d.CCV3D_ERR_ALIAS        # inside cache
+    st = call()
+    import torch
+    if not torch.cuda.is_available():
+        assert st == ccv3d.CCV3D_ERR_CUDA
+    stats = plan.stats()
+    assert stats["calls"] == 0 and stats["errors"] >= 9
+    assert stats["workspace_bytes"] == 0
+
+
+def test_tile_choice_on_bottleneck():
+    plan = ccv3d.Plan(ccv3d.desc_for(workloads.C2))
+    assert plan.path == {"tc": True, "tile_m": 128, "tile_n": 192}
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C3)).path["tile_n"] == 96
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C4_TIME)).path["tile_n"] == 256
+    thin = ccv3d.Plan(ccv3d.make_desc(N=1, Cin=3, Cout=16, H=8, W=8, T_x=1, cache_len=0))
+    assert thin.path["tc"] is False

@@ -1,0 +1,171 @@
+"""GPU parity: the C-ABI call against the FP64 oracle on the same seeded inputs.
+
+Small signatures are compared element by element over the whole output (they
+span several 128-pixel tiles, several Cout tiles and ragged tails); the
+decoder-sized workloads are compared at sampled outputs the oracle evaluates
+one by one, with new_cache compared in full and the whole output checked for
+NaN/Inf.  Tolerance: max|gpu - oracle| <= 2e-2 rms(oracle) for bf16 and
+1e-4 rms(oracle) for fp32.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_conv3d_video_b200 import ccv3d, workloads
+from causal_conv3d_video_b200.workloads import Conv
+from parity_util import (GpuCall, assert_close, expected_new_cache, inputs_for,
+                         oracle_params, sample_indices)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # multi-tile, ragged 20x37 map, every cache length
+    Conv("s64_c0", 64, 64, 20, 37, T_x=1, cache_len=0),
+    Conv("s64_c1", 64, 64, 20, 37, T_x=1, cache_len=1),
+    Conv("s64_c2", 64, 64, 20, 37, T_x=1, cache_len=2),
+    Conv("s64_c2_t3", 64, 64, 20, 37, T_x=3, cache_len=2),
+    Conv("s64_c0_t3", 64, 64, 20, 37, T_x=3, cache_len=0),
+    # Cout tiles: 384 -> 2 x 192, 768 -> 3 x 256, 400 -> 2 x 208 (ragged N)
+    Conv("s128to384", 128, 384, 12, 20, T_x=1, cache_len=2),
+    Conv("s64to400", 64, 400, 9, 15, T_x=1, cache_len=1),
+    Conv("s3x1x1_384to768", 384, 768, 10, 16, T_x=1, cache_len=2, kh=1, kw=1, pad=(0, 0)),
+    # K blocks: Cin 96 (BK 32), 48 and 16 (BK 16), Cout 96 / 48
+    Conv("s96", 96, 96, 24, 40, T_x=4, cache_len=2, sigma_b=0.1),
+    Conv("s192to96", 192, 96, 16, 24, T_x=2, cache_len=1, sigma_b=0.1),
+    Conv("s48to48", 48, 48, 11, 13, T_x=2, cache_len=2),
+    Conv("s16to384", 16, 384, 18, 32, T_x=1, cache_len=0),
+    # stride 2, dilations, odd sizes, batch 2
+    Conv("s_stride2", 64, 64, 36, 64, T_x=1, cache_len=2, stride=(2, 2)),
+    Conv("s_stride2_odd", 32, 32, 17, 23, T_x=2, cache_len=1, stride=(2, 2)),
+    Conv("s_dt2_c4", 64, 64, 18, 32, T_x=1, cache_len=4, dilation=(2, 1, 1)),
+    Conv("s_dt2_c1_t3", 64, 64, 18, 32, T_x=3, cache_len=1, dilation=(2, 1, 1)),
+    Conv("s_dil_hw2", 32, 32, 19, 27, T_x=1, cache_len=2, pad=(2, 2), dilation=(1, 2, 2)),
+    Conv("s_odd", 64, 64, 23, 41, T_x=1, cache_len=2),
+    Conv("s_batch2", 32, 48, 10, 12, T_x=2, cache_len=2, N=2),
+    # |C| > p_l^base (negative p_l: oldest cached frame dropped)
+    Conv("s_crop", 32, 32, 10, 12, T_x=1, cache_len=3),
+    # p_l^base = 4 > d_t(kt-1): leading output frames have no active tap (bias only)
+    Conv("s_biasonly", 32, 32, 10, 12, T_x=2, cache_len=0, pad_t_base=4, cache_keep=2),
+    # no bias, asymmetric pad/kernel
+    Conv("s_nobias", 64, 32, 14, 30, T_x=2, cache_len=2, has_bias=False),
+    Conv("s_k3x1x3", 32, 32, 14, 30, T_x=1, cache_len=2, kh=1, kw=3, pad=(0, 1)),
+]
+
+
+def _run_small(c, force_simt=False):
+    inp = inputs_for(c)
+    call = GpuCall(c, inp, force_simt=force_simt).run()
+    torch.cuda.synchronize()
+    ref, ref_nc = oracle.forward(oracle_params(c), inp["x"], inp["cache"], inp["w"],
+                                 inp["bias"])
+    got = call.out_f64()
+    assert got.shape == ref.shape
+    m = assert_close(got, ref, c.dtype, c.name)
+    nc = call.nc_f64()
+    if ref_nc.size:
+        assert np.array_equal(nc, ref_nc), c.name
+    assert call.guards_intact(), c.name
+    assert call.plan.status() == ccv3d.CCV3D_OK
+    return call, m
+
+
+def test_config1_fp32_exact_workload():
+    call, m = _run_small(workloads.C1)
+    assert call.plan.path["tc"] is False
+    assert call.plan.stats()["simt_path"] == 1
+
+
+@pytest.mark.parametrize("c", SMALL, ids=lambda c: c.name)
+def test_small_tensor_core(c):
+    call, _ = _run_small(c)
+    assert call.plan.path["tc"] is True
+    st = call.plan.stats()
+    assert st["calls"] == 1 and st["tc_path"] == 1 and st["errors"] == 0
+
+
+@pytest.mark.parametrize("c", SMALL[:4] + SMALL[12:15] + SMALL[19:21], ids=lambda c: c.name)
+def test_small_simt_bf16(c):
+    call, _ = _run_small(c, force_simt=True)
+    assert call.plan.path["tc"] is False
+
+
+@pytest.mark.parametrize("c", [
+    Conv("f32_s2", 8, 12, 13, 17, T_x=2, cache_len=1, stride=(2, 2), dtype="fp32"),
+    Conv("f32_dt2", 5, 7, 9, 11, T_x=1, cache_len=4, dilation=(2, 1, 1), dtype="fp32"),
+    Conv("f32_3x1x1", 24, 40, 6, 10, T_x=3, cache_len=0, kh=1, kw=1, pad=(0, 0), dtype="fp32"),
+    Conv("bf16_thin_cin3", 3, 16, 12, 12, T_x=2, cache_len=2),
+], ids=lambda c: c.name)
+def test_small_simt_other(c):
+    call, _ = _run_small(c)
+    assert call.plan.path["tc"] is False
+
+
+FULL = [n for n, c in workloads.WORKLOADS.items() if c.dtype == "bf16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    c = workloads.WORKLOADS[name]
+    inp = inputs_for(c)
+    call = GpuCall(c, inp).run()
+    torch.cuda.synchronize()
+    assert call.plan.path["tc"] is True
+    out = call.out
+    assert bool(torch.isfinite(out.float()).all())
+    idx = sample_indices(tuple(out.shape), call.plan, n_random=2000)
+    ref = oracle.points(oracle_params(c), inp["x"], inp["cache"], inp["w"], inp["bias"], idx)
+    got = out[tuple(torch.from_numpy(idx.T).cuda())].double().cpu().numpy()
+    assert_close(got, ref, c.dtype, name)
+    want_nc = expected_new_cache(c, inp)
+    assert np.array_equal(call.nc_f64(), want_nc)
+    assert call.guards_intact()
+    assert call.plan.status() == ccv3d.CCV3D_OK
+
+
+def test_repeat_calls_identical_and_counters():
+    c = SMALL[3]
+    inp = inputs_for(c)
+    call = GpuCall(c, inp).run()
+    first = call.out.clone()
+    for _ in range(4):
+        call.run()
+    torch.cuda.synchronize()
+    assert torch.equal(first, call.out)  # fixed reduction order: deterministic
+    st = call.plan.stats()
+    assert st["calls"] == 5 and st["tc_path"] == 5
+
+
+def test_other_stream():
+    c = SMALL[5]
+    inp = inputs_for(c)
+    ref_call = GpuCall(c, inp).run()
+    s = torch.cuda.Stream()
+    call = GpuCall(c, inp)
+    with torch.cuda.stream(s):
+        call.run(stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(ref_call.out, call.out)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    st = ccv3d.ccv3d_selftest_wait_timeout(50_000_000)  # 50 ms, nothing arrives
+    assert st == ccv3d.CCV3D_ERR_TIMEOUT
+    _run_small(SMALL[0])  # the context is still usable
+
+
+def test_forward_refusals_on_device():
+    c = SMALL[2]
+    inp = inputs_for(c)
+    call = GpuCall(c, inp)
+    p = call.plan
+    # new_cache aliasing x (ping-pong misuse)
+    rc = ccv3d.ccv3d_forward(p.handle, call.x, call.cache, call.w, call.bias, call.out,
+                             call.x, p.stride, p.pad, p.dilation, check=False)
+    assert rc == ccv3d.CCV3D_ERR_ALIAS
+    # misaligned x
+    rc = ccv3d.ccv3d_forward(p.handle, call.x.data_ptr() + 2, call.cache, call.w, call.bias,
+                             call.out, call.nc, p.stride, p.pad, p.dilation, check=False)
+    assert rc == ccv3d.CCV3D_ERR_ALIGNMENT
+    assert p.stats()["errors"] == 2 and p.stats()["calls"] == 0
