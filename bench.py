@@ -114,6 +114,11 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # NVML start-up can stall the driver for a moment: let the first
+            # sample arrive before the timed region begins.
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 15 and self.proc.poll() is None:
+                time.sleep(0.02)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
