@@ -21,6 +21,7 @@
 #include "ccv3d.h"
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
+#include "conv_tc2.cuh"
 #include "params.h"
 
 using namespace ccv3d;
@@ -30,7 +31,8 @@ struct ccv3d_plan_s {
     int T_o, H_o, W_o, z_len, p_l, keep;
     int delta[kMaxTaps], o_l[kMaxTaps], o_h[kMaxTaps];
     int path_tc;  // 1: tcgen05 implicit GEMM, 0: SIMT
-    int BK, BN, box_h, box_w, tiles_x, tiles_y, tiles_n, stages, tmem_cols;
+    int BK, BN, n_sub, box_h, box_w, tiles_x, tiles_y, tiles_n, stages, tmem_cols;
+    int pair;  // 1: CTA-pair kernel (M = 256 per pair), 0: one CTA per 128-row tile
     size_t smem_bytes;
     int device;
     int* d_status;
@@ -96,18 +98,29 @@ ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
     return CCV3D_OK;
 }
 
-constexpr size_t kSmemBudget = 200 * 1024;
+constexpr size_t kSmemBudget = 225 * 1024;
 
 template <int BK>
-int pick_stages(int bn) {
-    int s = 8;
-    while (s > 2 && tc_smem_bytes<BK>(bn, s) > kSmemBudget) --s;
+size_t smem_for(int pair, int bn, int stages) {
+    return pair ? tc2_smem_bytes<BK>(bn, stages) : tc_smem_bytes<BK>(bn, stages);
+}
+
+template <int BK>
+int pick_stages(int pair, int bn, int want) {
+    int s = want > 0 ? std::min(want, 12) : 8;
+    while (s > 2 && smem_for<BK>(pair, bn, s) > kSmemBudget) --s;
     return s;
 }
 
 bool force_simt() {
     const char* e = std::getenv("CCV3D_FORCE_PATH");
     return e != nullptr && std::strcmp(e, "simt") == 0;
+}
+
+// Tiling overrides for tuning sweeps (0 = the planner's choice).
+int env_int(const char* name) {
+    const char* e = std::getenv(name);
+    return e != nullptr ? std::atoi(e) : 0;
 }
 
 // Kernel choice and tiling.
@@ -118,9 +131,11 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     if (!tc_ok) return;
     // spatial box of 128 output pixels: fewest tiles, then widest rows
     int best_w = 0, best_tiles = 0;
+    const int want_w = env_int("CCV3D_BOX_W");
     for (int bw = 128; bw >= 8; bw /= 2) {
         const int bh = kTileM / bw;
         if (bw * d.stride_w > 256 || bh * d.stride_h > 256) continue;
+        if (want_w > 0 && bw != want_w) continue;
         const int tiles = ceil_div(p->H_o, bh) * ceil_div(p->W_o, bw);
         if (best_w == 0 || tiles < best_tiles) {
             best_w = bw;
@@ -132,13 +147,30 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->box_h = kTileM / best_w;
     p->tiles_x = ceil_div(p->W_o, p->box_w);
     p->tiles_y = ceil_div(p->H_o, p->box_h);
-    p->tiles_n = ceil_div(d.Cout, 256);
+    // Cout tile: up to 256 columns per MMA, up to 2 MMAs (512 TMEM columns).
+    // One CTA covers up to 384 output channels so that each A box is loaded
+    // once for all of them (measured best on the 384-channel decoder calls).
+    const int want_n = env_int("CCV3D_TILE_N");
+    const int max_n = (want_n >= 16 && want_n <= 512) ? want_n : 384;
+    p->tiles_n = ceil_div(d.Cout, max_n);
     p->BN = ((ceil_div(d.Cout, p->tiles_n) + 15) / 16) * 16;
+    p->n_sub = p->BN > 256 ? 2 : 1;
+    if (p->n_sub == 2 && p->BN % 32 != 0) p->BN = ((p->BN + 31) / 32) * 32;
     p->BK = d.Cin % 64 == 0 ? 64 : (d.Cin % 32 == 0 ? 32 : 16);
+    // CTA pairs whenever every pair MMA has N >= 32 (16 weight rows per CTA)
+    const char* pe = std::getenv("CCV3D_PAIR");
+    p->pair = (p->BN / p->n_sub) >= 32 ? 1 : 0;
+    if (pe != nullptr) p->pair = std::atoi(pe) != 0 && (p->BN / p->n_sub) >= 32;
+    // Short reductions (few k-blocks per tile) are dominated by each tile's
+    // fill and epilogue: keep the ring small enough for 3 CTAs per SM so one
+    // CTA's epilogue overlaps its neighbours' main loops.
+    const int kblocks = 3 * d.kh * d.kw * ceil_div(d.Cin, p->BK);
+    int want_s = env_int("CCV3D_STAGES");
+    if (want_s == 0 && kblocks <= 96) want_s = 4;
     switch (p->BK) {
-        case 64: p->stages = pick_stages<64>(p->BN); p->smem_bytes = tc_smem_bytes<64>(p->BN, p->stages); break;
-        case 32: p->stages = pick_stages<32>(p->BN); p->smem_bytes = tc_smem_bytes<32>(p->BN, p->stages); break;
-        default: p->stages = pick_stages<16>(p->BN); p->smem_bytes = tc_smem_bytes<16>(p->BN, p->stages); break;
+        case 64: p->stages = pick_stages<64>(p->pair, p->BN, want_s); p->smem_bytes = smem_for<64>(p->pair, p->BN, p->stages); break;
+        case 32: p->stages = pick_stages<32>(p->pair, p->BN, want_s); p->smem_bytes = smem_for<32>(p->pair, p->BN, p->stages); break;
+        default: p->stages = pick_stages<16>(p->pair, p->BN, want_s); p->smem_bytes = smem_for<16>(p->pair, p->BN, p->stages); break;
     }
     p->tmem_cols = 32;
     while (p->tmem_cols < p->BN) p->tmem_cols *= 2;
@@ -179,7 +211,9 @@ ccv3d_status encode_w(CUtensorMap* m, const void* base, const ccv3d_desc& d,
     const int taps = d.kt * d.kh * d.kw;
     const cuuint64_t dims[3] = {(cuuint64_t)d.Cin, (cuuint64_t)taps, (cuuint64_t)d.Cout};
     const cuuint64_t strides[2] = {(cuuint64_t)d.Cin * 2, (cuuint64_t)taps * d.Cin * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)p->BK, 1, (cuuint32_t)p->BN};
+    // rows per load: one MMA's N, or half of it when a CTA pair splits the MMA
+    const int rows = (p->BN / p->n_sub) / (p->pair ? 2 : 1);
+    const cuuint32_t box[3] = {(cuuint32_t)p->BK, 1, (cuuint32_t)rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -217,16 +251,23 @@ Taps make_taps(const ccv3d_plan_s* p) {
 }
 
 template <int BK>
-cudaError_t launch_tc(const TcParams& prm, int grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_tc(const TcParams& prm, int pair, int grid, size_t smem, cudaStream_t s) {
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
         attr = cudaFuncSetAttribute(conv_tc_kernel<BK>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)(227 * 1024));
+        if (attr == cudaSuccess)
+            attr = cudaFuncSetAttribute(conv_tc2_kernel<BK>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)(227 * 1024));
     });
     if (attr != cudaSuccess) return attr;
-    conv_tc_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
+    if (pair)
+        conv_tc2_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
+    else
+        conv_tc_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
     return cudaGetLastError();
 }
 
@@ -252,16 +293,24 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     prm.cache_len = d.cache_len; prm.T_x = d.T_x;
     prm.box_h = p->box_h; prm.box_w = p->box_w;
     prm.tiles_x = p->tiles_x; prm.tiles_y = p->tiles_y; prm.tiles_n = p->tiles_n;
-    prm.BN = p->BN; prm.n_cb = ceil_div(d.Cin, p->BK); prm.stages = p->stages;
+    prm.BN = p->BN; prm.n_sub = p->n_sub; prm.n_cb = ceil_div(d.Cin, p->BK);
+    prm.stages = p->stages;
     prm.tmem_cols = p->tmem_cols;
     prm.wait_limit_ns = kWaitLimitNs;
-    const long long grid = (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
+    prm.pairs_per_frame = (p->tiles_x * p->tiles_y + 1) / 2;
+    const long long grid =
+        p->pair ? 2LL * d.N * p->T_o * prm.pairs_per_frame * p->tiles_n
+                : (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
     if (grid > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
+    // spread the K-start offsets over one wave of concurrently running tiles
+    const long long units = p->pair ? grid / 2 : grid;
+    const long long wave = p->pair ? 74 : 148;
+    prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
     cudaError_t e;
     switch (p->BK) {
-        case 64: e = launch_tc<64>(prm, (int)grid, p->smem_bytes, stream); break;
-        case 32: e = launch_tc<32>(prm, (int)grid, p->smem_bytes, stream); break;
-        default: e = launch_tc<16>(prm, (int)grid, p->smem_bytes, stream); break;
+        case 64: e = launch_tc<64>(prm, p->pair, (int)grid, p->smem_bytes, stream); break;
+        case 32: e = launch_tc<32>(prm, p->pair, (int)grid, p->smem_bytes, stream); break;
+        default: e = launch_tc<16>(prm, p->pair, (int)grid, p->smem_bytes, stream); break;
     }
     return e == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
 }
@@ -363,7 +412,7 @@ ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t p, int* T_o, int* H_o, int* W_o,
 
 int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
     if (p == nullptr) return -1;
-    if (tile_m) *tile_m = p->path_tc ? kTileM : 0;
+    if (tile_m) *tile_m = p->path_tc ? kTileM * (p->pair ? 2 : 1) : 0;
     if (tile_n) *tile_n = p->path_tc ? p->BN : 0;
     return p->path_tc;
 }

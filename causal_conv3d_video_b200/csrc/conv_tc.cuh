@@ -50,8 +50,10 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int stages = p.stages;
-    const int BN = p.BN;
+    const int BN = p.BN;              // Cout columns of this CTA's tile
+    const int BNs = BN / p.n_sub;     // columns per MMA (<= 256)
     const int kB = BN * kRow;
+    const int kBs = BNs * kRow;
     uint8_t* sA = smem;
     uint8_t* sB = smem + (size_t)stages * kA;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kB);
@@ -112,11 +114,27 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
-            int it = 0;
-            bool ok = true;
+            // The reduction is walked from a per-tile starting point spread
+            // over [0, iters): CTAs running at the same time then read
+            // different weight rows instead of all hitting the same L2 lines.
+            int act[kMaxTaps], n_act = 0;
+            for (int k = 0; k < p.taps.kt; ++k)
+                if (o >= p.taps.o_l[k] && o < p.taps.o_h[k]) act[n_act++] = k;
+            const int per_tap = p.kh * p.kw * p.n_cb;
+            const int rot = iters > 0 ? (int)(((long long)blockIdx.x * iters) / p.rot_div) % iters : 0;
             const uint32_t stage_bytes = (uint32_t)(kA + kB);
-            for (int k = 0; k < p.taps.kt && ok; ++k) {
-                if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
+            for (int it = 0; it < iters; ++it) {
+                const int st = it % stages;
+                if (it >= stages &&
+                    !mbar_wait(smem_u32(&empty_bar[st]), ((it / stages) & 1) ^ 1, p.status,
+                               p.wait_limit_ns))
+                    break;
+                int kb = it + rot;  // k-block of the reduction loaded at step `it`
+                if (kb >= iters) kb -= iters;
+                const int k = act[kb / per_tap];
+                const int cb = kb % p.n_cb;
+                const int rs = (kb / p.n_cb) % (p.kh * p.kw);
+                const int r = rs / p.kw, s = rs % p.kw;
                 const int t = o + p.taps.delta[k];  // frame of Z
                 const CUtensorMap* src;
                 int f;
@@ -127,34 +145,22 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
                     src = &p.tmap_x;
                     f = n * p.T_x + (t - p.cache_len);
                 }
-                for (int r = 0; r < p.kh && ok; ++r) {
-                    const int y0 = ty * p.box_h * p.s_h + r * p.d_h - p.p_h;
-                    for (int s = 0; s < p.kw && ok; ++s) {
-                        const int x0 = tx * p.box_w * p.s_w + s * p.d_w - p.p_w;
-                        const int wrow = (k * p.kh + r) * p.kw + s;
-                        for (int cb = 0; cb < p.n_cb; ++cb, ++it) {
-                            const int st = it % stages;
-                            if (it >= stages &&
-                                !mbar_wait(smem_u32(&empty_bar[st]), ((it / stages) & 1) ^ 1,
-                                           p.status, p.wait_limit_ns)) {
-                                ok = false;
-                                break;
-                            }
-                            const uint32_t fb = smem_u32(&full_bar[st]);
-                            mbar_arrive_expect_tx(fb, stage_bytes);
-                            tma_load_4d(smem_u32(sA + (size_t)st * kA), src, fb, cb * BK, x0,
-                                        y0, f);
-                            tma_load_3d(smem_u32(sB + (size_t)st * kB), &p.tmap_w, fb,
-                                        cb * BK, wrow, n_tile * BN);
-                        }
-                    }
-                }
+                const int y0 = ty * p.box_h * p.s_h + r * p.d_h - p.p_h;
+                const int x0 = tx * p.box_w * p.s_w + s * p.d_w - p.p_w;
+                const int wrow = (k * p.kh + r) * p.kw + s;
+                const uint32_t fb = smem_u32(&full_bar[st]);
+                mbar_arrive_expect_tx(fb, stage_bytes);
+                tma_load_4d(smem_u32(sA + (size_t)st * kA), src, fb, cb * BK, x0,
+                            y0, f);
+                for (int j = 0; j < p.n_sub; ++j)
+                    tma_load_3d(smem_u32(sB + (size_t)st * kB + (size_t)j * kBs),
+                                &p.tmap_w, fb, cb * BK, wrow, n_tile * BN + j * BNs);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------- MMA issuer
-            const uint32_t idesc = idesc_bf16_m128((uint32_t)BN);
+            const uint32_t idesc = idesc_bf16_m128((uint32_t)BNs);
             for (int it = 0; it < iters; ++it) {
                 const int st = it % stages;
                 if (!mbar_wait(smem_u32(&full_bar[st]), (it / stages) & 1, p.status,
@@ -163,11 +169,14 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
                 tc_fence_after();
                 const uint64_t a_desc = smem_desc_kmajor(smem_u32(sA + (size_t)st * kA), kRow);
                 const uint64_t b_desc = smem_desc_kmajor(smem_u32(sB + (size_t)st * kB), kRow);
+                for (int j = 0; j < p.n_sub; ++j) {
+                    const uint64_t bj = b_desc + (uint64_t)((j * kBs) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    // +32 bytes of K per step inside the swizzle span
-                    umma_bf16(tmem_base, a_desc + 2u * kk, b_desc + 2u * kk, idesc,
-                              (it | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        // +32 bytes of K per step inside the swizzle span
+                        umma_bf16(tmem_base + (uint32_t)(j * BNs), a_desc + 2u * kk,
+                                  bj + 2u * kk, idesc, (it | kk) != 0 ? 1u : 0u);
+                }
                 umma_commit(smem_u32(&empty_bar[st]));
             }
             umma_commit(smem_u32(acc_bar));

@@ -1,0 +1,236 @@
+// conv_tc2.cuh -- the implicit-GEMM Conv3D on CTA pairs (tcgen05 cta_group::2).
+//
+// Same GEMM view as conv_tc.cuh (rows = output pixels of one output frame,
+// columns = Cout, reduction over active taps x kh x kw x Cin), but a cluster
+// of two CTAs computes a 256 x BN tile with M=256 pair MMAs:
+//   * each CTA loads its own 128-pixel A box (two neighbouring boxes of the
+//     same output frame, so both CTAs walk the same active taps) and HALF of
+//     the weight rows of every MMA; the even CTA issues the MMAs, which read
+//     A and B from both CTAs' shared memory;
+//   * both CTAs' TMA loads complete on the even CTA's "full" barrier (the
+//     even producer posts the byte count for the pair), and the even CTA's
+//     tcgen05.commit releases the stage on both CTAs' "empty" barriers;
+//   * each CTA holds its 128 accumulator rows in its own TMEM and runs its own
+//     epilogue (bias, bf16, store) and its slice of the new_cache copy.
+// Per SM this halves the weight bytes pulled from L2 per FLOP, the operand
+// that dominates on the wide-Cout decoder signatures.  No load is
+// multicast.  All waits are bounded.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "cache_copy.cuh"
+#include "conv_tc.cuh"
+#include "params.h"
+#include "ptx.cuh"
+
+namespace ccv3d {
+
+template <int BK>
+__host__ __device__ constexpr size_t tc2_smem_bytes(int bn, int stages) {
+    // per CTA: A box (128 rows) + half of the BN weight rows per stage
+    return 1024 + (size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes) +
+           (size_t)(2 * stages + 1) * 8 + 16 + (size_t)bn * 4;
+}
+
+template <int BK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+conv_tc2_kernel(const __grid_constant__ TcParams p) {
+    constexpr int kRow = TcSmem<BK>::kRowBytes;
+    constexpr int kA = TcSmem<BK>::kABytes;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int stages = p.stages;
+    const int BN = p.BN;            // accumulator columns of the pair tile
+    const int BNs = BN / p.n_sub;   // N of one pair MMA (<= 256)
+    const int hB = BNs / 2;         // weight rows per CTA per MMA
+    const int kBc = (BN / 2) * kRow;  // weight bytes per CTA per stage
+    const int kBh = hB * kRow;
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + (size_t)stages * kA;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kBc);
+    uint64_t* empty_bar = full_bar + stages;
+    uint64_t* acc_bar = empty_bar + stages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+    float* bias_s = reinterpret_cast<float*>(tmem_slot + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    // ---- pair tile: (n, o, pair of boxes) x n_tile
+    const int pair = blockIdx.x >> 1;
+    const int n_tile = pair % p.tiles_n;
+    const int m_pair = pair / p.tiles_n;
+    const int ppf = p.pairs_per_frame;
+    const int frame = m_pair / ppf;
+    const int box = (m_pair % ppf) * 2 + (int)rank;
+    const int o = frame % p.T_o;
+    const int n = frame / p.T_o;
+    int tx = 0, ty = p.tiles_y;  // a box past the frame's last one stores nothing
+    if (box < p.tiles_x * p.tiles_y) {
+        tx = box % p.tiles_x;
+        ty = box / p.tiles_x;
+    }
+
+    int n_active = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxTaps; ++k)
+        if (k < p.taps.kt && o >= p.taps.o_l[k] && o < p.taps.o_h[k]) ++n_active;
+    const int iters = n_active * p.kh * p.kw * p.n_cb;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        mbar_init(smem_u32(acc_bar), 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&p.tmap_x);
+        if (p.cache_len > 0) tma_prefetch_desc(&p.tmap_c);
+        tma_prefetch_desc(&p.tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+        tmem_relinquish_pair();
+    }
+    if (warp >= 2) {
+        for (int i = threadIdx.x - 64; i < BN; i += 128) {
+            const int co = n_tile * BN + i;
+            float b = 0.f;
+            if (p.bias != nullptr && co < p.Cout)
+                b = __bfloat162float(__ushort_as_bfloat16(p.bias[co]));
+            bias_s[i] = b;
+        }
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers initialised in both CTAs before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // --------------------------------- TMA producer (both CTAs)
+            // The reduction is walked from a per-tile starting point spread
+            // over [0, iters): CTAs running at the same time then read
+            // different weight rows instead of all hitting the same L2 lines.
+            int act[kMaxTaps], n_act = 0;
+            for (int k = 0; k < p.taps.kt; ++k)
+                if (o >= p.taps.o_l[k] && o < p.taps.o_h[k]) act[n_act++] = k;
+            const int per_tap = p.kh * p.kw * p.n_cb;
+            const int rot = iters > 0 ? (int)(((long long)pair * iters) / p.rot_div) % iters : 0;
+            const uint32_t pair_bytes = 2u * (uint32_t)(kA + kBc);
+            for (int it = 0; it < iters; ++it) {
+                const int st = it % stages;
+                if (it >= stages &&
+                    !mbar_wait(smem_u32(&empty_bar[st]), ((it / stages) & 1) ^ 1, p.status,
+                               p.wait_limit_ns))
+                    break;
+                int kb = it + rot;  // k-block of the reduction loaded at step `it`
+                if (kb >= iters) kb -= iters;
+                const int k = act[kb / per_tap];
+                const int cb = kb % p.n_cb;
+                const int rs = (kb / p.n_cb) % (p.kh * p.kw);
+                const int r = rs / p.kw, s = rs % p.kw;
+                const int t = o + p.taps.delta[k];  // frame of Z
+                const CUtensorMap* src;
+                int f;
+                if (t < p.cache_len) {
+                    src = &p.tmap_c;
+                    f = n * p.cache_len + t;
+                } else {
+                    src = &p.tmap_x;
+                    f = n * p.T_x + (t - p.cache_len);
+                }
+                const int y0 = ty * p.box_h * p.s_h + r * p.d_h - p.p_h;
+                const int x0 = tx * p.box_w * p.s_w + s * p.d_w - p.p_w;
+                const int wrow = (k * p.kh + r) * p.kw + s;
+                const uint32_t fb_local = smem_u32(&full_bar[st]);
+                if (leader) mbar_arrive_expect_tx(fb_local, pair_bytes);
+                const uint32_t fb = pair_leader_addr(fb_local);
+                tma_load_4d_pair(smem_u32(sA + (size_t)st * kA), src, fb, cb * BK,
+                                 x0, y0, f);
+                for (int j = 0; j < p.n_sub; ++j)
+                    tma_load_3d_pair(
+                        smem_u32(sB + (size_t)st * kBc + (size_t)j * kBh), &p.tmap_w,
+                        fb, cb * BK, wrow, n_tile * BN + j * BNs + (int)rank * hB);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------ MMA issuer (even CTA only)
+            const uint32_t idesc = idesc_bf16_m256((uint32_t)BNs);
+            for (int it = 0; it < iters; ++it) {
+                const int st = it % stages;
+                if (!mbar_wait(smem_u32(&full_bar[st]), (it / stages) & 1, p.status,
+                               p.wait_limit_ns))
+                    break;
+                tc_fence_after();
+                const uint64_t a_desc = smem_desc_kmajor(smem_u32(sA + (size_t)st * kA), kRow);
+                const uint64_t b_desc = smem_desc_kmajor(smem_u32(sB + (size_t)st * kBc), kRow);
+                for (int j = 0; j < p.n_sub; ++j) {
+                    const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16_pair(tmem_base + (uint32_t)(j * BNs), a_desc + 2u * kk,
+                                       bj + 2u * kk, idesc, (it | kk) != 0 ? 1u : 0u);
+                }
+                umma_commit_pair(smem_u32(&empty_bar[st]), (uint16_t)0x3);
+            }
+            umma_commit_pair(smem_u32(acc_bar), (uint16_t)0x3);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------- new_cache slice, then this CTA's epilogue
+        const int etid = threadIdx.x - 64;
+        copy_new_cache(p.copy, blockIdx.x, gridDim.x, etid, 128);
+
+        const bool ok = mbar_wait(smem_u32(acc_bar), 0, p.status, p.wait_limit_ns);
+        tc_fence_after();
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int y = ty * p.box_h + row / p.box_w;
+        const int x = tx * p.box_w + row % p.box_w;
+        const bool valid = ok && y < p.H_o && x < p.W_o;
+        uint16_t* orow = p.out + ((((long long)n * p.T_o + o) * p.H_o + y) * p.W_o + x) *
+                                     (long long)p.Cout;
+        const bool have_acc = iters > 0;
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+            tmem_ld_wait();
+            const int co = n_tile * BN + c0;
+            if (!valid || co >= p.Cout) continue;
+            uint32_t packed[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float a0 = (have_acc ? __uint_as_float(v[2 * j]) : 0.f) + bias_s[c0 + 2 * j];
+                const float a1 =
+                    (have_acc ? __uint_as_float(v[2 * j + 1]) : 0.f) + bias_s[c0 + 2 * j + 1];
+                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+                packed[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            if (co + 16 <= p.Cout) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + co);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (co + j < p.Cout)
+                        orow[co + j] = (uint16_t)(packed[j >> 1] >> ((j & 1) * 16));
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync();  // the peer's shared memory and barriers stay alive until both are done
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, (uint32_t)p.tmem_cols);
+    }
+}
+
+}  // namespace ccv3d

@@ -42,7 +42,9 @@ struct __align__(64) TcParams {
     int s_h, s_w, p_h, p_w, d_h, d_w;
     int cache_len, T_x;
     int box_h, box_w, tiles_x, tiles_y, tiles_n;
-    int BN, n_cb, stages, tmem_cols;
+    int BN, n_sub, n_cb, stages, tmem_cols;
+    int pairs_per_frame;     // CTA-pair kernel: ceil(tiles_x * tiles_y / 2)
+    int rot_div;             // tiles (or pairs) over which K-start offsets are spread
     uint64_t wait_limit_ns;
 };
 

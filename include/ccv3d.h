@@ -121,7 +121,8 @@ CCV3D_API ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t plan, int* T_o, int* H_
                                   int o_h[CCV3D_MAX_KT]);
 
 /* 1 when the plan runs the tcgen05 tensor-core kernel, 0 for the SIMT kernel;
- * tile_m/tile_n receive the GEMM tile (may be NULL). */
+ * tile_m/tile_n receive the GEMM tile of one CTA or CTA pair: tile_m is 256
+ * when a CTA pair shares each MMA (cta_group::2), else 128 (may be NULL). */
 CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
 
 /* Run one cached causal Conv3D call on `stream` (device pointers, layouts as

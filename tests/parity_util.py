@@ -35,24 +35,36 @@ def to_device(a, dtype):
     return torch.from_numpy(np.ascontiguousarray(a)).to(torch_dtype(dtype)).cuda()
 
 
+class plan_env:
+    """Temporarily set CCV3D_* planner overrides (read at plan time only)."""
+
+    def __init__(self, env):
+        self.env = env
+
+    def __enter__(self):
+        self.old = {k: os.environ.get(k) for k in self.env}
+        os.environ.update({k: str(v) for k, v in self.env.items()})
+
+    def __exit__(self, *exc):
+        for k, v in self.old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
 class GpuCall:
     """One plan + device buffers (with guard bands around the outputs)."""
 
     GUARD = 256  # elements of sentinel before and after each output
 
-    def __init__(self, c, inp, force_simt=False):
+    def __init__(self, c, inp, force_simt=False, env=None):
         self.c = c
-        old = os.environ.get("CCV3D_FORCE_PATH")
+        env = dict(env or {})
         if force_simt:
-            os.environ["CCV3D_FORCE_PATH"] = "simt"
-        try:
+            env["CCV3D_FORCE_PATH"] = "simt"
+        with plan_env(env):
             self.plan = ccv3d.Plan(ccv3d.desc_for(c))
-        finally:
-            if force_simt:
-                if old is None:
-                    del os.environ["CCV3D_FORCE_PATH"]
-                else:
-                    os.environ["CCV3D_FORCE_PATH"] = old
         dt = c.dtype
         self.x = to_device(inp["x"], dt)
         self.cache = to_device(inp["cache"], dt)

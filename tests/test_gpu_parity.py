@@ -47,15 +47,17 @@ SMALL = [
     Conv("s_crop", 32, 32, 10, 12, T_x=1, cache_len=3),
     # p_l^base = 4 > d_t(kt-1): leading output frames have no active tap (bias only)
     Conv("s_biasonly", 32, 32, 10, 12, T_x=2, cache_len=0, pad_t_base=4, cache_keep=2),
+    # 3 boxes per frame: the last CTA pair has a box past the frame
+    Conv("s_odd_boxes", 64, 64, 12, 32, T_x=2, cache_len=1),
     # no bias, asymmetric pad/kernel
     Conv("s_nobias", 64, 32, 14, 30, T_x=2, cache_len=2, has_bias=False),
     Conv("s_k3x1x3", 32, 32, 14, 30, T_x=1, cache_len=2, kh=1, kw=3, pad=(0, 1)),
 ]
 
 
-def _run_small(c, force_simt=False):
+def _run_small(c, force_simt=False, env=None):
     inp = inputs_for(c)
-    call = GpuCall(c, inp, force_simt=force_simt).run()
+    call = GpuCall(c, inp, force_simt=force_simt, env=env).run()
     torch.cuda.synchronize()
     ref, ref_nc = oracle.forward(oracle_params(c), inp["x"], inp["cache"], inp["w"],
                                  inp["bias"])
@@ -76,12 +78,21 @@ def test_config1_fp32_exact_workload():
     assert call.plan.stats()["simt_path"] == 1
 
 
+@pytest.mark.parametrize("pair", [1, 0], ids=["cta_pair", "single_cta"])
 @pytest.mark.parametrize("c", SMALL, ids=lambda c: c.name)
-def test_small_tensor_core(c):
-    call, _ = _run_small(c)
+def test_small_tensor_core(c, pair):
+    call, _ = _run_small(c, env={"CCV3D_PAIR": pair})
     assert call.plan.path["tc"] is True
     st = call.plan.stats()
     assert st["calls"] == 1 and st["tc_path"] == 1 and st["errors"] == 0
+
+
+@pytest.mark.parametrize("env", [{"CCV3D_TILE_N": 384}, {"CCV3D_TILE_N": 384, "CCV3D_PAIR": 0},
+                                 {"CCV3D_TILE_N": 128}, {"CCV3D_STAGES": 2}],
+                         ids=["n384_pair", "n384_single", "n128", "stages2"])
+@pytest.mark.parametrize("c", [SMALL[5], SMALL[6], SMALL[13]], ids=lambda c: c.name)
+def test_small_tile_variants(c, env):
+    _run_small(c, env=env)
 
 
 @pytest.mark.parametrize("c", SMALL[:4] + SMALL[12:15] + SMALL[19:21], ids=lambda c: c.name)
