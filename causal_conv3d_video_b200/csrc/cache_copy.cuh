@@ -36,9 +36,20 @@ __device__ __forceinline__ void copy_new_cache(const CopyJob& c, long long part,
         const uint8_t* src = z_frame(c, n, c.z_len - c.keep + j);
         uint8_t* dst = c.dst + f * c.frame_bytes;
         if (vb == 16) {
-            const int4* s = reinterpret_cast<const int4*>(src);
-            int4* d = reinterpret_cast<int4*>(dst);
-            for (long long v = lo + tid; v < hi; v += nthreads) d[v] = __ldg(s + v);
+            // kU independent 16-byte loads in flight per thread before their
+            // stores (source and destination never overlap: checked on host)
+            constexpr int kU = 8;
+            const int4* __restrict__ s = reinterpret_cast<const int4*>(src);
+            int4* __restrict__ d = reinterpret_cast<int4*>(dst);
+            long long v = lo + tid;
+            for (; v + (long long)(kU - 1) * nthreads < hi; v += (long long)kU * nthreads) {
+                int4 r[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) r[u] = __ldg(s + v + (long long)u * nthreads);
+#pragma unroll
+                for (int u = 0; u < kU; ++u) __stcs(d + v + (long long)u * nthreads, r[u]);
+            }
+            for (; v < hi; v += nthreads) __stcs(d + v, __ldg(s + v));
         } else if (vb == 4) {
             const int* s = reinterpret_cast<const int*>(src);
             int* d = reinterpret_cast<int*>(dst);

@@ -22,6 +22,7 @@
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
 #include "conv_tc2.cuh"
+#include "conv_tcp.cuh"
 #include "params.h"
 
 using namespace ccv3d;
@@ -33,9 +34,15 @@ struct ccv3d_plan_s {
     int path_tc;  // 1: tcgen05 implicit GEMM, 0: SIMT
     int BK, BN, n_sub, box_h, box_w, tiles_x, tiles_y, tiles_n, stages, tmem_cols;
     int pair;  // 1: CTA-pair kernel (M = 256 per pair), 0: one CTA per 128-row tile
+    int persist;  // 1: persistent stream-K pair kernel
+    int G, n_acc;  // persistent: CTA pairs launched, TMEM accumulator buffers
+    long long frame_start[kMaxFrames + 1], sk_total;
     size_t smem_bytes;
     int device;
     int* d_status;
+    void* scratch;  // persistent: flags [2G] then fp32 partial tiles [2G][128][BN]
+    size_t scratch_bytes;
+    std::atomic<unsigned> epoch{0};
     std::atomic<uint64_t> calls{0}, tc{0}, simt{0}, unsupported{0}, errors{0};
 };
 
@@ -100,16 +107,48 @@ ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
 
 constexpr size_t kSmemBudget = 225 * 1024;
 
+// kind: 0 one CTA per tile, 1 CTA pair, 2 persistent CTA pair
 template <int BK>
-size_t smem_for(int pair, int bn, int stages) {
-    return pair ? tc2_smem_bytes<BK>(bn, stages) : tc_smem_bytes<BK>(bn, stages);
+size_t smem_for(int kind, int bn, int stages) {
+    return kind == 2 ? tcp_smem_bytes<BK>(bn, stages)
+                     : (kind == 1 ? tc2_smem_bytes<BK>(bn, stages) : tc_smem_bytes<BK>(bn, stages));
 }
 
 template <int BK>
-int pick_stages(int pair, int bn, int want) {
+int pick_stages(int kind, int bn, int want) {
     int s = want > 0 ? std::min(want, 12) : 8;
-    while (s > 2 && smem_for<BK>(pair, bn, s) > kSmemBudget) --s;
+    while (s > 2 && smem_for<BK>(kind, bn, s) > kSmemBudget) --s;
     return s;
+}
+
+template <int BK>
+void set_smem_attrs() {
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(conv_tc_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
+        cudaFuncSetAttribute(conv_tc2_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
+        cudaFuncSetAttribute(conv_tcp_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
+        cudaGetLastError();
+    });
+}
+
+// CTA pairs of the persistent kernel that can be resident at once.
+template <int BK>
+int resident_pairs(size_t smem) {
+    set_smem_attrs<BK>();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kTcpThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, conv_tcp_kernel<BK>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
 bool force_simt() {
@@ -161,20 +200,68 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     const char* pe = std::getenv("CCV3D_PAIR");
     p->pair = (p->BN / p->n_sub) >= 32 ? 1 : 0;
     if (pe != nullptr) p->pair = std::atoi(pe) != 0 && (p->BN / p->n_sub) >= 32;
-    // Short reductions (few k-blocks per tile) are dominated by each tile's
-    // fill and epilogue: keep the ring small enough for 3 CTAs per SM so one
-    // CTA's epilogue overlaps its neighbours' main loops.
-    const int kblocks = 3 * d.kh * d.kw * ceil_div(d.Cin, p->BK);
-    int want_s = env_int("CCV3D_STAGES");
-    if (want_s == 0 && kblocks <= 96) want_s = 4;
-    switch (p->BK) {
-        case 64: p->stages = pick_stages<64>(p->pair, p->BN, want_s); p->smem_bytes = smem_for<64>(p->pair, p->BN, p->stages); break;
-        case 32: p->stages = pick_stages<32>(p->pair, p->BN, want_s); p->smem_bytes = smem_for<32>(p->pair, p->BN, p->stages); break;
-        default: p->stages = pick_stages<16>(p->pair, p->BN, want_s); p->smem_bytes = smem_for<16>(p->pair, p->BN, p->stages); break;
+    // Persistent stream-K on CTA pairs (opt-in: CCV3D_PERSIST=1) when every
+    // output frame has an active tap and the frames fit the schedule table.
+    // Measured on B200 it is slower than one launch of pair tiles on every
+    // decoder signature: the calls are bound by aggregate L2->SM traffic,
+    // which spreading the k-blocks over all SM pairs does not reduce.
+    p->persist = 0;
+    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
+    const int frames = d.N * p->T_o;
+    if (p->pair && frames <= kMaxFrames && env_int("CCV3D_PERSIST") > 0) {
+        bool all_active = true;
+        long long acc = 0;
+        const long long tiles_per_frame =
+            (long long)((p->tiles_x * p->tiles_y + 1) / 2) * p->tiles_n;
+        for (int f = 0; f < frames; ++f) {
+            const int o = f % p->T_o;
+            int a = 0;
+            for (int k = 0; k < d.kt; ++k) a += (o >= p->o_l[k] && o < p->o_h[k]) ? 1 : 0;
+            all_active = all_active && a > 0;
+            p->frame_start[f] = acc;
+            acc += tiles_per_frame * a * per_tap;
+        }
+        p->frame_start[frames] = acc;
+        p->sk_total = acc;
+        p->persist = all_active ? 1 : 0;
     }
+    const int kind = p->persist ? 2 : p->pair;
+    // Short reductions (few k-blocks per tile) are dominated by each tile's
+    // fill and epilogue: without the persistent kernel, keep the ring small
+    // enough for 3 CTAs per SM so one CTA's epilogue overlaps the others.
+    int want_s = env_int("CCV3D_STAGES");
+    if (want_s == 0 && !p->persist && 3 * per_tap <= 96) want_s = 4;
+    switch (p->BK) {
+        case 64: p->stages = pick_stages<64>(kind, p->BN, want_s); p->smem_bytes = smem_for<64>(kind, p->BN, p->stages); break;
+        case 32: p->stages = pick_stages<32>(kind, p->BN, want_s); p->smem_bytes = smem_for<32>(kind, p->BN, p->stages); break;
+        default: p->stages = pick_stages<16>(kind, p->BN, want_s); p->smem_bytes = smem_for<16>(kind, p->BN, p->stages); break;
+    }
+    p->n_acc = (p->persist && 2 * p->BN <= 512) ? 2 : 1;
     p->tmem_cols = 32;
-    while (p->tmem_cols < p->BN) p->tmem_cols *= 2;
+    while (p->tmem_cols < p->n_acc * p->BN) p->tmem_cols *= 2;
     p->path_tc = 1;
+}
+
+// Persistent grid size: one CTA pair per resident pair slot, but at least 32
+// k-blocks per pair.  CCV3D_SK_PAIRS forces a size (tests of split tiles).
+void size_persistent(ccv3d_plan_s* p, bool have_device) {
+    if (!p->persist) return;
+    int pairs = 74;
+    if (have_device) {
+        int n = 0;
+        switch (p->BK) {
+            case 64: n = resident_pairs<64>(p->smem_bytes); break;
+            case 32: n = resident_pairs<32>(p->smem_bytes); break;
+            default: n = resident_pairs<16>(p->smem_bytes); break;
+        }
+        if (n > 0) pairs = n;
+    }
+    long long G = std::min<long long>(pairs, std::max<long long>(1, p->sk_total / 32));
+    const int want = env_int("CCV3D_SK_PAIRS");
+    if (want > 0) G = std::min<long long>(want, pairs);
+    p->G = (int)std::max<long long>(1, std::min<long long>(G, p->sk_total));
+    const size_t flags = ((size_t)2 * p->G * sizeof(unsigned) + 255) / 256 * 256;
+    p->scratch_bytes = flags + (size_t)2 * p->G * kTileM * p->BN * sizeof(float);
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -251,20 +338,11 @@ Taps make_taps(const ccv3d_plan_s* p) {
 }
 
 template <int BK>
-cudaError_t launch_tc(const TcParams& prm, int pair, int grid, size_t smem, cudaStream_t s) {
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [] {
-        attr = cudaFuncSetAttribute(conv_tc_kernel<BK>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)(227 * 1024));
-        if (attr == cudaSuccess)
-            attr = cudaFuncSetAttribute(conv_tc2_kernel<BK>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)(227 * 1024));
-    });
-    if (attr != cudaSuccess) return attr;
-    if (pair)
+cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s) {
+    set_smem_attrs<BK>();
+    if (kind == 2)
+        conv_tcp_kernel<BK><<<grid, kTcpThreads, smem, s>>>(prm);
+    else if (kind == 1)
         conv_tc2_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
     else
         conv_tc_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
@@ -298,19 +376,36 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     prm.tmem_cols = p->tmem_cols;
     prm.wait_limit_ns = kWaitLimitNs;
     prm.pairs_per_frame = (p->tiles_x * p->tiles_y + 1) / 2;
-    const long long grid =
+    long long grid =
         p->pair ? 2LL * d.N * p->T_o * prm.pairs_per_frame * p->tiles_n
                 : (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
+    if (p->persist) {
+        if (p->scratch == nullptr) return CCV3D_ERR_CUDA;
+        grid = 2LL * p->G;
+        const int frames = d.N * p->T_o;
+        for (int f = 0; f <= frames; ++f) prm.sk.frame_start[f] = p->frame_start[f];
+        prm.sk.total = p->sk_total;
+        prm.sk.n_frames = frames;
+        prm.sk.G = p->G;
+        prm.sk.n_acc = p->n_acc;
+        const size_t flags = ((size_t)2 * p->G * sizeof(unsigned) + 255) / 256 * 256;
+        prm.sk.flags = static_cast<unsigned*>(p->scratch);
+        prm.sk.partial = reinterpret_cast<float*>(static_cast<char*>(p->scratch) + flags);
+        unsigned e = p->epoch.fetch_add(1) + 1;
+        if (e == 0) e = p->epoch.fetch_add(1) + 1;  // 0 marks "never published"
+        prm.sk.epoch = e;
+    }
     if (grid > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
     // spread the K-start offsets over one wave of concurrently running tiles
     const long long units = p->pair ? grid / 2 : grid;
     const long long wave = p->pair ? 74 : 148;
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
+    const int kind = p->persist ? 2 : p->pair;
     cudaError_t e;
     switch (p->BK) {
-        case 64: e = launch_tc<64>(prm, p->pair, (int)grid, p->smem_bytes, stream); break;
-        case 32: e = launch_tc<32>(prm, p->pair, (int)grid, p->smem_bytes, stream); break;
-        default: e = launch_tc<16>(prm, p->pair, (int)grid, p->smem_bytes, stream); break;
+        case 64: e = launch_tc<64>(prm, kind, (int)grid, p->smem_bytes, stream); break;
+        case 32: e = launch_tc<32>(prm, kind, (int)grid, p->smem_bytes, stream); break;
+        default: e = launch_tc<16>(prm, kind, (int)grid, p->smem_bytes, stream); break;
     }
     return e == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
 }
@@ -378,18 +473,29 @@ ccv3d_status ccv3d_plan(ccv3d_plan_t* out, const ccv3d_desc* desc) {
     // ccv3d_forward refuses with CCV3D_ERR_CUDA.
     p->device = -1;
     p->d_status = nullptr;
+    p->scratch = nullptr;
+    p->scratch_bytes = 0;
     int ndev = 0;
-    if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
-        if (cudaGetDevice(&p->device) != cudaSuccess ||
-            cudaMalloc(&p->d_status, 256) != cudaSuccess ||
-            cudaMemset(p->d_status, 0, 256) != cudaSuccess) {
+    const bool have_device = cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0;
+    if (!have_device) cudaGetLastError();
+    size_persistent(p, have_device);
+    if (have_device) {
+        bool ok = cudaGetDevice(&p->device) == cudaSuccess &&
+                  cudaMalloc(&p->d_status, 256) == cudaSuccess &&
+                  cudaMemset(p->d_status, 0, 256) == cudaSuccess;
+        if (ok && p->scratch_bytes > 0) {
+            // split-tile flags start at 0 ("never published"); launches tag
+            // theirs with a per-plan epoch, so no clearing between calls
+            ok = cudaMalloc(&p->scratch, p->scratch_bytes) == cudaSuccess &&
+                 cudaMemset(p->scratch, 0, p->scratch_bytes) == cudaSuccess;
+        }
+        if (!ok) {
             cudaGetLastError();
             if (p->d_status) cudaFree(p->d_status);
+            if (p->scratch) cudaFree(p->scratch);
             delete p;
             return CCV3D_ERR_CUDA;
         }
-    } else {
-        cudaGetLastError();
     }
     *out = p;
     return CCV3D_OK;
@@ -477,7 +583,7 @@ ccv3d_status ccv3d_get_stats(ccv3d_plan_t p, ccv3d_stats* s) {
     s->simt_path = p->simt.load();
     s->unsupported = p->unsupported.load();
     s->errors = p->errors.load();
-    s->workspace_bytes = 0;
+    s->workspace_bytes = p->scratch_bytes;
     return CCV3D_OK;
 }
 
@@ -495,6 +601,7 @@ ccv3d_status ccv3d_get_status(ccv3d_plan_t p) {
 void ccv3d_destroy(ccv3d_plan_t p) {
     if (p == nullptr) return;
     if (p->d_status) cudaFree(p->d_status);
+    if (p->scratch) cudaFree(p->scratch);
     delete p;
 }
 

@@ -20,6 +20,7 @@
 
 #include "cache_copy.cuh"
 #include "conv_tc.cuh"
+#include "kwalk.cuh"
 #include "params.h"
 #include "ptx.cuh"
 
@@ -110,65 +111,55 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && iters > 0) {
             // --------------------------------- TMA producer (both CTAs)
-            // The reduction is walked from a per-tile starting point spread
-            // over [0, iters): CTAs running at the same time then read
-            // different weight rows instead of all hitting the same L2 lines.
-            int act[kMaxTaps], n_act = 0;
-            for (int k = 0; k < p.taps.kt; ++k)
-                if (o >= p.taps.o_l[k] && o < p.taps.o_h[k]) act[n_act++] = k;
-            const int per_tap = p.kh * p.kw * p.n_cb;
-            const int rot = iters > 0 ? (int)(((long long)pair * iters) / p.rot_div) % iters : 0;
+            // Each pair starts its reduction at a different k-block, so
+            // pairs running at the same time read different weight rows.
+            int act[kMaxTaps];
+            const int n_act = active_tap_list(p, o, act);
+            const int rot = (int)(((long long)pair * iters) / p.rot_div) % iters;
             const uint32_t pair_bytes = 2u * (uint32_t)(kA + kBc);
+            const int ybase = ty * p.box_h * p.s_h - p.p_h;
+            const int xbase = tx * p.box_w * p.s_w - p.p_w;
+            KWalk w;
+            w.set(rot, p);
+            TapSrc ts = tap_source(p, act[w.ti], n, o);
+            Ring ring;
             for (int it = 0; it < iters; ++it) {
-                const int st = it % stages;
-                if (it >= stages &&
-                    !mbar_wait(smem_u32(&empty_bar[st]), ((it / stages) & 1) ^ 1, p.status,
-                               p.wait_limit_ns))
+                if (it >= stages && !mbar_wait(smem_u32(&empty_bar[ring.st]), ring.ph ^ 1u,
+                                               p.status, p.wait_limit_ns))
                     break;
-                int kb = it + rot;  // k-block of the reduction loaded at step `it`
-                if (kb >= iters) kb -= iters;
-                const int k = act[kb / per_tap];
-                const int cb = kb % p.n_cb;
-                const int rs = (kb / p.n_cb) % (p.kh * p.kw);
-                const int r = rs / p.kw, s = rs % p.kw;
-                const int t = o + p.taps.delta[k];  // frame of Z
-                const CUtensorMap* src;
-                int f;
-                if (t < p.cache_len) {
-                    src = &p.tmap_c;
-                    f = n * p.cache_len + t;
-                } else {
-                    src = &p.tmap_x;
-                    f = n * p.T_x + (t - p.cache_len);
-                }
-                const int y0 = ty * p.box_h * p.s_h + r * p.d_h - p.p_h;
-                const int x0 = tx * p.box_w * p.s_w + s * p.d_w - p.p_w;
-                const int wrow = (k * p.kh + r) * p.kw + s;
-                const uint32_t fb_local = smem_u32(&full_bar[st]);
+                const int y0 = ybase + w.r * p.d_h;
+                const int x0 = xbase + w.s * p.d_w;
+                const int wrow = ts.wtap + w.r * p.kw + w.s;
+                const uint32_t fb_local = smem_u32(&full_bar[ring.st]);
                 if (leader) mbar_arrive_expect_tx(fb_local, pair_bytes);
                 const uint32_t fb = pair_leader_addr(fb_local);
-                tma_load_4d_pair(smem_u32(sA + (size_t)st * kA), src, fb, cb * BK,
-                                 x0, y0, f);
+                tma_load_4d_pair(smem_u32(sA + ring.st * kA), ts.map, fb, w.cb * BK, x0, y0,
+                                 ts.frame);
                 for (int j = 0; j < p.n_sub; ++j)
-                    tma_load_3d_pair(
-                        smem_u32(sB + (size_t)st * kBc + (size_t)j * kBh), &p.tmap_w,
-                        fb, cb * BK, wrow, n_tile * BN + j * BNs + (int)rank * hB);
+                    tma_load_3d_pair(smem_u32(sB + ring.st * kBc + j * kBh), &p.tmap_w, fb,
+                                     w.cb * BK, wrow, n_tile * BN + j * BNs + (int)rank * hB);
+                ring.next(stages);
+                if (w.next(p)) {
+                    if (w.ti == n_act) w.ti = 0;
+                    ts = tap_source(p, act[w.ti], n, o);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ------------------------------ MMA issuer (even CTA only)
             const uint32_t idesc = idesc_bf16_m256((uint32_t)BNs);
+            const uint64_t a0 = smem_desc_kmajor(smem_u32(sA), kRow);
+            const uint64_t b0 = smem_desc_kmajor(smem_u32(sB), kRow);
+            Ring ring;
             for (int it = 0; it < iters; ++it) {
-                const int st = it % stages;
-                if (!mbar_wait(smem_u32(&full_bar[st]), (it / stages) & 1, p.status,
-                               p.wait_limit_ns))
+                if (!mbar_wait(smem_u32(&full_bar[ring.st]), ring.ph, p.status, p.wait_limit_ns))
                     break;
                 tc_fence_after();
-                const uint64_t a_desc = smem_desc_kmajor(smem_u32(sA + (size_t)st * kA), kRow);
-                const uint64_t b_desc = smem_desc_kmajor(smem_u32(sB + (size_t)st * kBc), kRow);
+                const uint64_t a_desc = a0 + (uint64_t)((ring.st * kA) >> 4);
+                const uint64_t b_desc = b0 + (uint64_t)((ring.st * kBc) >> 4);
                 for (int j = 0; j < p.n_sub; ++j) {
                     const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
 #pragma unroll
@@ -176,7 +167,8 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
                         umma_bf16_pair(tmem_base + (uint32_t)(j * BNs), a_desc + 2u * kk,
                                        bj + 2u * kk, idesc, (it | kk) != 0 ? 1u : 0u);
                 }
-                umma_commit_pair(smem_u32(&empty_bar[st]), (uint16_t)0x3);
+                umma_commit_pair(smem_u32(&empty_bar[ring.st]), (uint16_t)0x3);
+                ring.next(stages);
             }
             umma_commit_pair(smem_u32(acc_bar), (uint16_t)0x3);
         }

@@ -1,0 +1,404 @@
+// conv_tcp.cuh -- persistent, stream-K implicit-GEMM Conv3D on CTA pairs.
+//
+// The work of one call is the list of pair tiles (two 128-pixel boxes of one
+// output frame x a Cout tile), each a reduction of iters(o) k-blocks, where
+// iters(o) = (active taps of frame o) x kh x kw x ceil(Cin/BK) follows the
+// paper's per-tap intervals (Sec. 4).  The k-blocks of all tiles, laid end to
+// end, are cut into G equal ranges, one per resident CTA pair (stream-K), so
+// every SM pair gets the same number of MMAs whatever the tile count.
+//
+// A tile cut by range boundaries is finished by the pair whose range holds
+// its first k-block (the "owner"): that pair reaches the tile last, at the end
+// of its range, while every other pair holding a piece of the tile meets it
+// first, at the start of its range.  Those pairs store their fp32 partial
+// accumulators in the scratch area (one slot per CTA: only a range's first
+// piece can be partial) and publish a flag carrying the launch's epoch; the
+// owner waits for the flags (bounded), adds the partials, then applies bias
+// and rounding once.
+//
+// Per CTA: warp 0 streams TMA loads, warp 1 holds TMEM (the even CTA's lane 0
+// issues the pair MMAs), warps 2-5 run the epilogues and warps 6-9 copy this
+// CTA's slice of new_cache while the GEMM runs.  With Cout tiles of <= 256 columns the accumulator is double
+// buffered in TMEM, so a tile's epilogue overlaps the next tile's main loop.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "cache_copy.cuh"
+#include "conv_tc.cuh"
+#include "conv_tc2.cuh"
+#include "kwalk.cuh"
+#include "params.h"
+#include "ptx.cuh"
+
+namespace ccv3d {
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ uint32_t mapa_cluster(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Named barrier over the four epilogue warps (barrier 1, 128 threads).
+__device__ __forceinline__ void epi_bar() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// One piece of a pair's range: pair tile `tile` (frame f, index in frame),
+// k-blocks [kb0, kb1) of its reduction of `iters` k-blocks.
+struct Seg {
+    long long tile_start;  // global k-block index of the tile's first k-block
+    int f, tile_in_frame, iters, kb0, kb1;
+};
+
+// Range of k-blocks of pair g: [start(g), start(g+1)).
+__device__ __forceinline__ long long sk_start(const TcParams& p, int g) {
+    return (long long)g * p.sk.total / p.sk.G;  // g <= G <= 128, total < 2^40
+}
+
+__device__ __forceinline__ int active_taps(const TcParams& p, int o) {
+    int a = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxTaps; ++k)
+        if (k < p.taps.kt && o >= p.taps.o_l[k] && o < p.taps.o_h[k]) ++a;
+    return a;
+}
+
+// The segment of pair tile work containing global k-block I, clipped to end.
+__device__ __forceinline__ Seg sk_locate(const TcParams& p, long long I, long long end) {
+    Seg s;
+    int f = 0;
+    while (f + 1 < p.sk.n_frames && p.sk.frame_start[f + 1] <= I) ++f;
+    const int o = f % p.T_o;
+    const int iters = active_taps(p, o) * p.kh * p.kw * p.n_cb;
+    const long long local = I - p.sk.frame_start[f];
+    s.f = f;
+    s.iters = iters;
+    s.tile_in_frame = (int)(local / iters);
+    s.tile_start = p.sk.frame_start[f] + (long long)s.tile_in_frame * iters;
+    s.kb0 = (int)(I - s.tile_start);
+    const long long e = end - s.tile_start;
+    s.kb1 = e < iters ? (int)e : iters;
+    return s;
+}
+
+// Pair whose range holds global k-block J.
+__device__ __forceinline__ int sk_owner_of(const TcParams& p, long long J) {
+    int g = (int)(J * p.sk.G / p.sk.total);
+    if (g >= p.sk.G) g = p.sk.G - 1;
+    while (g + 1 < p.sk.G && sk_start(p, g + 1) <= J) ++g;
+    while (g > 0 && sk_start(p, g) > J) --g;
+    return g;
+}
+
+template <int BK>
+__host__ __device__ constexpr size_t tcp_smem_bytes(int bn, int stages) {
+    // A box + half the weight rows per stage, ring barriers, 2 x (acc full,
+    // acc empty) barriers, TMEM address slot
+    return 1024 + (size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes) +
+           (size_t)(2 * stages + 4) * 8 + 16;
+}
+
+constexpr int kTcpThreads = 320;  // + warps 6-9: the new_cache copy
+
+template <int BK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcpThreads, 1)
+conv_tcp_kernel(const __grid_constant__ TcParams p) {
+    constexpr int kRow = TcSmem<BK>::kRowBytes;
+    constexpr int kA = TcSmem<BK>::kABytes;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int stages = p.stages;
+    const int BN = p.BN;
+    const int BNs = BN / p.n_sub;
+    const int hB = BNs / 2;
+    const int kBc = (BN / 2) * kRow;
+    const int kBh = hB * kRow;
+    const int n_acc = p.sk.n_acc;
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + (size_t)stages * kA;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kBc);
+    uint64_t* empty_bar = full_bar + stages;
+    uint64_t* acc_full = empty_bar + stages;   // [2]
+    uint64_t* acc_empty = acc_full + 2;        // [2], used in the even CTA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int g = blockIdx.x >> 1;  // this pair's range
+    const long long range0 = sk_start(p, g), range1 = sk_start(p, g + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&acc_full[b]), 1);
+            mbar_init(smem_u32(&acc_empty[b]), 8);  // 4 epilogue warps x 2 CTAs
+        }
+        fence_mbar_init();
+        tma_prefetch_desc(&p.tmap_x);
+        if (p.cache_len > 0) tma_prefetch_desc(&p.tmap_c);
+        tma_prefetch_desc(&p.tmap_w);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------ TMA producer
+            const uint32_t pair_bytes = 2u * (uint32_t)(kA + kBc);
+            Ring ring;  // continues across segments
+            long long issued = 0;
+            bool ok = true;
+            for (long long I = range0; I < range1 && ok;) {
+                const Seg sg = sk_locate(p, I, range1);
+                const int o = sg.f % p.T_o, n = sg.f / p.T_o;
+                const int pp = sg.tile_in_frame / p.tiles_n;
+                const int n_tile = sg.tile_in_frame % p.tiles_n;
+                const int box = pp * 2 + (int)rank;
+                int tx = 0, ty = p.tiles_y;
+                if (box < p.tiles_x * p.tiles_y) {
+                    tx = box % p.tiles_x;
+                    ty = box / p.tiles_x;
+                }
+                int act[kMaxTaps];
+                active_tap_list(p, o, act);
+                const int ybase = ty * p.box_h * p.s_h - p.p_h;
+                const int xbase = tx * p.box_w * p.s_w - p.p_w;
+                const int nrow = n_tile * BN + (int)rank * hB;
+                KWalk w;
+                w.set(sg.kb0, p);
+                TapSrc ts = tap_source(p, act[w.ti], n, o);
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                    if (issued >= stages &&
+                        !mbar_wait(smem_u32(&empty_bar[ring.st]), ring.ph ^ 1u, p.status,
+                                   p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const int y0 = ybase + w.r * p.d_h;
+                    const int x0 = xbase + w.s * p.d_w;
+                    const int wrow = ts.wtap + w.r * p.kw + w.s;
+                    const uint32_t fb_local = smem_u32(&full_bar[ring.st]);
+                    if (leader) mbar_arrive_expect_tx(fb_local, pair_bytes);
+                    const uint32_t fb = pair_leader_addr(fb_local);
+                    tma_load_4d_pair(smem_u32(sA + ring.st * kA), ts.map, fb, w.cb * BK, x0, y0,
+                                     ts.frame);
+                    for (int j = 0; j < p.n_sub; ++j)
+                        tma_load_3d_pair(smem_u32(sB + ring.st * kBc + j * kBh), &p.tmap_w, fb,
+                                         w.cb * BK, wrow, nrow + j * BNs);
+                    ring.next(stages);
+                    ++issued;
+                    if (w.next(p) && kb + 1 < sg.kb1) ts = tap_source(p, act[w.ti], n, o);
+                }
+                I = sg.tile_start + sg.kb1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------- MMA issuer (even CTA only)
+            const uint32_t idesc = idesc_bf16_m256((uint32_t)BNs);
+            const uint64_t a0 = smem_desc_kmajor(smem_u32(sA), kRow);
+            const uint64_t b0 = smem_desc_kmajor(smem_u32(sB), kRow);
+            Ring ring;
+            int seg = 0;
+            bool ok = true;
+            for (long long I = range0; I < range1 && ok; ++seg) {
+                const Seg sg = sk_locate(p, I, range1);
+                const int b = n_acc == 2 ? (seg & 1) : 0;
+                const int round = n_acc == 2 ? (seg >> 1) : seg;
+                if (round > 0 &&
+                    !mbar_wait(smem_u32(&acc_empty[b]), (uint32_t)((round & 1) ^ 1), p.status,
+                               p.wait_limit_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                    if (!mbar_wait(smem_u32(&full_bar[ring.st]), ring.ph, p.status,
+                                   p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = a0 + (uint64_t)((ring.st * kA) >> 4);
+                    const uint64_t b_desc = b0 + (uint64_t)((ring.st * kBc) >> 4);
+                    const uint32_t first = kb == sg.kb0 ? 1u : 0u;
+                    for (int j = 0; j < p.n_sub; ++j) {
+                        const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16_pair(d_tmem + (uint32_t)(j * BNs), a_desc + 2u * kk,
+                                           bj + 2u * kk, idesc, (first && kk == 0) ? 0u : 1u);
+                    }
+                    umma_commit_pair(smem_u32(&empty_bar[ring.st]), (uint16_t)0x3);
+                    ring.next(stages);
+                }
+                umma_commit_pair(smem_u32(&acc_full[b]), (uint16_t)0x3);
+                I = sg.tile_start + sg.kb1;
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ----------------- new_cache slice, beside the GEMM of this CTA
+        copy_new_cache(p.copy, blockIdx.x, gridDim.x, threadIdx.x - 192, 128);
+    } else {
+        // ------------------------------------------------- the epilogues
+        const int etid = threadIdx.x - 64;
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t empty_leader = mapa_cluster(smem_u32(&acc_empty[0]), 0);
+        int seg = 0;
+        bool ok = true;
+        for (long long I = range0; I < range1; ++seg) {
+            const Seg sg = sk_locate(p, I, range1);
+            const int b = n_acc == 2 ? (seg & 1) : 0;
+            const int round = n_acc == 2 ? (seg >> 1) : seg;
+            const int o = sg.f % p.T_o, n = sg.f / p.T_o;
+            const int pp = sg.tile_in_frame / p.tiles_n;
+            const int n_tile = sg.tile_in_frame % p.tiles_n;
+            const int box = pp * 2 + (int)rank;
+            int tx = 0, ty = p.tiles_y;
+            if (box < p.tiles_x * p.tiles_y) {
+                tx = box % p.tiles_x;
+                ty = box / p.tiles_x;
+            }
+            if (ok && !mbar_wait(smem_u32(&acc_full[b]), (uint32_t)(round & 1), p.status,
+                                 p.wait_limit_ns))
+                ok = false;
+            tc_fence_after();
+            const bool owner = sg.kb0 == 0;
+            const bool whole = owner && sg.kb1 == sg.iters;
+            // pairs holding the other pieces of this tile (owner only)
+            int g_last = g;
+            if (owner && !whole) g_last = sk_owner_of(p, sg.tile_start + sg.iters - 1);
+            if (owner && !whole && ok) {
+                // wait until every contributor of this CTA's rank has published
+                for (int gc = g + 1; gc <= g_last && ok; ++gc) {
+                    const unsigned* flag = p.sk.flags + 2 * gc + rank;
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(flag) != p.sk.epoch) {
+                        if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+                            atomicCAS(p.status, 0, kStatusTimeout);
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+            }
+            const int y = ty * p.box_h + row / p.box_w;
+            const int x = tx * p.box_w + row % p.box_w;
+            const bool valid = y < p.H_o && x < p.W_o;
+            uint16_t* orow = p.out + ((((long long)n * p.T_o + o) * p.H_o + y) * p.W_o + x) *
+                                         (long long)p.Cout;
+            float* mine = p.sk.partial + ((size_t)(2 * g + rank) * kTileM + row) * BN;
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) +
+                                       (uint32_t)(b * BN + c0), v);
+                tmem_ld_wait();
+                if (!ok) continue;
+                float a[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) a[j] = __uint_as_float(v[j]);
+                if (!owner) {
+                    // a piece of a tile owned by an earlier pair: publish fp32
+                    float4* dst = reinterpret_cast<float4*>(mine + c0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_float4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+                    continue;
+                }
+                for (int gc = g + 1; gc <= g_last; ++gc) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.sk.partial + ((size_t)(2 * gc + rank) * kTileM + row) * BN + c0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 w4 = __ldcg(src + j);
+                        a[4 * j] += w4.x;
+                        a[4 * j + 1] += w4.y;
+                        a[4 * j + 2] += w4.z;
+                        a[4 * j + 3] += w4.w;
+                    }
+                }
+                const int co = n_tile * BN + c0;
+                if (!valid || co >= p.Cout) continue;
+                uint32_t packed[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float b0 = 0.f, b1 = 0.f;
+                    if (p.bias != nullptr) {
+                        if (co + 2 * j < p.Cout)
+                            b0 = __bfloat162float(__ushort_as_bfloat16(p.bias[co + 2 * j]));
+                        if (co + 2 * j + 1 < p.Cout)
+                            b1 = __bfloat162float(__ushort_as_bfloat16(p.bias[co + 2 * j + 1]));
+                    }
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * j] + b0, a[2 * j + 1] + b1);
+                    packed[j] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                if (co + 16 <= p.Cout) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + co);
+                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (co + j < p.Cout)
+                            orow[co + j] = (uint16_t)(packed[j >> 1] >> ((j & 1) * 16));
+                }
+            }
+            // TMEM buffer b is drained: hand it back to the MMA issuer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(smem_u32(&acc_empty[b]));
+                else
+                    mbar_arrive_remote(empty_leader + (uint32_t)(b * 8));
+            }
+            if (!owner) {
+                // publish this CTA's piece: stores visible before the flag
+                __threadfence();
+                epi_bar();  // all 128 epilogue threads (owner is uniform)
+                if (etid == 0 && ok) st_release_gpu(p.sk.flags + 2 * g + rank, p.sk.epoch);
+            }
+            I = sg.tile_start + sg.kb1;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, (uint32_t)p.tmem_cols);
+    }
+}
+
+}  // namespace ccv3d

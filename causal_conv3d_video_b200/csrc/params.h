@@ -29,6 +29,20 @@ struct Taps {
     int o_h[kMaxTaps];
 };
 
+constexpr int kMaxFrames = 64;  // (n, o) frames a persistent stream-K launch can hold
+
+// Stream-K schedule of the persistent pair kernel.
+struct StreamK {
+    long long frame_start[kMaxFrames + 1];  // first k-block of each frame's tiles
+    long long total;                        // k-blocks of all tiles
+    int n_frames;                           // N * T_o
+    int G;                                  // CTA pairs in the persistent grid
+    int n_acc;                              // TMEM accumulator buffers (1 or 2)
+    float* partial;                         // [2G][128][BN] fp32 pieces of split tiles
+    unsigned* flags;                        // [2G] epoch of the last published piece
+    unsigned epoch;                         // this launch's tag (never 0)
+};
+
 struct __align__(64) TcParams {
     CUtensorMap tmap_x;      // x      as [N*T_x, H, W, Cin], box [BK, bw*s_w, bh*s_h, 1]
     CUtensorMap tmap_c;      // cache  as [N*|C|, H, W, Cin] (unused when |C| = 0)
@@ -45,6 +59,7 @@ struct __align__(64) TcParams {
     int BN, n_sub, n_cb, stages, tmem_cols;
     int pairs_per_frame;     // CTA-pair kernel: ceil(tiles_x * tiles_y / 2)
     int rot_div;             // tiles (or pairs) over which K-start offsets are spread
+    StreamK sk;
     uint64_t wait_limit_ns;
 };
 

@@ -78,13 +78,31 @@ def test_config1_fp32_exact_workload():
     assert call.plan.stats()["simt_path"] == 1
 
 
-@pytest.mark.parametrize("pair", [1, 0], ids=["cta_pair", "single_cta"])
+KERNELS = {"persistent": {"CCV3D_PERSIST": 1}, "pair": {}, "single": {"CCV3D_PAIR": 0}}
+
+
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
 @pytest.mark.parametrize("c", SMALL, ids=lambda c: c.name)
-def test_small_tensor_core(c, pair):
-    call, _ = _run_small(c, env={"CCV3D_PAIR": pair})
+def test_small_tensor_core(c, kernel):
+    call, _ = _run_small(c, env=KERNELS[kernel])
     assert call.plan.path["tc"] is True
     st = call.plan.stats()
     assert st["calls"] == 1 and st["tc_path"] == 1 and st["errors"] == 0
+
+
+@pytest.mark.parametrize("pairs", [2, 3, 5, 11])
+@pytest.mark.parametrize("c", [SMALL[3], SMALL[5], SMALL[8], SMALL[12], SMALL[15], SMALL[18]],
+                         ids=lambda c: c.name)
+def test_small_stream_k_split_tiles(c, pairs):
+    """Few persistent pairs: tiles are cut across pairs and finished by their
+    owner from published fp32 pieces; repeated calls reuse the scratch flags."""
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 1, "CCV3D_SK_PAIRS": pairs})
+    first = call.out.clone()
+    call.run()
+    call.run()
+    torch.cuda.synchronize()
+    assert torch.equal(first, call.out)
+    assert call.plan.status() == ccv3d.CCV3D_OK
 
 
 @pytest.mark.parametrize("env", [{"CCV3D_TILE_N": 384}, {"CCV3D_TILE_N": 384, "CCV3D_PAIR": 0},
