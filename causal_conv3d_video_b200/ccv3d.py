@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libccv3d.so")
 CCV3D_BF16, CCV3D_FP32 = 0, 1
 STATUS = {0: "CCV3D_OK", 1: "CCV3D_ERR_INVALID", 2: "CCV3D_ERR_UNSUPPORTED",
           3: "CCV3D_ERR_EMPTY_OUTPUT", 4: "CCV3D_ERR_ALIGNMENT", 5: "CCV3D_ERR_ALIAS",
-          6: "CCV3D_ERR_CUDA", 7: "CCV3D_ERR_TIMEOUT"}
+          6: "CCV3D_ERR_CUDA", 7: "CCV3D_ERR_TIMEOUT", 8: "CCV3D_ERR_SCRATCH_LIMIT"}
 for _code, _name in STATUS.items():
     globals()[_name] = _code
 CCV3D_MAX_KT = 3
@@ -24,7 +24,8 @@ CCV3D_MAX_KT = 3
 # every symbol include/ccv3d.h declares
 EXPORTED = ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_plan_path", "ccv3d_forward",
             "ccv3d_get_stats", "ccv3d_get_status", "ccv3d_destroy", "ccv3d_strerror",
-            "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout")
+            "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout", "ccv3d_forward_noalloc")
+CCV3D_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class ccv3d_desc(ctypes.Structure):
@@ -66,8 +67,11 @@ def _load():
     lib.ccv3d_plan_sizes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t),
                                      ctypes.POINTER(ctypes.c_size_t), ip]
     lib.ccv3d_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.ccv3d_forward_noalloc.argtypes = [ctypes.POINTER(ccv3d_desc), vp, vp, vp, vp, vp, vp,
+                                          ip, ip, ip, vp]
     for f in ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_forward", "ccv3d_get_stats",
-              "ccv3d_get_status", "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout"):
+              "ccv3d_get_status", "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout",
+              "ccv3d_forward_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     del i3
     return lib
@@ -144,6 +148,22 @@ def ccv3d_forward(plan, x, cache, w, bias, out, new_cache, stride, pad, dilation
                            _ptr(new_cache), s, p, d, _stream(stream))
     if rc != 0 and check:
         raise CCV3DError(rc, "ccv3d_forward")
+    return rc
+
+
+def ccv3d_forward_noalloc(desc: ccv3d_desc, x, cache, w, bias, out, new_cache, stride, pad,
+                          dilation, stream=None, check: bool = True) -> int:
+    """The no-allocation variant of ccv3d_forward: no plan, no device memory
+    allocated by the library (its scratch is a fixed array inside the shared
+    library, shared by all such calls on a device -- they must not overlap on
+    the GPU).  For callers that may not allocate device memory."""
+    s = (ctypes.c_int * 2)(*stride)
+    p = (ctypes.c_int * 2)(*pad)
+    d = (ctypes.c_int * 3)(*dilation)
+    rc = lib.ccv3d_forward_noalloc(ctypes.byref(desc), _ptr(x), _ptr(cache), _ptr(w), _ptr(bias),
+                                   _ptr(out), _ptr(new_cache), s, p, d, _stream(stream))
+    if rc != 0 and check:
+        raise CCV3DError(rc, "ccv3d_forward_noalloc")
     return rc
 
 

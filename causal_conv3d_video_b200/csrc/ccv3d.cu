@@ -32,6 +32,7 @@ struct ccv3d_plan_s {
     int T_o, H_o, W_o, z_len, p_l, keep;
     int delta[kMaxTaps], o_l[kMaxTaps], o_h[kMaxTaps];
     int path_tc;  // 1: tcgen05 implicit GEMM, 0: SIMT
+    int path_tc_candidate;  // the tensor-core tiling below is filled in
     int BK, BN, n_sub, box_h, box_w, tiles_x, tiles_y, tiles_n, stages, tmem_cols;
     int pair;  // 1: CTA-pair kernel (M = 256 per pair), 0: one CTA per 128-row tile
     int persist;  // 1: persistent stream-K pair kernel
@@ -162,6 +163,50 @@ int env_int(const char* name) {
     return e != nullptr ? std::atoi(e) : 0;
 }
 
+// Schedule of the persistent stream-K pair kernel: usable when the plan runs
+// CTA pairs, every output frame has an active tap and the (n, o) frames fit
+// the schedule table.  Sets p->persist; returns it.
+bool setup_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    p->persist = 0;
+    if (!p->path_tc_candidate || !p->pair) return false;
+    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
+    const int frames = d.N * p->T_o;
+    if (frames > kMaxFrames) return false;
+    long long acc = 0;
+    const long long tiles_per_frame = (long long)((p->tiles_x * p->tiles_y + 1) / 2) * p->tiles_n;
+    for (int f = 0; f < frames; ++f) {
+        const int o = f % p->T_o;
+        int a = 0;
+        for (int k = 0; k < d.kt; ++k) a += (o >= p->o_l[k] && o < p->o_h[k]) ? 1 : 0;
+        if (a == 0) return false;
+        p->frame_start[f] = acc;
+        acc += tiles_per_frame * a * per_tap;
+    }
+    p->frame_start[frames] = acc;
+    p->sk_total = acc;
+    p->persist = 1;
+    return true;
+}
+
+// Ring depth, shared memory and TMEM columns of the chosen tensor-core kernel.
+void size_tc(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
+    const int kind = p->persist ? 2 : p->pair;
+    // Short reductions (few k-blocks per tile) are dominated by each tile's
+    // fill and epilogue: without the persistent kernel, keep the ring small
+    // enough for 3 CTAs per SM so one CTA's epilogue overlaps the others.
+    int want_s = env_int("CCV3D_STAGES");
+    if (want_s == 0 && !p->persist && 3 * per_tap <= 96) want_s = 4;
+    switch (p->BK) {
+        case 64: p->stages = pick_stages<64>(kind, p->BN, want_s); p->smem_bytes = smem_for<64>(kind, p->BN, p->stages); break;
+        case 32: p->stages = pick_stages<32>(kind, p->BN, want_s); p->smem_bytes = smem_for<32>(kind, p->BN, p->stages); break;
+        default: p->stages = pick_stages<16>(kind, p->BN, want_s); p->smem_bytes = smem_for<16>(kind, p->BN, p->stages); break;
+    }
+    p->n_acc = (p->persist && 2 * p->BN <= 512) ? 2 : 1;
+    p->tmem_cols = 32;
+    while (p->tmem_cols < p->n_acc * p->BN) p->tmem_cols *= 2;
+}
+
 // Kernel choice and tiling.
 void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->path_tc = 0;
@@ -200,45 +245,14 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     const char* pe = std::getenv("CCV3D_PAIR");
     p->pair = (p->BN / p->n_sub) >= 32 ? 1 : 0;
     if (pe != nullptr) p->pair = std::atoi(pe) != 0 && (p->BN / p->n_sub) >= 32;
-    // Persistent stream-K on CTA pairs (opt-in: CCV3D_PERSIST=1) when every
-    // output frame has an active tap and the frames fit the schedule table.
-    // Measured on B200 it is slower than one launch of pair tiles on every
-    // decoder signature: the calls are bound by aggregate L2->SM traffic,
-    // which spreading the k-blocks over all SM pairs does not reduce.
+    p->path_tc_candidate = 1;
+    // Persistent stream-K on CTA pairs (opt-in: CCV3D_PERSIST=1).  Measured
+    // on B200 it is slower than one launch of pair tiles on every decoder
+    // signature: the calls are bound by aggregate L2->SM traffic, which
+    // spreading the k-blocks over all SM pairs does not reduce.
     p->persist = 0;
-    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
-    const int frames = d.N * p->T_o;
-    if (p->pair && frames <= kMaxFrames && env_int("CCV3D_PERSIST") > 0) {
-        bool all_active = true;
-        long long acc = 0;
-        const long long tiles_per_frame =
-            (long long)((p->tiles_x * p->tiles_y + 1) / 2) * p->tiles_n;
-        for (int f = 0; f < frames; ++f) {
-            const int o = f % p->T_o;
-            int a = 0;
-            for (int k = 0; k < d.kt; ++k) a += (o >= p->o_l[k] && o < p->o_h[k]) ? 1 : 0;
-            all_active = all_active && a > 0;
-            p->frame_start[f] = acc;
-            acc += tiles_per_frame * a * per_tap;
-        }
-        p->frame_start[frames] = acc;
-        p->sk_total = acc;
-        p->persist = all_active ? 1 : 0;
-    }
-    const int kind = p->persist ? 2 : p->pair;
-    // Short reductions (few k-blocks per tile) are dominated by each tile's
-    // fill and epilogue: without the persistent kernel, keep the ring small
-    // enough for 3 CTAs per SM so one CTA's epilogue overlaps the others.
-    int want_s = env_int("CCV3D_STAGES");
-    if (want_s == 0 && !p->persist && 3 * per_tap <= 96) want_s = 4;
-    switch (p->BK) {
-        case 64: p->stages = pick_stages<64>(kind, p->BN, want_s); p->smem_bytes = smem_for<64>(kind, p->BN, p->stages); break;
-        case 32: p->stages = pick_stages<32>(kind, p->BN, want_s); p->smem_bytes = smem_for<32>(kind, p->BN, p->stages); break;
-        default: p->stages = pick_stages<16>(kind, p->BN, want_s); p->smem_bytes = smem_for<16>(kind, p->BN, p->stages); break;
-    }
-    p->n_acc = (p->persist && 2 * p->BN <= 512) ? 2 : 1;
-    p->tmem_cols = 32;
-    while (p->tmem_cols < p->n_acc * p->BN) p->tmem_cols *= 2;
+    if (env_int("CCV3D_PERSIST") > 0) setup_persistent(d, p);
+    size_tc(d, p);
     p->path_tc = 1;
 }
 
@@ -441,6 +455,37 @@ ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const void* cache, const v
     return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
 }
 
+// Argument checks of a forward call against its plan (no device work).
+ccv3d_status check_call(const ccv3d_plan_s* p, const void* x, const void* cache, const void* w,
+                        const void* bias, const void* out, const void* nc, const int stride[2],
+                        const int pad[2], const int dilation[3]) {
+    const ccv3d_desc& d = p->d;
+    if (stride == nullptr || pad == nullptr || dilation == nullptr) return CCV3D_ERR_INVALID;
+    if (stride[0] != d.stride_h || stride[1] != d.stride_w || pad[0] != d.pad_h ||
+        pad[1] != d.pad_w || dilation[0] != d.dil_t || dilation[1] != d.dil_h ||
+        dilation[2] != d.dil_w)
+        return CCV3D_ERR_INVALID;
+    if (x == nullptr || w == nullptr || out == nullptr || (d.cache_len > 0 && cache == nullptr) ||
+        (d.has_bias && bias == nullptr) || (p->keep > 0 && nc == nullptr))
+        return CCV3D_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out) ||
+        (d.cache_len > 0 && !aligned16(cache)) || (nc != nullptr && !aligned16(nc)) ||
+        (d.has_bias && (reinterpret_cast<uintptr_t>(bias) % elt(d)) != 0))
+        return CCV3D_ERR_ALIGNMENT;
+    const size_t e = elt(d);
+    const size_t frame = (size_t)d.H * d.W * d.Cin * e;
+    const size_t x_bytes = (size_t)d.N * d.T_x * frame;
+    const size_t c_bytes = d.cache_len > 0 ? (size_t)d.N * d.cache_len * frame : 0;
+    const size_t nc_bytes = nc != nullptr ? (size_t)d.N * p->keep * frame : 0;
+    const size_t o_bytes = (size_t)d.N * p->T_o * p->H_o * p->W_o * d.Cout * e;
+    const size_t w_bytes = (size_t)d.Cout * d.kt * d.kh * d.kw * d.Cin * e;
+    if (overlaps(nc, nc_bytes, x, x_bytes) || overlaps(nc, nc_bytes, cache, c_bytes) ||
+        overlaps(out, o_bytes, x, x_bytes) || overlaps(out, o_bytes, cache, c_bytes) ||
+        overlaps(out, o_bytes, w, w_bytes) || overlaps(out, o_bytes, nc, nc_bytes))
+        return CCV3D_ERR_ALIAS;
+    return CCV3D_OK;
+}
+
 __global__ void wait_selftest_kernel(int* status, uint64_t limit_ns) {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
@@ -537,34 +582,12 @@ ccv3d_status ccv3d_forward(ccv3d_plan_t p, const void* x, const void* cache, con
                            const void* bias, void* out, void* nc, const int stride[2],
                            const int pad[2], const int dilation[3], cudaStream_t stream) {
     if (p == nullptr) return CCV3D_ERR_INVALID;
-    const ccv3d_desc& d = p->d;
     auto refuse = [&](ccv3d_status s) {
         p->errors.fetch_add(1, std::memory_order_relaxed);
         return s;
     };
-    if (stride == nullptr || pad == nullptr || dilation == nullptr) return refuse(CCV3D_ERR_INVALID);
-    if (stride[0] != d.stride_h || stride[1] != d.stride_w || pad[0] != d.pad_h ||
-        pad[1] != d.pad_w || dilation[0] != d.dil_t || dilation[1] != d.dil_h ||
-        dilation[2] != d.dil_w)
-        return refuse(CCV3D_ERR_INVALID);
-    if (x == nullptr || w == nullptr || out == nullptr || (d.cache_len > 0 && cache == nullptr) ||
-        (d.has_bias && bias == nullptr) || (p->keep > 0 && nc == nullptr))
-        return refuse(CCV3D_ERR_INVALID);
-    if (!aligned16(x) || !aligned16(w) || !aligned16(out) ||
-        (d.cache_len > 0 && !aligned16(cache)) || (nc != nullptr && !aligned16(nc)) ||
-        (d.has_bias && (reinterpret_cast<uintptr_t>(bias) % elt(d)) != 0))
-        return refuse(CCV3D_ERR_ALIGNMENT);
-    const size_t e = elt(d);
-    const size_t frame = (size_t)d.H * d.W * d.Cin * e;
-    const size_t x_bytes = (size_t)d.N * d.T_x * frame;
-    const size_t c_bytes = d.cache_len > 0 ? (size_t)d.N * d.cache_len * frame : 0;
-    const size_t nc_bytes = nc != nullptr ? (size_t)d.N * p->keep * frame : 0;
-    const size_t o_bytes = (size_t)d.N * p->T_o * p->H_o * p->W_o * d.Cout * e;
-    const size_t w_bytes = (size_t)d.Cout * d.kt * d.kh * d.kw * d.Cin * e;
-    if (overlaps(nc, nc_bytes, x, x_bytes) || overlaps(nc, nc_bytes, cache, c_bytes) ||
-        overlaps(out, o_bytes, x, x_bytes) || overlaps(out, o_bytes, cache, c_bytes) ||
-        overlaps(out, o_bytes, w, w_bytes) || overlaps(out, o_bytes, nc, nc_bytes))
-        return refuse(CCV3D_ERR_ALIAS);
+    const ccv3d_status chk = check_call(p, x, cache, w, bias, out, nc, stride, pad, dilation);
+    if (chk != CCV3D_OK) return refuse(chk);
     if (p->d_status == nullptr) return refuse(CCV3D_ERR_CUDA);
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return refuse(CCV3D_ERR_INVALID);
@@ -615,6 +638,8 @@ const char* ccv3d_strerror(ccv3d_status s) {
         case CCV3D_ERR_ALIAS: return "output buffer overlaps an input";
         case CCV3D_ERR_CUDA: return "CUDA error";
         case CCV3D_ERR_TIMEOUT: return "bounded device wait timed out";
+        case CCV3D_ERR_SCRATCH_LIMIT:
+            return "call needs more device scratch than the no-allocation entry point holds";
     }
     return "unknown status";
 }
@@ -636,4 +661,74 @@ ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream)
     return v == 0 ? CCV3D_ERR_CUDA : CCV3D_OK;
 }
 
+
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// ccv3d_forward_noalloc: the persistent stream-K kernel with its scratch in a
+// static device array instead of plan-owned memory.  The array's name is a
+// host-side stand-in in host code; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CCV3D_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocDevices = 64;
+constexpr size_t kNoallocStatusBytes = 256;  // status word, padded; then the flags
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocDevices];
+std::atomic<unsigned> g_noalloc_calls[kNoallocDevices];
+
+ccv3d_status noalloc_scratch(int dev, void** out) {
+    if (dev < 0 || dev >= kNoallocDevices) return CCV3D_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return CCV3D_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return CCV3D_OK;
+}
+
+}  // namespace
+
+extern "C" ccv3d_status ccv3d_forward_noalloc(const ccv3d_desc* desc, const void* x,
+                                              const void* cache, const void* w,
+                                              const void* bias, void* out, void* nc,
+                                              const int stride[2], const int pad[2],
+                                              const int dilation[3], cudaStream_t stream) {
+    if (desc == nullptr) return CCV3D_ERR_INVALID;
+    ccv3d_plan_s p{};  // host stack only
+    p.d = *desc;
+    ccv3d_status st = compute_intervals(*desc, &p);
+    if (st != CCV3D_OK) return st;
+    choose_path(*desc, &p);
+    if (!p.path_tc || !setup_persistent(*desc, &p)) return CCV3D_ERR_UNSUPPORTED;
+    size_tc(*desc, &p);
+    st = check_call(&p, x, cache, w, bias, out, nc, stride, pad, dilation);
+    if (st != CCV3D_OK) return st;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return CCV3D_ERR_CUDA;
+    }
+    size_persistent(&p, true);
+    if (kNoallocStatusBytes + p.scratch_bytes > (size_t)CCV3D_NOALLOC_SCRATCH_BYTES)
+        return CCV3D_ERR_SCRATCH_LIMIT;
+    void* base = nullptr;
+    st = noalloc_scratch(dev, &base);
+    if (st != CCV3D_OK) return st;
+    p.device = dev;
+    p.d_status = static_cast<int*>(base);
+    p.scratch = static_cast<unsigned char*>(base) + kNoallocStatusBytes;
+    p.epoch.store(g_noalloc_calls[dev].fetch_add(1));
+    if (cudaMemsetAsync(p.d_status, 0, sizeof(int), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CCV3D_ERR_CUDA;
+    }
+    return run_tc(&p, x, cache, w, bias, out, nc, stream);
+}

@@ -71,7 +71,9 @@ typedef enum {
     CCV3D_ERR_ALIAS = 5,        /* new_cache overlaps x or cache, or out
                                    overlaps an input */
     CCV3D_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
-    CCV3D_ERR_TIMEOUT = 7       /* a bounded device-side wait ran out */
+    CCV3D_ERR_TIMEOUT = 7,      /* a bounded device-side wait ran out */
+    CCV3D_ERR_SCRATCH_LIMIT = 8 /* ccv3d_forward_noalloc: the call needs more
+                                   device scratch than its fixed array holds */
 } ccv3d_status;
 
 /* Conv3D call signature.  Sizes are in elements/frames. */
@@ -162,6 +164,48 @@ CCV3D_API ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t plan, size_t* out_bytes,
  * reported it, and the context stays usable), CCV3D_OK if the wait completed
  * (a defect), or CCV3D_ERR_CUDA. */
 CCV3D_API ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Forward call that allocates nothing.
+ *
+ * The paper has no counterpart to this entry point: it serves callers that
+ * must not allocate device memory, directly or through this library -- code
+ * that runs inside a caching allocator's own hooks, or under a serving
+ * runtime that owns the whole device-memory budget and forbids cudaMalloc /
+ * cudaFree (and the device-wide synchronisation cudaFree implies) outside its
+ * pool.  Such a caller cannot create a plan (ccv3d_plan allocates the plan's
+ * status block and, for split tiles, its scratch), so this call takes the
+ * signature itself and plans on the host stack each time.
+ *
+ * It runs the persistent stream-K CTA-pair kernel.  That kernel's device
+ * scratch -- a status word, the split-tile flags and the fp32 partial tiles --
+ * lives in one static array of CCV3D_NOALLOC_SCRATCH_BYTES bytes compiled into
+ * this library: every GPU that loads the library holds the array until the
+ * process exits, whether or not it calls this function.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.
+ *
+ * All calls share the array and it keeps what the last call left there, so
+ * calls that overlap on the GPU (other streams, other host threads) race:
+ * the caller must order them.  Each call clears the status word before its
+ * launch; the split-tile flags carry a per-device call number, so stale flags
+ * from earlier calls are never mistaken for this call's.
+ *
+ * Arguments and layouts are those of ccv3d_forward, with the signature in
+ * `desc` instead of a plan.  Covered: bf16 signatures that run on the
+ * CTA-pair tensor-core path with at most 64 (n, o) output frames, each with
+ * an active tap; others return CCV3D_ERR_UNSUPPORTED.  A call whose scratch
+ * (2 x pairs x 128 x Cout-tile x 4 bytes, plus flags) would not fit returns
+ * CCV3D_ERR_SCRATCH_LIMIT before any device work.  Other errors as
+ * ccv3d_forward; a device-side wait that runs out is recorded in the shared
+ * status word, which this entry point does not read back (it never
+ * synchronises the host).  No device memory is allocated or freed. */
+#define CCV3D_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+CCV3D_API ccv3d_status ccv3d_forward_noalloc(const ccv3d_desc* desc, const void* x,
+                                             const void* cache, const void* w,
+                                             const void* bias, void* out, void* new_cache,
+                                             const int stride[2], const int pad[2],
+                                             const int dilation[3], cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -116,7 +116,7 @@ def test_null_arguments():
         ccv3d.CCV3D_ERR_INVALID
     assert ccv3d.ccv3d_plan_path(None)["tc"] is False
     ccv3d.ccv3d_destroy(None)  # ignored
-    for s in range(8):
+    for s in range(9):
         assert ccv3d.ccv3d_strerror(s)
 
 
