@@ -3,8 +3,8 @@
 Shapes only: no arithmetic of the operator lives here.  Every workload is a
 single call signature (plus the seeded value recipe) in NTHWC layout, N=1.
 The value recipe follows the decoder study's synthetic-latent practice
-("Cache-Aware Conv3D Lowering Across Embedded World-Model Decoders", Sec. 5:
-decoder-compatible synthetic BF16 latents, batch size 1): activations
+("Cache-Aware Conv3D Lowering Across Embedded World-Model Decoders", evaluation
+setup of Tab. 2: decoder-compatible synthetic BF16 latents, batch size 1): activations
 N(0,1), weights N(0, 1/(Cin*kt*kh*kw)) (variance), bias N(0, sigma_b^2).
 """
 from __future__ import annotations
