@@ -214,35 +214,73 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError(f"device status after timing: {status}")
 
     # ---- end to end through the C ABI with host buffers -------------------
-    x, c, w, b, out, nc = sets[0]
-    hx = torch.empty(x.shape, dtype=dt, pin_memory=True).copy_(x)
-    hc = torch.empty(c.shape, dtype=dt, pin_memory=True).copy_(c) if c is not None else None
-    ho = torch.empty(out.shape, dtype=dt, pin_memory=True)
-    hn = torch.empty(nc.shape, dtype=dt, pin_memory=True) if nc is not None else None
+    # Each step uploads its x and cache from pinned host memory, runs the call
+    # and reads out and new_cache back to pinned host memory.  Steps are
+    # pipelined over three streams with two device buffer sets, as a
+    # streaming decoder runs them: step i+1's upload and step i-1's download
+    # overlap step i's compute (PCIe is full duplex).
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
-    h2d = hx.numel() * hx.element_size() + (hc.numel() * hc.element_size() if hc is not None else 0)
-    d2h = ho.numel() * ho.element_size() + (hn.numel() * hn.element_size() if hn is not None else 0)
+    w0, b0 = sets[0][2], sets[0][3]
+    bufs = []
+    for i in range(2):
+        x, c, _, _, out, nc = sets[i]
+        bufs.append((x, c, out, nc))
+    x0, c0, out0, nc0 = bufs[0]
+    hx = [torch.empty(x0.shape, dtype=dt, pin_memory=True).copy_(x0) for _ in range(2)]
+    hc = ([torch.empty(c0.shape, dtype=dt, pin_memory=True).copy_(c0) for _ in range(2)]
+          if c0 is not None else [None, None])
+    ho = [torch.empty(out0.shape, dtype=dt, pin_memory=True) for _ in range(2)]
+    hn = ([torch.empty(nc0.shape, dtype=dt, pin_memory=True) for _ in range(2)]
+          if nc0 is not None else [None, None])
+    h2d = x0.numel() * x0.element_size() + (c0.numel() * c0.element_size() if c0 is not None else 0)
+    d2h = out0.numel() * out0.element_size() + (nc0.numel() * nc0.element_size() if nc0 is not None else 0)
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
 
-    def e2e_step():
-        x.copy_(hx, non_blocking=True)
-        if hc is not None:
-            c.copy_(hc, non_blocking=True)
-        plan.forward(x, c, w, b, out, nc, stream)
-        ho.copy_(out, non_blocking=True)
-        if hn is not None:
-            hn.copy_(nc, non_blocking=True)
+    def e2e_run(steps, start_ev=None, end_ev=None):
+        uploaded = [None, None]   # event: buffer i's inputs are on the device
+        computed = [None, None]   # event: buffer i's outputs are written
+        freed = [None, None]      # event: buffer i's outputs are read back
+        if start_ev is not None:
+            start_ev.record(stream)
+            s_up.wait_stream(stream)
+            s_down.wait_stream(stream)
+        for i in range(steps):
+            k = i % 2
+            x, c, out, nc = bufs[k]
+            with torch.cuda.stream(s_up):
+                if computed[k] is not None:
+                    s_up.wait_event(computed[k])  # previous call on this buffer set read x/cache
+                x.copy_(hx[k], non_blocking=True)
+                if c is not None:
+                    c.copy_(hc[k], non_blocking=True)
+                uploaded[k] = ev()
+                uploaded[k].record(s_up)
+            stream.wait_event(uploaded[k])
+            if freed[k] is not None:
+                stream.wait_event(freed[k])  # out/new_cache of buffer set k were read back
+            plan.forward(x, c, w0, b0, out, nc, stream)
+            computed[k] = ev()
+            computed[k].record(stream)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(computed[k])
+                ho[k].copy_(out, non_blocking=True)
+                if nc is not None:
+                    hn[k].copy_(nc, non_blocking=True)
+                freed[k] = ev()
+                freed[k].record(s_down)
+        if end_ev is not None:
+            stream.wait_stream(s_up)
+            stream.wait_stream(s_down)
+            end_ev.record(stream)
 
-    for _ in range(3):
-        e2e_step()
+    e2e_run(3)
     torch.cuda.synchronize()
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         tdist.barrier()
     torch.cuda.synchronize()
-    ea.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    eb.record(stream)
+    e2e_run(e2e_steps, ea, eb)
     torch.cuda.synchronize()
     e2e_ms = ea.elapsed_time(eb)
 
@@ -285,6 +323,7 @@ def run_gpu(args, rank, world, local_rank):
             "plan": "one plan per signature, made before timing",
             "planner_us": round(plan_us, 1),
             "path": "tcgen05" if plan.path["tc"] else "simt",
+            "kernel": plan.kernel,
             "tile": [plan.path["tile_m"], plan.path["tile_n"]],
         },
         "us_per_call_median": round(statistics.median(per) * 1e3, 2),
@@ -302,14 +341,89 @@ def run_gpu(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "steps": e2e_steps,
-                "what": "pinned host x+cache -> device, ccv3d_forward, out+new_cache -> "
-                        "pinned host; weights resident"},
+                "what": "per step: pinned host x+cache -> device, ccv3d_forward, "
+                        "out+new_cache -> pinned host; weights resident; steps pipelined "
+                        "over upload/compute/download streams"},
         "gpu_launches": int(launches),
         "clocks": csum,
     }
+    if args.sequence:
+        line["decode17"] = run_sequence(args, dev)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(conv, args.cpu_seconds)
     return line
+
+
+# ------------------------------------------------- decode-sequence leg
+def run_sequence(args, dev):
+    """Time the synthetic 17-frame decode: 164 calls over 28 signatures, each
+    module's cache threaded from chunk to chunk (ping-pong buffers), all on one
+    stream.  Plans are made once per signature.  Inputs are seeded N(0,1)
+    frames generated on the device (timing only; parity is in the tests)."""
+    import torch
+    from causal_conv3d_video_b200 import ccv3d
+
+    calls = workloads.decode17_schedule()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    plans, frames, outs, mods = {}, {}, {}, {}
+    flops = 0.0
+    for call in calls:
+        c = call.conv
+        sig = workloads.signature(c)
+        if sig not in plans:
+            plans[sig] = ccv3d.Plan(ccv3d.desc_for(c))
+        plan = plans[sig]
+        flops += algorithmic(c, plan.intervals)[0]
+        xs = (1, c.T_x, c.H, c.W, c.Cin)
+        if xs not in frames:
+            frames[xs] = torch.randn(xs, generator=gen, device=dev).to(torch.bfloat16)
+        os_ = plan.out_shape()
+        if os_ not in outs:
+            outs[os_] = torch.empty(os_, dtype=torch.bfloat16, device=dev)
+        if call.module not in mods:
+            w = (torch.randn((c.Cout, c.kt, c.kh, c.kw, c.Cin), generator=gen, device=dev)
+                 / (c.Cin * c.kt * c.kh * c.kw) ** 0.5).to(torch.bfloat16)
+            b = (0.02 * torch.randn((c.Cout,), generator=gen, device=dev)).to(torch.bfloat16)
+            cs = (1, 2, c.H, c.W, c.Cin)
+            caches = [torch.randn(cs, generator=gen, device=dev).to(torch.bfloat16)
+                      for _ in range(2)]
+            mods[call.module] = [w, b, caches, 0]
+    stream = torch.cuda.current_stream(dev)
+
+    def one_pass():
+        for m in mods.values():
+            m[3] = 0
+        for call in calls:
+            c = call.conv
+            plan = plans[workloads.signature(c)]
+            w, b, caches, cur = mods[call.module]
+            cache = caches[cur][:, :c.cache_len] if c.cache_len > 0 else None
+            keep = plan.sizes["new_cache_frames"]
+            nc = caches[1 - cur][:, :keep]
+            plan.forward(frames[(1, c.T_x, c.H, c.W, c.Cin)], cache, w, b,
+                         outs[plan.out_shape()], nc, stream)
+            mods[call.module][3] = 1 - cur
+
+    for _ in range(2):
+        one_pass()
+    torch.cuda.synchronize()
+    passes = max(1, args.sequence_passes)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(passes):
+        one_pass()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    ms = ea.elapsed_time(eb) / passes
+    for plan in plans.values():
+        if plan.status() != 0:
+            raise RuntimeError("device status after the decode sequence")
+    kernels = sorted({p.kernel for p in plans.values()})
+    return {"calls": len(calls), "signatures": len(plans), "ms_per_sequence": round(ms, 3),
+            "tflops": round(flops / (ms / 1e3) / 1e12, 2), "gflop_per_sequence": round(flops / 1e9, 1),
+            "passes": passes, "kernels": kernels,
+            "what": "164-call synthetic 17-frame decode, caches threaded, one stream"}
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -414,6 +528,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sequence", action="store_true",
+                    help="also time the 164-call synthetic decode sequence")
+    ap.add_argument("--sequence-passes", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -24,7 +24,8 @@ CCV3D_MAX_KT = 3
 # every symbol include/ccv3d.h declares
 EXPORTED = ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_plan_path", "ccv3d_forward",
             "ccv3d_get_stats", "ccv3d_get_status", "ccv3d_destroy", "ccv3d_strerror",
-            "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout", "ccv3d_forward_noalloc")
+            "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout", "ccv3d_forward_noalloc",
+            "ccv3d_plan_kernel")
 CCV3D_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -64,6 +65,8 @@ def _load():
     lib.ccv3d_destroy.restype = None
     lib.ccv3d_strerror.argtypes = [ctypes.c_int]
     lib.ccv3d_strerror.restype = ctypes.c_char_p
+    lib.ccv3d_plan_kernel.argtypes = [vp]
+    lib.ccv3d_plan_kernel.restype = ctypes.c_char_p
     lib.ccv3d_plan_sizes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t),
                                      ctypes.POINTER(ctypes.c_size_t), ip]
     lib.ccv3d_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
@@ -125,6 +128,10 @@ def ccv3d_plan_path(plan):
     tm, tn = ctypes.c_int(), ctypes.c_int()
     tc = lib.ccv3d_plan_path(plan, ctypes.byref(tm), ctypes.byref(tn))
     return {"tc": bool(tc == 1), "tile_m": tm.value, "tile_n": tn.value}
+
+
+def ccv3d_plan_kernel(plan) -> str:
+    return lib.ccv3d_plan_kernel(plan).decode()
 
 
 def ccv3d_plan_sizes(plan):
@@ -220,6 +227,7 @@ class Plan:
         self.intervals = ccv3d_plan_intervals(self.handle)
         self.sizes = ccv3d_plan_sizes(self.handle)
         self.path = ccv3d_plan_path(self.handle)
+        self.kernel = ccv3d_plan_kernel(self.handle)
 
     @property
     def stride(self):

@@ -22,6 +22,7 @@
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
 #include "conv_tc2.cuh"
+#include "conv_tc2h.cuh"
 #include "conv_tcp.cuh"
 #include "params.h"
 
@@ -36,6 +37,8 @@ struct ccv3d_plan_s {
     int BK, BN, n_sub, box_h, box_w, tiles_x, tiles_y, tiles_n, stages, tmem_cols;
     int pair;  // 1: CTA-pair kernel (M = 256 per pair), 0: one CTA per 128-row tile
     int persist;  // 1: persistent stream-K pair kernel
+    int halo;     // 1: pair kernel loading each input row strip once per (tap, channel block)
+    int halo_w;   // halo: pixels per strip
     int G, n_acc;  // persistent: CTA pairs launched, TMEM accumulator buffers
     long long frame_start[kMaxFrames + 1], sk_total;
     size_t smem_bytes;
@@ -108,11 +111,20 @@ ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
 
 constexpr size_t kSmemBudget = 225 * 1024;
 
-// kind: 0 one CTA per tile, 1 CTA pair, 2 persistent CTA pair
+// kind: 0 one CTA per tile, 1 CTA pair, 2 persistent CTA pair (3: halo pair,
+// sized by halo_smem_for)
 template <int BK>
 size_t smem_for(int kind, int bn, int stages) {
     return kind == 2 ? tcp_smem_bytes<BK>(bn, stages)
                      : (kind == 1 ? tc2_smem_bytes<BK>(bn, stages) : tc_smem_bytes<BK>(bn, stages));
+}
+
+size_t halo_smem_for(int bk, int bn, int stages, int kh, int kw, int halo_w) {
+    switch (bk) {
+        case 64: return tc2h_smem_bytes<64>(bn, stages, kh, kw, halo_w);
+        case 32: return tc2h_smem_bytes<32>(bn, stages, kh, kw, halo_w);
+        default: return tc2h_smem_bytes<16>(bn, stages, kh, kw, halo_w);
+    }
 }
 
 template <int BK>
@@ -131,6 +143,8 @@ void set_smem_attrs() {
         cudaFuncSetAttribute(conv_tc2_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaFuncSetAttribute(conv_tcp_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
+        cudaFuncSetAttribute(conv_tc2h_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaGetLastError();
     });
@@ -168,6 +182,7 @@ int env_int(const char* name) {
 // the schedule table.  Sets p->persist; returns it.
 bool setup_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->persist = 0;
+    p->halo = 0;  // the persistent kernel has its own (non-halo) stages
     if (!p->path_tc_candidate || !p->pair) return false;
     const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
     const int frames = d.N * p->T_o;
@@ -205,6 +220,32 @@ void size_tc(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->n_acc = (p->persist && 2 * p->BN <= 512) ? 2 : 1;
     p->tmem_cols = 32;
     while (p->tmem_cols < p->n_acc * p->BN) p->tmem_cols *= 2;
+}
+
+// Halo variant of the pair kernel (opt-in: CCV3D_HALO=1): tiles of one
+// 128-pixel output row at unit W stride, when a stage (kh strips + kh*kw
+// weight tiles) fits at least 3 deep; prefers the widest channel block that
+// does.  It halves the L2->SM operand bytes of the thin-channel full-size
+// calls, but its large stages leave room for one CTA per SM, and on B200 the
+// plain pair kernel with four CTAs per SM is faster on those calls.
+void setup_halo(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    p->halo = 0;
+    if (!p->pair || p->persist || env_int("CCV3D_HALO") <= 0) return;
+    if (p->box_w != 128 || p->box_h != 1 || d.stride_w != 1) return;
+    const int halo_w = 128 + (d.kw - 1) * d.dil_w;
+    if (halo_w > 256) return;
+    for (int bk : {64, 32, 16}) {
+        if (d.Cin % bk != 0) continue;
+        int s = 8;
+        while (s >= 3 && halo_smem_for(bk, p->BN, s, d.kh, d.kw, halo_w) > kSmemBudget) --s;
+        if (s < 3) continue;
+        p->halo = 1;
+        p->halo_w = halo_w;
+        p->BK = bk;
+        p->stages = s;
+        p->smem_bytes = halo_smem_for(bk, p->BN, s, d.kh, d.kw, halo_w);
+        return;
+    }
 }
 
 // Kernel choice and tiling.
@@ -253,6 +294,7 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->persist = 0;
     if (env_int("CCV3D_PERSIST") > 0) setup_persistent(d, p);
     size_tc(d, p);
+    setup_halo(d, p);
     p->path_tc = 1;
 }
 
@@ -294,9 +336,13 @@ ccv3d_status encode_act(CUtensorMap* m, const void* base, int frames, const ccv3
                                 (cuuint64_t)frames};
     const cuuint64_t strides[3] = {(cuuint64_t)d.Cin * 2, (cuuint64_t)d.W * d.Cin * 2,
                                    (cuuint64_t)d.H * d.W * d.Cin * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)p->BK, (cuuint32_t)(p->box_w * d.stride_w),
-                               (cuuint32_t)(p->box_h * d.stride_h), 1};
-    const cuuint32_t estr[4] = {1, (cuuint32_t)d.stride_w, (cuuint32_t)d.stride_h, 1};
+    // halo kernel: one input row strip of halo_w pixels; otherwise the
+    // shifted, strided box of box_h x box_w output pixels
+    const cuuint32_t box[4] = {(cuuint32_t)p->BK,
+                               (cuuint32_t)(p->halo ? p->halo_w : p->box_w * d.stride_w),
+                               (cuuint32_t)(p->halo ? 1 : p->box_h * d.stride_h), 1};
+    const cuuint32_t estr[4] = {1, p->halo ? 1u : (cuuint32_t)d.stride_w,
+                                p->halo ? 1u : (cuuint32_t)d.stride_h, 1};
     const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -323,6 +369,27 @@ ccv3d_status encode_w(CUtensorMap* m, const void* base, const ccv3d_desc& d,
                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+// Output as a 4-D tensor [N*T_o, H_o, W_o, Cout] for the epilogue's tensor
+// stores: boxes of (16/32/64 channels) x box_w x box_h pixels of one frame,
+// swizzled like the staging buffer; rows and channels past the tensor are
+// clipped by the hardware.
+ccv3d_status encode_out(CUtensorMap* m, void* base, const ccv3d_desc& d, const ccv3d_plan_s* p) {
+    const int kch = out_block_channels(p->BN);
+    const cuuint64_t dims[4] = {(cuuint64_t)d.Cout, (cuuint64_t)p->W_o, (cuuint64_t)p->H_o,
+                                (cuuint64_t)d.N * p->T_o};
+    const cuuint64_t strides[3] = {(cuuint64_t)d.Cout * 2, (cuuint64_t)p->W_o * d.Cout * 2,
+                                   (cuuint64_t)p->H_o * p->W_o * d.Cout * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)kch, (cuuint32_t)p->box_w, (cuuint32_t)p->box_h, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = kch == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : kch == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box,
+                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
 }
 
@@ -354,7 +421,9 @@ Taps make_taps(const ccv3d_plan_s* p) {
 template <int BK>
 cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s) {
     set_smem_attrs<BK>();
-    if (kind == 2)
+    if (kind == 3)
+        conv_tc2h_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
+    else if (kind == 2)
         conv_tcp_kernel<BK><<<grid, kTcpThreads, smem, s>>>(prm);
     else if (kind == 1)
         conv_tc2_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
@@ -372,6 +441,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     ccv3d_status st = encode_act(&prm.tmap_x, x, d.N * d.T_x, d, p);
     if (st == CCV3D_OK && d.cache_len > 0) st = encode_act(&prm.tmap_c, cache, d.N * d.cache_len, d, p);
     if (st == CCV3D_OK) st = encode_w(&prm.tmap_w, w, d, p);
+    if (st == CCV3D_OK) st = encode_out(&prm.tmap_out, out, d, p);
     if (st != CCV3D_OK) return st;
     prm.bias = d.has_bias ? static_cast<const uint16_t*>(bias) : nullptr;
     prm.out = static_cast<uint16_t*>(out);
@@ -414,7 +484,8 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     const long long units = p->pair ? grid / 2 : grid;
     const long long wave = p->pair ? 74 : 148;
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
-    const int kind = p->persist ? 2 : p->pair;
+    const int kind = p->halo ? 3 : (p->persist ? 2 : p->pair);
+    prm.halo_w = p->halo_w;
     cudaError_t e;
     switch (p->BK) {
         case 64: e = launch_tc<64>(prm, kind, (int)grid, p->smem_bytes, stream); break;
@@ -566,6 +637,14 @@ int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
     if (tile_m) *tile_m = p->path_tc ? kTileM * (p->pair ? 2 : 1) : 0;
     if (tile_n) *tile_n = p->path_tc ? p->BN : 0;
     return p->path_tc;
+}
+
+const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
+    if (p == nullptr) return "";
+    if (!p->path_tc) return "simt";
+    if (p->halo) return "tc_pair_halo";
+    if (p->persist) return "tc_persistent";
+    return p->pair ? "tc_pair" : "tc_single";
 }
 
 ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t p, size_t* out_bytes, size_t* nc_bytes,

@@ -14,13 +14,15 @@
 //   warp 0     TMA producer (one lane): A box + B box per pipeline stage
 //   warp 1     TMEM owner; one lane issues tcgen05.mma (M=128, N=BN, K=16)
 //   warps 2-5  copy a slice of new_cache while the GEMM runs, then the
-//              epilogue: tcgen05.ld -> + bias (fp32) -> bf16 (RNE) -> global
+//              epilogue: tcgen05.ld -> + bias (fp32) -> bf16 (RNE) -> swizzled
+//              shared-memory stage (the idle ring) -> TMA tensor store
 // Every mbarrier wait is bounded (mbar_wait); a timeout is recorded in the
 // status block and the roles drain and exit instead of hanging.
 #pragma once
 #include <cuda_bf16.h>
 
 #include "cache_copy.cuh"
+#include "epilogue.cuh"
 #include "kwalk.cuh"
 #include "params.h"
 #include "ptx.cuh"
@@ -33,11 +35,19 @@ struct TcSmem {
     static constexpr int kABytes = kTileM * kRowBytes;  // one A stage
 };
 
+// Bytes of the operand ring, which the epilogue reuses to stage its
+// 128 x bn bf16 output tile (1024-byte multiple).
+__host__ __device__ constexpr size_t ring_bytes(size_t ring, int bn) {
+    const size_t stage_out = (size_t)kTileM * bn * 2;
+    const size_t r = ring > stage_out ? ring : stage_out;
+    return (r + 1023) / 1024 * 1024;
+}
+
 // Dynamic shared memory needed for `stages` stages of an N=BN tile.
 template <int BK>
 __host__ __device__ constexpr size_t tc_smem_bytes(int bn, int stages) {
     return 1024 /* alignment slack */ +
-           (size_t)stages * (TcSmem<BK>::kABytes + (size_t)bn * TcSmem<BK>::kRowBytes) +
+           ring_bytes((size_t)stages * (TcSmem<BK>::kABytes + (size_t)bn * TcSmem<BK>::kRowBytes), bn) +
            (size_t)(2 * stages + 1) * 8 /* mbarriers */ + 16 /* tmem slot */ +
            (size_t)bn * 4 /* bias */;
 }
@@ -57,7 +67,8 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
     const int kBs = BNs * kRow;
     uint8_t* sA = smem;
     uint8_t* sB = smem + (size_t)stages * kA;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kB);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(
+        smem + ring_bytes((size_t)stages * (kA + kB), BN));
     uint64_t* empty_bar = full_bar + stages;
     uint64_t* acc_bar = empty_bar + stages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
@@ -182,37 +193,15 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
 
         const bool ok = mbar_wait(smem_u32(acc_bar), 0, p.status, p.wait_limit_ns);
         tc_fence_after();
+        // the ring is idle once the accumulator is complete: stage the output there
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int row = q * 32 + lane;
-        const int y = ty * p.box_h + row / p.box_w;
-        const int x = tx * p.box_w + row % p.box_w;
-        const bool valid = ok && y < p.H_o && x < p.W_o;
-        uint16_t* orow = p.out + ((((long long)n * p.T_o + o) * p.H_o + y) * p.W_o + x) *
-                                     (long long)p.Cout;
+        const int frame = n * p.T_o + o;
+        const int x0 = tx * p.box_w, y0 = ty * p.box_h, co0 = n_tile * BN;
         const bool have_acc = iters > 0;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-            tmem_ld_wait();
-            const int co = n_tile * BN + c0;
-            if (!valid || co >= p.Cout) continue;
-            uint32_t packed[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float a0 = (have_acc ? __uint_as_float(v[2 * j]) : 0.f) + bias_s[c0 + 2 * j];
-                const float a1 =
-                    (have_acc ? __uint_as_float(v[2 * j + 1]) : 0.f) + bias_s[c0 + 2 * j + 1];
-                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-                packed[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            if (co + 16 <= p.Cout) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + co);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            } else {
-                for (int j = 0; j < 16 && co + j < p.Cout; ++j)
-                    orow[co + j] = (uint16_t)(packed[j >> 1] >> ((j & 1) * 16));
-            }
+        switch (out_block_channels(BN)) {
+            case 64: epilogue_store<64>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, ok); break;
+            case 32: epilogue_store<32>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, ok); break;
+            default: epilogue_store<16>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, ok); break;
         }
     }
 

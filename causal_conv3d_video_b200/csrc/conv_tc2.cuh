@@ -11,7 +11,8 @@
 //     even producer posts the byte count for the pair), and the even CTA's
 //     tcgen05.commit releases the stage on both CTAs' "empty" barriers;
 //   * each CTA holds its 128 accumulator rows in its own TMEM and runs its own
-//     epilogue (bias, bf16, store) and its slice of the new_cache copy.
+//     epilogue (bias, bf16, TMA store staged in its idle ring) and its slice
+//     of the new_cache copy.
 // Per SM this halves the weight bytes pulled from L2 per FLOP, the operand
 // that dominates on the wide-Cout decoder signatures.  No load is
 // multicast.  All waits are bounded.
@@ -20,6 +21,7 @@
 
 #include "cache_copy.cuh"
 #include "conv_tc.cuh"
+#include "epilogue.cuh"
 #include "kwalk.cuh"
 #include "params.h"
 #include "ptx.cuh"
@@ -29,7 +31,9 @@ namespace ccv3d {
 template <int BK>
 __host__ __device__ constexpr size_t tc2_smem_bytes(int bn, int stages) {
     // per CTA: A box (128 rows) + half of the BN weight rows per stage
-    return 1024 + (size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes) +
+    return 1024 +
+           ring_bytes((size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes),
+                      bn) +
            (size_t)(2 * stages + 1) * 8 + 16 + (size_t)bn * 4;
 }
 
@@ -49,7 +53,8 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
     const int kBh = hB * kRow;
     uint8_t* sA = smem;
     uint8_t* sB = smem + (size_t)stages * kA;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kBc);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(
+        smem + ring_bytes((size_t)stages * (kA + kBc), BN));
     uint64_t* empty_bar = full_bar + stages;
     uint64_t* acc_bar = empty_bar + stages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
@@ -180,39 +185,17 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
 
         const bool ok = mbar_wait(smem_u32(acc_bar), 0, p.status, p.wait_limit_ns);
         tc_fence_after();
+        // every pair MMA has completed: neither CTA's ring is read any more,
+        // so this CTA stages its output rows there
         const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const int y = ty * p.box_h + row / p.box_w;
-        const int x = tx * p.box_w + row % p.box_w;
-        const bool valid = ok && y < p.H_o && x < p.W_o;
-        uint16_t* orow = p.out + ((((long long)n * p.T_o + o) * p.H_o + y) * p.W_o + x) *
-                                     (long long)p.Cout;
+        const int frame = n * p.T_o + o;
+        const int x0 = tx * p.box_w, y0 = ty * p.box_h, co0 = n_tile * BN;
         const bool have_acc = iters > 0;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-            tmem_ld_wait();
-            const int co = n_tile * BN + c0;
-            if (!valid || co >= p.Cout) continue;
-            uint32_t packed[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float a0 = (have_acc ? __uint_as_float(v[2 * j]) : 0.f) + bias_s[c0 + 2 * j];
-                const float a1 =
-                    (have_acc ? __uint_as_float(v[2 * j + 1]) : 0.f) + bias_s[c0 + 2 * j + 1];
-                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-                packed[j] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            if (co + 16 <= p.Cout) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + co);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (co + j < p.Cout)
-                        orow[co + j] = (uint16_t)(packed[j >> 1] >> ((j & 1) * 16));
-            }
+        const bool store = ok && ty < p.tiles_y;  // a box past the frame stores nothing
+        switch (out_block_channels(BN)) {
+            case 64: epilogue_store<64>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, store); break;
+            case 32: epilogue_store<32>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, store); break;
+            default: epilogue_store<16>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, store); break;
         }
     }
 

@@ -26,6 +26,7 @@
 #include "cache_copy.cuh"
 #include "conv_tc.cuh"
 #include "conv_tc2.cuh"
+#include "epilogue.cuh"
 #include "kwalk.cuh"
 #include "params.h"
 #include "ptx.cuh"
@@ -53,10 +54,6 @@ __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Named barrier over the four epilogue warps (barrier 1, 128 threads).
-__device__ __forceinline__ void epi_bar() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-}
 
 // One piece of a pair's range: pair tile `tile` (frame f, index in frame),
 // k-blocks [kb0, kb1) of its reduction of `iters` k-blocks.

@@ -47,6 +47,7 @@ struct __align__(64) TcParams {
     CUtensorMap tmap_x;      // x      as [N*T_x, H, W, Cin], box [BK, bw*s_w, bh*s_h, 1]
     CUtensorMap tmap_c;      // cache  as [N*|C|, H, W, Cin] (unused when |C| = 0)
     CUtensorMap tmap_w;      // weight as [Cout, kt*kh*kw, Cin], box [BK, 1, BN]
+    CUtensorMap tmap_out;    // out as [N*T_o, H_o, W_o, Cout], box [kCh, box_w, box_h, 1]
     const uint16_t* bias;    // bf16 [Cout] or null
     uint16_t* out;           // bf16 [N, T_o, H_o, W_o, Cout]
     int* status;
@@ -59,6 +60,7 @@ struct __align__(64) TcParams {
     int BN, n_sub, n_cb, stages, tmem_cols;
     int pairs_per_frame;     // CTA-pair kernel: ceil(tiles_x * tiles_y / 2)
     int rot_div;             // tiles (or pairs) over which K-start offsets are spread
+    int halo_w;              // halo kernel: pixels per input strip (128 + (kw-1)*d_w)
     StreamK sk;
     uint64_t wait_limit_ns;
 };

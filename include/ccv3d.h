@@ -127,6 +127,10 @@ CCV3D_API ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t plan, int* T_o, int* H_
  * when a CTA pair shares each MMA (cta_group::2), else 128 (may be NULL). */
 CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
 
+/* Name of the kernel the plan launches: "tc_pair_halo", "tc_pair",
+ * "tc_single", "tc_persistent" or "simt" (static string; "" for NULL). */
+CCV3D_API const char* ccv3d_plan_kernel(ccv3d_plan_t plan);
+
 /* Run one cached causal Conv3D call on `stream` (device pointers, layouts as
  * above).  stride = {s_h, s_w}, pad = {p_h, p_w}, dilation = {d_t, d_h, d_w}
  * must equal the plan's (the call signature of the paper's patched module).

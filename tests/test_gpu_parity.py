@@ -113,6 +113,25 @@ def test_small_tile_variants(c, env):
     _run_small(c, env=env)
 
 
+HALO = [
+    # one 128-pixel output row per tile: the input strip is loaded once per (tap, channel block)
+    Conv("h96_3x256", 96, 96, 3, 384, T_x=2, cache_len=1, sigma_b=0.1),    # 9 boxes: odd
+    Conv("h64_6x256", 64, 64, 6, 256, T_x=1, cache_len=2),
+    Conv("h32to48_3x200", 32, 48, 3, 200, T_x=3, cache_len=0),              # ragged row
+    Conv("h192to96_2x256", 192, 96, 2, 256, T_x=4, cache_len=2, sigma_b=0.1),
+    Conv("h64_dilw2", 64, 64, 4, 256, T_x=1, cache_len=2, pad=(2, 2), dilation=(1, 2, 2)),
+    Conv("h64_k3x1x1", 64, 128, 4, 256, T_x=1, cache_len=2, kh=1, kw=1, pad=(0, 0)),
+    Conv("h64_s2h", 64, 64, 9, 256, T_x=1, cache_len=2, stride=(2, 1)),
+]
+
+
+@pytest.mark.parametrize("halo", [1, 0], ids=["halo", "no_halo"])
+@pytest.mark.parametrize("c", HALO, ids=lambda c: c.name)
+def test_small_halo_strips(c, halo):
+    call, _ = _run_small(c, env={"CCV3D_HALO": halo})
+    assert (call.plan.kernel == "tc_pair_halo") == bool(halo), call.plan.kernel
+
+
 @pytest.mark.parametrize("c", SMALL[:4] + SMALL[12:15] + SMALL[19:21], ids=lambda c: c.name)
 def test_small_simt_bf16(c):
     call, _ = _run_small(c, force_simt=True)

@@ -31,34 +31,43 @@ def _close(a, b, dtype):
     return float(np.max(np.abs(a - b))) <= TOL[dtype] * rms
 
 
+@pytest.mark.parametrize("env", [{}, {"CCV3D_HALO": 1}], ids=["default", "halo_planner"])
 @pytest.mark.parametrize("c", [
     Conv("na_384ch_18x40_c2", 384, 384, 18, 40, T_x=1, cache_len=2),
     Conv("na_96ch_24x128_c1_t3", 96, 96, 24, 128, T_x=3, cache_len=1, sigma_b=0.1),
 ], ids=lambda c: c.name)
-def test_noalloc_matches_forward_twice(c):
+def test_noalloc_matches_forward_twice(c, env):
+    """Two calls in a row agree with ccv3d_forward; also when the planner's
+    options would pick another kernel for ccv3d_forward."""
     torch.cuda.set_device(0)
     desc = ccv3d.desc_for(c)
-    plan = ccv3d.Plan(desc)
+    with plan_env(env):
+        plan = ccv3d.Plan(desc)
     for call in range(2):  # the second call reuses the scratch the first left
-        b = _buffers(plan, c, seed_base=100 * call)
-        out_ref, nc_ref = plan.alloc_outputs("cuda")
-        plan.forward(b["x"], b["cache"], b["w"], b["bias"], out_ref, nc_ref)
-        out, nc = plan.alloc_outputs("cuda")
-        out.fill_(float("nan"))
-        torch.cuda.synchronize()
-        reserved = torch.cuda.memory_reserved()
-        free_before = torch.cuda.mem_get_info()[0]
-        rc = ccv3d.ccv3d_forward_noalloc(desc, b["x"], b["cache"], b["w"], b["bias"], out, nc,
-                                         c.stride, c.pad, c.dilation)
-        torch.cuda.synchronize()
-        assert rc == ccv3d.CCV3D_OK
-        assert torch.cuda.memory_reserved() == reserved
-        if call == 1:  # the first call may load the kernel's code; later ones take nothing
-            assert torch.cuda.mem_get_info()[0] == free_before
-        assert bool(torch.isfinite(out.float()).all())
-        assert _close(out, out_ref, c.dtype), (c.name, call)
-        if nc is not None:
-            assert torch.equal(nc, nc_ref)
+        with plan_env(env):
+            _noalloc_vs_forward(c, desc, plan, call)
+
+
+def _noalloc_vs_forward(c, desc, plan, call):
+    b = _buffers(plan, c, seed_base=100 * call)
+    out_ref, nc_ref = plan.alloc_outputs("cuda")
+    plan.forward(b["x"], b["cache"], b["w"], b["bias"], out_ref, nc_ref)
+    out, nc = plan.alloc_outputs("cuda")
+    out.fill_(float("nan"))
+    torch.cuda.synchronize()
+    reserved = torch.cuda.memory_reserved()
+    free_before = torch.cuda.mem_get_info()[0]
+    rc = ccv3d.ccv3d_forward_noalloc(desc, b["x"], b["cache"], b["w"], b["bias"], out, nc,
+                                     c.stride, c.pad, c.dilation)
+    torch.cuda.synchronize()
+    assert rc == ccv3d.CCV3D_OK
+    assert torch.cuda.memory_reserved() == reserved
+    if call == 1:  # the first call may load the kernel's code; later ones take nothing
+        assert torch.cuda.mem_get_info()[0] == free_before
+    assert bool(torch.isfinite(out.float()).all())
+    assert _close(out, out_ref, c.dtype), (c.name, call)
+    if nc is not None:
+        assert torch.equal(nc, nc_ref)
 
 
 def test_noalloc_refuses_what_it_cannot_hold():
