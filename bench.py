@@ -155,6 +155,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------- replicas over ranks
+def max_over_ranks(times_ms, device=None):
+    """Each rank's timings -> the maximum over all ranks (the job ends when
+    its slowest replica ends).  Works on any initialised process group:
+    NCCL with a CUDA device, gloo with the CPU."""
+    import torch
+    import torch.distributed as tdist
+
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(flops_per_call, calls_per_rank, max_ms, world):
+    """Whole-job TFLOP/s: every rank ran `calls_per_rank` independent calls
+    (weak scaling: fixed work per GPU), the job took the slowest rank's time."""
+    return world * flops_per_call * calls_per_rank / (max_ms / 1e3) / 1e12
+
+
 # --------------------------------------------------------------- GPU arm
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -285,9 +304,7 @@ def run_gpu(args, rank, world, local_rank):
     e2e_ms = ea.elapsed_time(eb)
 
     if dist:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+        total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     if rank != 0:
         return None
@@ -295,8 +312,8 @@ def run_gpu(args, rank, world, local_rank):
     avg_launch_s = (sum(per) / len(per)) / 1e3
     achieved = flops / avg_launch_s / 1e12
     peak = peaks["bf16_tflops"]
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
-    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+    value = job_throughput(flops, args.steps, total_ms, world)
+    e2e_value = job_throughput(flops, e2e_steps, e2e_ms, world)
     csum = clocks.summary()
     line = {
         "metric": "cached causal Conv3D effective TFLOP/s (bf16), 1 GPU",
