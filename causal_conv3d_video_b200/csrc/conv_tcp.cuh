@@ -102,12 +102,111 @@ __device__ __forceinline__ int sk_owner_of(const TcParams& p, long long J) {
     return g;
 }
 
+// Epilogue of one segment of the persistent kernel, for this CTA's 128 rows of
+// TMEM accumulator buffer `tmem_acc`, in blocks of kCh channels:
+//   * a piece of a tile owned by an earlier pair ("contributor") is published
+//     as fp32 in this CTA's scratch slot, laid out [16-channel chunk][row][16]
+//     so that a warp's stores (and the owner's loads) are contiguous;
+//   * the owner adds the contributors' pieces, then bias, rounds to bf16 and
+//     writes the block through one of two swizzled staging buffers with a TMA
+//     tensor store (the previous store from that buffer is waited for first).
+template <int kCh>
+__device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t tmem_acc,
+                                                     int q, int lane, int etid, bool owner,
+                                                     bool ok, int g, int g_last, int rank,
+                                                     int BN, int co0, int x0, int y0,
+                                                     int frame, bool store, uint8_t* staging,
+                                                     int& slot) {
+    constexpr int kRowB = kCh * 2;
+    constexpr int kBuf = kTileM * kRowB;
+    const int row = q * 32 + lane;
+    const size_t slot_floats = (size_t)kTileM * BN;
+    float* mine = p.sk.partial + (size_t)(2 * g + rank) * slot_floats;
+    for (int b = 0; b < BN / kCh; ++b) {
+        uint32_t v[kCh];
+#pragma unroll
+        for (int j = 0; j < kCh / 16; ++j)
+            tmem_ld_32x32b_x16(tmem_acc + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kCh + j * 16),
+                               *reinterpret_cast<uint32_t(*)[16]>(&v[j * 16]));
+        tmem_ld_wait();
+        if (!owner) {
+            if (ok) {
+#pragma unroll
+                for (int j = 0; j < kCh / 16; ++j) {
+                    const int chunk = b * (kCh / 16) + j;
+                    float4* dst = reinterpret_cast<float4*>(mine + ((size_t)chunk * kTileM + row) * 16);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_float4(__uint_as_float(v[j * 16 + 4 * e]),
+                                             __uint_as_float(v[j * 16 + 4 * e + 1]),
+                                             __uint_as_float(v[j * 16 + 4 * e + 2]),
+                                             __uint_as_float(v[j * 16 + 4 * e + 3]));
+                }
+            }
+            continue;
+        }
+        float a[kCh];
+#pragma unroll
+        for (int i = 0; i < kCh; ++i) a[i] = __uint_as_float(v[i]);
+        for (int gc = g + 1; gc <= g_last && ok; ++gc) {
+            const float* src = p.sk.partial + (size_t)(2 * gc + rank) * slot_floats;
+#pragma unroll
+            for (int j = 0; j < kCh / 16; ++j) {
+                const int chunk = b * (kCh / 16) + j;
+                const float4* s4 = reinterpret_cast<const float4*>(src + ((size_t)chunk * kTileM + row) * 16);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 w4 = __ldcg(s4 + e);
+                    a[j * 16 + 4 * e] += w4.x;
+                    a[j * 16 + 4 * e + 1] += w4.y;
+                    a[j * 16 + 4 * e + 2] += w4.z;
+                    a[j * 16 + 4 * e + 3] += w4.w;
+                }
+            }
+        }
+        // staging buffer `slot`: its previous tensor store must have read it
+        if (etid == 0) bulk_wait_group_read1();
+        epi_bar();
+        uint8_t* blk = staging + slot * kBuf + (size_t)row * kRowB;
+#pragma unroll
+        for (int c = 0; c < kCh / 8; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int ch = co0 + b * kCh + c * 8 + 2 * i;
+                float b0 = 0.f, b1 = 0.f;
+                if (p.bias != nullptr) {
+                    if (ch < p.Cout) b0 = __bfloat162float(__ushort_as_bfloat16(__ldg(p.bias + ch)));
+                    if (ch + 1 < p.Cout) b1 = __bfloat162float(__ushort_as_bfloat16(__ldg(p.bias + ch + 1)));
+                }
+                const __nv_bfloat162 h =
+                    __floats2bfloat162_rn(a[c * 8 + 2 * i] + b0, a[c * 8 + 2 * i + 1] + b1);
+                w[i] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(blk + (swizzled_chunk<kRowB>(c, row) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        epi_bar();
+        if (etid == 0 && store && ok) {
+            tma_store_4d(&p.tmap_out, smem_u32(staging + slot * kBuf), co0 + b * kCh, x0, y0, frame);
+            bulk_commit_group();
+        }
+        slot ^= 1;
+    }
+}
+
+// Two staging buffers of one output block (kCh channels x 128 rows, bf16).
+__host__ __device__ constexpr size_t tcp_staging_bytes(int bn) {
+    return (size_t)2 * kTileM * out_block_channels(bn) * 2;
+}
+
 template <int BK>
 __host__ __device__ constexpr size_t tcp_smem_bytes(int bn, int stages) {
     // A box + half the weight rows per stage, ring barriers, 2 x (acc full,
     // acc empty) barriers, TMEM address slot
     return 1024 + (size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes) +
-           (size_t)(2 * stages + 4) * 8 + 16;
+           tcp_staging_bytes(bn) + (size_t)(2 * stages + 4) * 8 + 16;
 }
 
 constexpr int kTcpThreads = 320;  // + warps 6-9: the new_cache copy
@@ -129,7 +228,10 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
     const int n_acc = p.sk.n_acc;
     uint8_t* sA = smem;
     uint8_t* sB = smem + (size_t)stages * kA;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + (size_t)stages * kBc);
+    // staging buffers: aligned to their swizzle atom (kA is a multiple of
+    // 4 KB and kBc of 8 rows x kRow; the 64-channel case has kBc % 1024 == 0)
+    uint8_t* staging = sB + (size_t)stages * kBc;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + tcp_staging_bytes(BN));
     uint64_t* empty_bar = full_bar + stages;
     uint64_t* acc_full = empty_bar + stages;   // [2]
     uint64_t* acc_empty = acc_full + 2;        // [2], used in the even CTA
@@ -269,9 +371,8 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
         // ------------------------------------------------- the epilogues
         const int etid = threadIdx.x - 64;
         const int q = warp & 3;
-        const int row = q * 32 + lane;
         const uint32_t empty_leader = mapa_cluster(smem_u32(&acc_empty[0]), 0);
-        int seg = 0;
+        int seg = 0, slot = 0;
         bool ok = true;
         for (long long I = range0; I < range1; ++seg) {
             const Seg sg = sk_locate(p, I, range1);
@@ -309,66 +410,14 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
                     }
                 }
             }
-            const int y = ty * p.box_h + row / p.box_w;
-            const int x = tx * p.box_w + row % p.box_w;
-            const bool valid = y < p.H_o && x < p.W_o;
-            uint16_t* orow = p.out + ((((long long)n * p.T_o + o) * p.H_o + y) * p.W_o + x) *
-                                         (long long)p.Cout;
-            float* mine = p.sk.partial + ((size_t)(2 * g + rank) * kTileM + row) * BN;
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) +
-                                       (uint32_t)(b * BN + c0), v);
-                tmem_ld_wait();
-                if (!ok) continue;
-                float a[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) a[j] = __uint_as_float(v[j]);
-                if (!owner) {
-                    // a piece of a tile owned by an earlier pair: publish fp32
-                    float4* dst = reinterpret_cast<float4*>(mine + c0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_float4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
-                    continue;
-                }
-                for (int gc = g + 1; gc <= g_last; ++gc) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        p.sk.partial + ((size_t)(2 * gc + rank) * kTileM + row) * BN + c0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float4 w4 = __ldcg(src + j);
-                        a[4 * j] += w4.x;
-                        a[4 * j + 1] += w4.y;
-                        a[4 * j + 2] += w4.z;
-                        a[4 * j + 3] += w4.w;
-                    }
-                }
-                const int co = n_tile * BN + c0;
-                if (!valid || co >= p.Cout) continue;
-                uint32_t packed[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float b0 = 0.f, b1 = 0.f;
-                    if (p.bias != nullptr) {
-                        if (co + 2 * j < p.Cout)
-                            b0 = __bfloat162float(__ushort_as_bfloat16(p.bias[co + 2 * j]));
-                        if (co + 2 * j + 1 < p.Cout)
-                            b1 = __bfloat162float(__ushort_as_bfloat16(p.bias[co + 2 * j + 1]));
-                    }
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * j] + b0, a[2 * j + 1] + b1);
-                    packed[j] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                if (co + 16 <= p.Cout) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + co);
-                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (co + j < p.Cout)
-                            orow[co + j] = (uint16_t)(packed[j >> 1] >> ((j & 1) * 16));
-                }
+            const int fo = n * p.T_o + o;
+            const int x0 = tx * p.box_w, y0 = ty * p.box_h, co0 = n_tile * BN;
+            const bool store = ty < p.tiles_y;  // a box past the frame stores nothing
+            const uint32_t tacc = tmem_base + (uint32_t)(b * BN);
+            switch (out_block_channels(BN)) {
+                case 64: tcp_segment_epilogue<64>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot); break;
+                case 32: tcp_segment_epilogue<32>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot); break;
+                default: tcp_segment_epilogue<16>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot); break;
             }
             // TMEM buffer b is drained: hand it back to the MMA issuer
             tc_fence_before();
@@ -387,6 +436,7 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             }
             I = sg.tile_start + sg.kb1;
         }
+        if (etid == 0) bulk_wait_group0();  // output stores complete before exit
     }
 
     __syncwarp();
