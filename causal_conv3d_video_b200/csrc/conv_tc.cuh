@@ -77,16 +77,18 @@ conv_tc_kernel(const __grid_constant__ TcParams p) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- tile coordinates: (n, o, ty, tx) x n_tile, n_tile fastest so that
-    // neighbouring CTAs share the A operand in L2.
+    // ---- tile coordinates: (ty, tx, n, o) x n_tile, n_tile fastest so that
+    // neighbouring CTAs share the A operand in L2, then the output frame so
+    // that the tiles reading one source frame through different temporal
+    // taps run close together.
     const int n_tile = blockIdx.x % p.tiles_n;
     int m_tile = blockIdx.x / p.tiles_n;
-    const int tx = m_tile % p.tiles_x;
-    m_tile /= p.tiles_x;
-    const int ty = m_tile % p.tiles_y;
-    m_tile /= p.tiles_y;
     const int o = m_tile % p.T_o;
-    const int n = m_tile / p.T_o;
+    m_tile /= p.T_o;
+    const int n = m_tile % p.N;
+    m_tile /= p.N;
+    const int tx = m_tile % p.tiles_x;
+    const int ty = m_tile / p.tiles_x;
 
     int n_active = 0;
 #pragma unroll

@@ -79,9 +79,11 @@ conv_tc2h_kernel(const __grid_constant__ TcParams p) {
     const int pair = blockIdx.x >> 1;
     const int n_tile = pair % p.tiles_n;
     const int m_pair = pair / p.tiles_n;
-    const int ppf = p.pairs_per_frame;
-    const int frame = m_pair / ppf;
-    const int box = (m_pair % ppf) * 2 + (int)rank;
+    // output frame fastest: the tiles that read one source frame through
+    // different temporal taps run close together and share it in L2
+    const int frames = p.N * p.T_o;
+    const int frame = m_pair % frames;
+    const int box = (m_pair / frames) * 2 + (int)rank;
     const int o = frame % p.T_o;
     const int n = frame / p.T_o;
     int tx = 0, ty = p.tiles_y;
