@@ -408,7 +408,7 @@ def run_sequence(args, dev):
             mods[call.module] = [w, b, caches, 0]
     stream = torch.cuda.current_stream(dev)
 
-    def one_pass():
+    def one_pass(stream=stream):
         for m in mods.values():
             m[3] = 0
         for call in calls:
@@ -436,11 +436,36 @@ def run_sequence(args, dev):
     for plan in plans.values():
         if plan.status() != 0:
             raise RuntimeError("device status after the decode sequence")
+    # the same pass captured once as a CUDA graph (164 kernel nodes), replayed
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(graph, stream=cap):
+        one_pass(cap)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(passes):
+        graph.replay()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    ms_graph = ea.elapsed_time(eb) / passes
+    for plan in plans.values():
+        if plan.status() != 0:
+            raise RuntimeError("device status after the graph-replayed decode sequence")
+    del graph
     kernels = sorted({p.kernel for p in plans.values()})
     return {"calls": len(calls), "signatures": len(plans), "ms_per_sequence": round(ms, 3),
             "tflops": round(flops / (ms / 1e3) / 1e12, 2), "gflop_per_sequence": round(flops / 1e9, 1),
+            "ms_per_sequence_graph": round(ms_graph, 3),
+            "tflops_graph": round(flops / (ms_graph / 1e3) / 1e12, 2),
             "passes": passes, "kernels": kernels,
-            "what": "164-call synthetic 17-frame decode, caches threaded, one stream"}
+            "kernel_per_signature": {f"{k[0]}->{k[1]} k{k[2]}{k[3]}{k[4]} {k[5]}x{k[6]} T{k[7]} C{k[8]}":
+                                     p.kernel for k, p in plans.items()},
+            "what": "164-call synthetic 17-frame decode, caches threaded, one stream; "
+                    "eager launches, and the same pass captured as one CUDA graph"}
 
 
 # ------------------------------------------------------------- CPU oracle

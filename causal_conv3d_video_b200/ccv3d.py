@@ -25,7 +25,7 @@ CCV3D_MAX_KT = 3
 EXPORTED = ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_plan_path", "ccv3d_forward",
             "ccv3d_get_stats", "ccv3d_get_status", "ccv3d_destroy", "ccv3d_strerror",
             "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout", "ccv3d_forward_noalloc",
-            "ccv3d_plan_kernel")
+            "ccv3d_plan_kernel", "ccv3d_plan_tiling")
 CCV3D_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -67,6 +67,8 @@ def _load():
     lib.ccv3d_strerror.restype = ctypes.c_char_p
     lib.ccv3d_plan_kernel.argtypes = [vp]
     lib.ccv3d_plan_kernel.restype = ctypes.c_char_p
+    lib.ccv3d_plan_tiling.argtypes = [vp, ip, ip, ip]
+    lib.ccv3d_plan_tiling.restype = ctypes.c_int
     lib.ccv3d_plan_sizes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t),
                                      ctypes.POINTER(ctypes.c_size_t), ip]
     lib.ccv3d_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
@@ -132,6 +134,14 @@ def ccv3d_plan_path(plan):
 
 def ccv3d_plan_kernel(plan) -> str:
     return lib.ccv3d_plan_kernel(plan).decode()
+
+
+def ccv3d_plan_tiling(plan) -> dict:
+    kb, st, g = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    rc = lib.ccv3d_plan_tiling(plan, ctypes.byref(kb), ctypes.byref(st), ctypes.byref(g))
+    if rc not in (0, 2):
+        raise CCV3DError(rc, "ccv3d_plan_tiling")
+    return {"k_block": kb.value, "stages": st.value, "workspace_pairs": g.value}
 
 
 def ccv3d_plan_sizes(plan):
@@ -228,6 +238,7 @@ class Plan:
         self.sizes = ccv3d_plan_sizes(self.handle)
         self.path = ccv3d_plan_path(self.handle)
         self.kernel = ccv3d_plan_kernel(self.handle)
+        self.tiling = ccv3d_plan_tiling(self.handle)
 
     @property
     def stride(self):

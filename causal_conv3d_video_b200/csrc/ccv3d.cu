@@ -130,7 +130,14 @@ size_t halo_smem_for(int bk, int bn, int stages, int kh, int kw, int halo_w) {
 template <int BK>
 int pick_stages(int kind, int bn, int want) {
     int s = want > 0 ? std::min(want, 12) : 8;
-    while (s > 2 && smem_for<BK>(kind, bn, s) > kSmemBudget) --s;
+    int lo = 2;
+    if (kind == 2) {
+        // the persistent kernel's owner fetches whole fp32 output blocks of
+        // the contributors into its idle ring: keep room for one
+        while (tcp_ring_bytes<BK>(bn, lo) < (size_t)kTileM * out_block_channels(bn) * 4) ++lo;
+        s = std::max(s, lo);
+    }
+    while (s > lo && smem_for<BK>(kind, bn, s) > kSmemBudget) --s;
     return s;
 }
 
@@ -177,16 +184,21 @@ int env_int(const char* name) {
     return e != nullptr ? std::atoi(e) : 0;
 }
 
+// Widest channel block (k-block depth) that divides Cin.
+int widest_bk(int Cin) { return Cin % 64 == 0 ? 64 : (Cin % 32 == 0 ? 32 : 16); }
+
 // Schedule of the persistent stream-K pair kernel: usable when the plan runs
 // CTA pairs, every output frame has an active tap and the (n, o) frames fit
-// the schedule table.  Sets p->persist; returns it.
+// the schedule table.  On success the plan switches to it (persist = 1, no
+// halo strips, the widest channel block: a halo sizing may have narrowed it)
+// and true is returned; otherwise the plan is left as it was.
 bool setup_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
-    p->persist = 0;
-    p->halo = 0;  // the persistent kernel has its own (non-halo) stages
     if (!p->path_tc_candidate || !p->pair) return false;
-    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
     const int frames = d.N * p->T_o;
     if (frames > kMaxFrames) return false;
+    const int bk = widest_bk(d.Cin);
+    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, bk);
+    long long start[kMaxFrames + 1];
     long long acc = 0;
     const long long tiles_per_frame = (long long)((p->tiles_x * p->tiles_y + 1) / 2) * p->tiles_n;
     for (int f = 0; f < frames; ++f) {
@@ -194,11 +206,14 @@ bool setup_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
         int a = 0;
         for (int k = 0; k < d.kt; ++k) a += (o >= p->o_l[k] && o < p->o_h[k]) ? 1 : 0;
         if (a == 0) return false;
-        p->frame_start[f] = acc;
+        start[f] = acc;
         acc += tiles_per_frame * a * per_tap;
     }
-    p->frame_start[frames] = acc;
+    start[frames] = acc;
+    for (int f = 0; f <= frames; ++f) p->frame_start[f] = start[f];
     p->sk_total = acc;
+    p->BK = bk;
+    p->halo = 0;
     p->persist = 1;
     return true;
 }
@@ -254,6 +269,25 @@ void setup_halo(const ccv3d_desc& d, ccv3d_plan_s* p) {
     }
 }
 
+// Whether the persistent stream-K kernel should replace one launch of pair
+// tiles (the plan as sized for that launch).  Measured over the decoder
+// signatures on B200, stream-K is 5-30% faster where
+//   * the launch runs at least two waves of pair tiles (one per SM pair) and
+//     its last wave is ragged (waves / ceil(waves) < 0.9), e.g. 180x320
+//     outputs, stride-2 and 3x1x1 calls; or
+//   * the halo kernel would run a call of Cout >= 192 (360x640 calls);
+// and slower where the tiles make less than two waves (the fix-up of split
+// tiles is not amortised), where the waves are nearly even, and on the thin
+// 720x1280 calls the halo kernel suits.  CCV3D_PERSIST=0/1 overrides.
+bool prefer_persistent(const ccv3d_desc& d, const ccv3d_plan_s& p) {
+    if (!p.pair) return false;
+    if (p.halo) return d.Cout >= 192;
+    const long long tiles =
+        (long long)d.N * p.T_o * ((p.tiles_x * p.tiles_y + 1) / 2) * p.tiles_n;
+    const double waves = (double)tiles / (kSmCount / 2);
+    return waves >= 2.0 && waves / std::ceil(waves) < 0.9;
+}
+
 // Kernel choice and tiling.
 void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->path_tc = 0;
@@ -287,20 +321,18 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->BN = ((ceil_div(d.Cout, p->tiles_n) + 15) / 16) * 16;
     p->n_sub = p->BN > 256 ? 2 : 1;
     if (p->n_sub == 2 && p->BN % 32 != 0) p->BN = ((p->BN + 31) / 32) * 32;
-    p->BK = d.Cin % 64 == 0 ? 64 : (d.Cin % 32 == 0 ? 32 : 16);
+    p->BK = widest_bk(d.Cin);
     // CTA pairs whenever every pair MMA has N >= 32 (16 weight rows per CTA)
     const char* pe = std::getenv("CCV3D_PAIR");
     p->pair = (p->BN / p->n_sub) >= 32 ? 1 : 0;
     if (pe != nullptr) p->pair = std::atoi(pe) != 0 && (p->BN / p->n_sub) >= 32;
     p->path_tc_candidate = 1;
-    // Persistent stream-K on CTA pairs (opt-in: CCV3D_PERSIST=1).  Measured
-    // on B200 it is slower than one launch of pair tiles on every decoder
-    // signature: the calls are bound by aggregate L2->SM traffic, which
-    // spreading the k-blocks over all SM pairs does not reduce.
     p->persist = 0;
-    if (env_int("CCV3D_PERSIST") > 0) setup_persistent(d, p);
     size_tc(d, p);
     setup_halo(d, p);
+    const char* ps = std::getenv("CCV3D_PERSIST");
+    const bool persist = ps != nullptr ? std::atoi(ps) > 0 : prefer_persistent(d, *p);
+    if (persist && setup_persistent(d, p)) size_tc(d, p);
     p->path_tc = 1;
 }
 
@@ -488,7 +520,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     if (grid > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
     // spread the K-start offsets over one wave of concurrently running tiles
     const long long units = p->pair ? grid / 2 : grid;
-    const long long wave = p->pair ? 74 : 148;
+    const long long wave = p->pair ? kSmCount / 2 : kSmCount;
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
     const int kind = p->halo ? 3 : (p->persist ? 2 : p->pair);
     prm.halo_w = p->halo_w;
@@ -651,6 +683,18 @@ const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
     if (p->halo) return "tc_pair_halo";
     if (p->persist) return "tc_persistent";
     return p->pair ? "tc_pair" : "tc_single";
+}
+
+ccv3d_status ccv3d_plan_tiling(ccv3d_plan_t p, int* k_block, int* stages, int* workspace_pairs) {
+    if (k_block) *k_block = 0;
+    if (stages) *stages = 0;
+    if (workspace_pairs) *workspace_pairs = 0;
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    if (!p->path_tc) return CCV3D_ERR_UNSUPPORTED;
+    if (k_block) *k_block = p->BK;
+    if (stages) *stages = p->stages;
+    if (workspace_pairs) *workspace_pairs = p->persist ? p->G : 0;
+    return CCV3D_OK;
 }
 
 ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t p, size_t* out_bytes, size_t* nc_bytes,

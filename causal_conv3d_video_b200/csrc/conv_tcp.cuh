@@ -54,6 +54,23 @@ __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Order this thread's earlier generic-proxy observations of global memory
+// before its later async-proxy (bulk copy) reads of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Plain (untiled) bulk copy of `bytes` bytes global -> this CTA's shared
+// memory, completing on mbarrier `bar`.  Both addresses and `bytes` are
+// multiples of 16.
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 
 // One piece of a pair's range: pair tile `tile` (frame f, index in frame),
 // k-blocks [kb0, kb1) of its reduction of `iters` k-blocks.
@@ -102,85 +119,130 @@ __device__ __forceinline__ int sk_owner_of(const TcParams& p, long long J) {
     return g;
 }
 
+// Fp32 partial tile layout in a scratch slot, for one CTA's 128 x BN piece:
+// blocks of kCh channels, each block [16-channel chunk][quad e][row][4
+// floats], so that a warp's float4 stores (thread = row) cover 512 contiguous
+// bytes and one block is one contiguous run the owner fetches in one copy.
+template <int kCh>
+__device__ __forceinline__ size_t tcp_partial_index(int b, int j, int e, int row) {
+    return (size_t)b * (kTileM * kCh) + ((size_t)(j * 4 + e) * kTileM + row) * 4;
+}
+
 // Epilogue of one segment of the persistent kernel, for this CTA's 128 rows of
 // TMEM accumulator buffer `tmem_acc`, in blocks of kCh channels:
 //   * a piece of a tile owned by an earlier pair ("contributor") is published
-//     as fp32 in this CTA's scratch slot, laid out [16-channel chunk][row][16]
-//     so that a warp's stores (and the owner's loads) are contiguous;
+//     as fp32 in this CTA's scratch slot (layout above);
 //   * the owner adds the contributors' pieces, then bias, rounds to bf16 and
 //     writes the block through one of two swizzled staging buffers with a TMA
 //     tensor store (the previous store from that buffer is waited for first).
+//     A tile with contributors is always the last segment of the owner's
+//     range, so the operand ring is idle by then: the contributors' blocks are
+//     fetched into it with bulk copies, up to `n_fbuf` in flight, one fetch
+//     barrier per ring buffer; `fetch_uses` counts this CTA's fetches so far
+//     (the parity of each buffer's next completion).
 template <int kCh>
 __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t tmem_acc,
                                                      int q, int lane, int etid, bool owner,
                                                      bool ok, int g, int g_last, int rank,
                                                      int BN, int co0, int x0, int y0,
                                                      int frame, bool store, uint8_t* staging,
-                                                     int& slot) {
+                                                     int& slot, uint8_t* ring, int n_fbuf,
+                                                     uint64_t* fetch_bar, uint32_t& fetch_uses,
+                                                     const float* bias_s) {
     constexpr int kRowB = kCh * 2;
     constexpr int kBuf = kTileM * kRowB;
+    constexpr uint32_t kUnit = kTileM * kCh * 4;  // bytes of one fp32 block
     const int row = q * 32 + lane;
     const size_t slot_floats = (size_t)kTileM * BN;
-    float* mine = p.sk.partial + (size_t)(2 * g + rank) * slot_floats;
-    for (int b = 0; b < BN / kCh; ++b) {
+    const int nblk = BN / kCh;
+    if (!owner) {
+        float* mine = p.sk.partial + (size_t)(2 * g + rank) * slot_floats;
+        for (int b = 0; b < nblk; ++b) {
+            uint32_t v[kCh];
+#pragma unroll
+            for (int j = 0; j < kCh / 16; ++j)
+                tmem_ld_32x32b_x16(tmem_acc + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kCh + j * 16),
+                                   *reinterpret_cast<uint32_t(*)[16]>(&v[j * 16]));
+            tmem_ld_wait();
+            if (!ok) continue;
+#pragma unroll
+            for (int j = 0; j < kCh / 16; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    *reinterpret_cast<float4*>(mine + tcp_partial_index<kCh>(b, j, e, row)) =
+                        make_float4(__uint_as_float(v[j * 16 + 4 * e]),
+                                    __uint_as_float(v[j * 16 + 4 * e + 1]),
+                                    __uint_as_float(v[j * 16 + 4 * e + 2]),
+                                    __uint_as_float(v[j * 16 + 4 * e + 3]));
+        }
+        return;
+    }
+    // ---- owner: fetch units u = (block b, contributor c), block-major
+    const int ncon = ok ? g_last - g : 0;
+    const int units = nblk * ncon;
+    const uint32_t use0 = fetch_uses;
+    auto issue = [&](int u) {
+        const int b = u / ncon, c = u - b * ncon;
+        const int buf = (int)((use0 + (uint32_t)u) % (uint32_t)n_fbuf);
+        const float* src = p.sk.partial + (size_t)(2 * (g + 1 + c) + rank) * slot_floats +
+                           (size_t)b * (kTileM * kCh);
+        const uint32_t bar = smem_u32(&fetch_bar[buf]);
+        mbar_arrive_expect_tx(bar, kUnit);
+        bulk_load_g2s(smem_u32(ring + (size_t)buf * kUnit), src, kUnit, bar);
+    };
+    if (etid == 0 && units > 0) {
+        fence_proxy_async_global();  // the flags were acquired through the generic proxy
+        for (int u = 0; u < units && u < n_fbuf; ++u) issue(u);
+    }
+    bool fetched = true;
+    int u = 0;
+    for (int b = 0; b < nblk; ++b) {
         uint32_t v[kCh];
 #pragma unroll
         for (int j = 0; j < kCh / 16; ++j)
             tmem_ld_32x32b_x16(tmem_acc + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kCh + j * 16),
                                *reinterpret_cast<uint32_t(*)[16]>(&v[j * 16]));
         tmem_ld_wait();
-        if (!owner) {
-            if (ok) {
-#pragma unroll
-                for (int j = 0; j < kCh / 16; ++j) {
-                    const int chunk = b * (kCh / 16) + j;
-                    float4* dst = reinterpret_cast<float4*>(mine + ((size_t)chunk * kTileM + row) * 16);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_float4(__uint_as_float(v[j * 16 + 4 * e]),
-                                             __uint_as_float(v[j * 16 + 4 * e + 1]),
-                                             __uint_as_float(v[j * 16 + 4 * e + 2]),
-                                             __uint_as_float(v[j * 16 + 4 * e + 3]));
-                }
-            }
-            continue;
-        }
         float a[kCh];
 #pragma unroll
         for (int i = 0; i < kCh; ++i) a[i] = __uint_as_float(v[i]);
-        for (int gc = g + 1; gc <= g_last && ok; ++gc) {
-            const float* src = p.sk.partial + (size_t)(2 * gc + rank) * slot_floats;
+        for (int c = 0; c < ncon; ++c, ++u) {
+            const uint32_t use = use0 + (uint32_t)u;
+            const int buf = (int)(use % (uint32_t)n_fbuf);
+            if (fetched && !mbar_wait(smem_u32(&fetch_bar[buf]), (use / (uint32_t)n_fbuf) & 1u,
+                                      p.status, p.wait_limit_ns))
+                fetched = false;
+            if (!fetched) continue;
+            const float* src = reinterpret_cast<const float*>(ring + (size_t)buf * kUnit);
 #pragma unroll
-            for (int j = 0; j < kCh / 16; ++j) {
-                const int chunk = b * (kCh / 16) + j;
-                const float4* s4 = reinterpret_cast<const float4*>(src + ((size_t)chunk * kTileM + row) * 16);
+            for (int j = 0; j < kCh / 16; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float4 w4 = __ldcg(s4 + e);
+                    const float4 w4 =
+                        *reinterpret_cast<const float4*>(src + tcp_partial_index<kCh>(0, j, e, row));
                     a[j * 16 + 4 * e] += w4.x;
                     a[j * 16 + 4 * e + 1] += w4.y;
                     a[j * 16 + 4 * e + 2] += w4.z;
                     a[j * 16 + 4 * e + 3] += w4.w;
                 }
-            }
         }
         // staging buffer `slot`: its previous tensor store must have read it
         if (etid == 0) bulk_wait_group_read1();
-        epi_bar();
+        epi_bar();  // also: every thread is done with this block's fetch buffers
+        if (etid == 0 && fetched) {
+            fence_proxy_async_smem();
+            for (int r = u - ncon; r < u; ++r)
+                if (r + n_fbuf < units) issue(r + n_fbuf);
+        }
         uint8_t* blk = staging + slot * kBuf + (size_t)row * kRowB;
 #pragma unroll
         for (int c = 0; c < kCh / 8; ++c) {
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int ch = co0 + b * kCh + c * 8 + 2 * i;
-                float b0 = 0.f, b1 = 0.f;
-                if (p.bias != nullptr) {
-                    if (ch < p.Cout) b0 = __bfloat162float(__ushort_as_bfloat16(__ldg(p.bias + ch)));
-                    if (ch + 1 < p.Cout) b1 = __bfloat162float(__ushort_as_bfloat16(__ldg(p.bias + ch + 1)));
-                }
-                const __nv_bfloat162 h =
-                    __floats2bfloat162_rn(a[c * 8 + 2 * i] + b0, a[c * 8 + 2 * i + 1] + b1);
+                const int ch = b * kCh + c * 8 + 2 * i;
+                const __nv_bfloat162 h = __floats2bfloat162_rn(a[c * 8 + 2 * i] + bias_s[ch],
+                                                               a[c * 8 + 2 * i + 1] + bias_s[ch + 1]);
                 w[i] = *reinterpret_cast<const uint32_t*>(&h);
             }
             *reinterpret_cast<uint4*>(blk + (swizzled_chunk<kRowB>(c, row) << 4)) =
@@ -194,6 +256,7 @@ __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t
         }
         slot ^= 1;
     }
+    fetch_uses = use0 + (uint32_t)units;
 }
 
 // Two staging buffers of one output block (kCh channels x 128 rows, bf16).
@@ -201,12 +264,20 @@ __host__ __device__ constexpr size_t tcp_staging_bytes(int bn) {
     return (size_t)2 * kTileM * out_block_channels(bn) * 2;
 }
 
+constexpr int kTcpFetchBufs = 8;  // most partial-block fetch buffers in flight
+
+template <int BK>
+__host__ __device__ constexpr size_t tcp_ring_bytes(int bn, int stages) {
+    return (size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes);
+}
+
 template <int BK>
 __host__ __device__ constexpr size_t tcp_smem_bytes(int bn, int stages) {
-    // A box + half the weight rows per stage, ring barriers, 2 x (acc full,
-    // acc empty) barriers, TMEM address slot
-    return 1024 + (size_t)stages * (TcSmem<BK>::kABytes + (size_t)(bn / 2) * TcSmem<BK>::kRowBytes) +
-           tcp_staging_bytes(bn) + (size_t)(2 * stages + 4) * 8 + 16;
+    // A box + half the weight rows per stage, output staging, ring barriers,
+    // 2 x (acc full, acc empty) barriers, fetch barriers, TMEM address slot,
+    // the Cout tile's bias
+    return 1024 + tcp_ring_bytes<BK>(bn, stages) + tcp_staging_bytes(bn) +
+           (size_t)(2 * stages + 4 + kTcpFetchBufs) * 8 + 16 + (size_t)bn * 4;
 }
 
 constexpr int kTcpThreads = 320;  // + warps 6-9: the new_cache copy
@@ -235,7 +306,9 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
     uint64_t* empty_bar = full_bar + stages;
     uint64_t* acc_full = empty_bar + stages;   // [2]
     uint64_t* acc_empty = acc_full + 2;        // [2], used in the even CTA
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    uint64_t* fetch_bar = acc_empty + 2;       // [kTcpFetchBufs]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fetch_bar + kTcpFetchBufs);
+    float* bias_s = reinterpret_cast<float*>(tmem_slot + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -253,6 +326,7 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             mbar_init(smem_u32(&acc_full[b]), 1);
             mbar_init(smem_u32(&acc_empty[b]), 8);  // 4 epilogue warps x 2 CTAs
         }
+        for (int b = 0; b < kTcpFetchBufs; ++b) mbar_init(smem_u32(&fetch_bar[b]), 1);
         fence_mbar_init();
         tma_prefetch_desc(&p.tmap_x);
         if (p.cache_len > 0) tma_prefetch_desc(&p.tmap_c);
@@ -374,6 +448,13 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
         const uint32_t empty_leader = mapa_cluster(smem_u32(&acc_empty[0]), 0);
         int seg = 0, slot = 0;
         bool ok = true;
+        uint32_t fetch_uses = 0;
+        int bias_tile = -1;  // Cout tile whose bias bias_s holds
+        // fp32 partial blocks the idle ring holds at once (the planner keeps
+        // the ring at least one block large)
+        int n_fbuf = (int)(tcp_ring_bytes<BK>(BN, stages) /
+                           ((size_t)kTileM * out_block_channels(BN) * 4));
+        if (n_fbuf > kTcpFetchBufs) n_fbuf = kTcpFetchBufs;
         for (long long I = range0; I < range1; ++seg) {
             const Seg sg = sk_locate(p, I, range1);
             const int b = n_acc == 2 ? (seg & 1) : 0;
@@ -393,6 +474,17 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             tc_fence_after();
             const bool owner = sg.kb0 == 0;
             const bool whole = owner && sg.kb1 == sg.iters;
+            if (owner && n_tile != bias_tile) {
+                epi_bar();  // the previous tile's epilogue is done with bias_s
+                for (int i = etid; i < BN; i += 128) {
+                    const int co = n_tile * BN + i;
+                    bias_s[i] = (p.bias != nullptr && co < p.Cout)
+                                    ? __bfloat162float(__ushort_as_bfloat16(__ldg(p.bias + co)))
+                                    : 0.f;
+                }
+                epi_bar();
+                bias_tile = n_tile;
+            }
             // pairs holding the other pieces of this tile (owner only)
             int g_last = g;
             if (owner && !whole) g_last = sk_owner_of(p, sg.tile_start + sg.iters - 1);
@@ -415,10 +507,16 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             const bool store = ty < p.tiles_y;  // a box past the frame stores nothing
             const uint32_t tacc = tmem_base + (uint32_t)(b * BN);
             switch (out_block_channels(BN)) {
-                case 64: tcp_segment_epilogue<64>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot); break;
-                case 32: tcp_segment_epilogue<32>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot); break;
-                default: tcp_segment_epilogue<16>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot); break;
+                case 64: tcp_segment_epilogue<64>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot, smem, n_fbuf, fetch_bar, fetch_uses, bias_s); break;
+                case 32: tcp_segment_epilogue<32>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot, smem, n_fbuf, fetch_bar, fetch_uses, bias_s); break;
+                default: tcp_segment_epilogue<16>(p, tacc, q, lane, etid, owner, ok, g, g_last, (int)rank, BN, co0, x0, y0, fo, store, staging, slot, smem, n_fbuf, fetch_bar, fetch_uses, bias_s); break;
             }
+            // Contributors' flags consumed (every epilogue thread has passed
+            // its flag wait: the fix-up has block barriers): clear them, so a
+            // replay of the same launch parameters (a captured graph, whose
+            // epoch is fixed) waits for fresh pieces again.
+            if (owner && !whole && ok && etid == 0)
+                for (int gc = g + 1; gc <= g_last; ++gc) p.sk.flags[2 * gc + rank] = 0u;
             // TMEM buffer b is drained: hand it back to the MMA issuer
             tc_fence_before();
             __syncwarp();

@@ -8,6 +8,7 @@ namespace ccv3d {
 
 constexpr int kMaxTaps = 3;
 constexpr int kTileM = 128;          // output pixels per GEMM tile (UMMA M)
+constexpr int kSmCount = 148;        // B200 SMs (scheduling heuristics only)
 constexpr int kTcThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 

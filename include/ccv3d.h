@@ -131,6 +131,15 @@ CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
  * "tc_single", "tc_persistent" or "simt" (static string; "" for NULL). */
 CCV3D_API const char* ccv3d_plan_kernel(ccv3d_plan_t plan);
 
+/* Reduction tiling of a tensor-core plan (inspection; no counterpart in the
+ * paper): k_block = input channels per pipeline stage (64, 32 or 16), stages
+ * = depth of the shared-memory ring, workspace_pairs = CTA pairs of the
+ * persistent stream-K kernel (0 for the other kernels).  Any output pointer
+ * may be NULL.  Errors: INVALID for a NULL plan, UNSUPPORTED for a SIMT plan
+ * (outputs are then 0). */
+CCV3D_API ccv3d_status ccv3d_plan_tiling(ccv3d_plan_t plan, int* k_block, int* stages,
+                                         int* workspace_pairs);
+
 /* Run one cached causal Conv3D call on `stream` (device pointers, layouts as
  * above).  stride = {s_h, s_w}, pad = {p_h, p_w}, dilation = {d_t, d_h, d_w}
  * must equal the plan's (the call signature of the paper's patched module).

@@ -162,3 +162,40 @@ def test_tile_choice_on_bottleneck():
     assert ccv3d.Plan(ccv3d.desc_for(workloads.C4_TIME)).path["tile_n"] == 384
     thin = ccv3d.Plan(ccv3d.make_desc(N=1, Cin=3, Cout=16, H=8, W=8, T_x=1, cache_len=0))
     assert thin.path["tc"] is False
+
+
+@pytest.mark.parametrize("conv,kernel", [
+    (workloads.C2, "tc_pair"),                      # 0.8 wave of pair tiles
+    (workloads.C3, "tc_pair_halo"),                 # thin 720x1280: halo strips
+    (workloads.C4_TIME, "tc_persistent"),           # 6.1 waves, ragged last wave
+    (workloads.C4_STRIDE, "tc_persistent"),         # 3.04 waves
+    (workloads.C4_DIL, "tc_persistent"),
+    (workloads.C4_ODD, "tc_pair"),
+    (workloads.Conv("g8", 192, 192, 360, 640, T_x=2, cache_len=2), "tc_persistent"),  # halo, Cout 192
+    (workloads.Conv("g5", 384, 384, 360, 640, T_x=2, cache_len=2), "tc_pair"),        # 24.3 even waves
+], ids=lambda v: getattr(v, "name", v))
+def test_kernel_choice(conv, kernel, monkeypatch):
+    """Persistent stream-K where one launch of pair tiles leaves a ragged
+    last wave over >= 2 waves, or where the halo kernel would run Cout >= 192;
+    CCV3D_PERSIST=0/1 overrides."""
+    monkeypatch.delenv("CCV3D_PERSIST", raising=False)
+    assert ccv3d.Plan(ccv3d.desc_for(conv)).kernel == kernel
+    monkeypatch.setenv("CCV3D_PERSIST", "0")
+    assert ccv3d.Plan(ccv3d.desc_for(conv)).kernel != "tc_persistent"
+    monkeypatch.setenv("CCV3D_PERSIST", "1")
+    plan = ccv3d.Plan(ccv3d.desc_for(conv))
+    assert plan.kernel == "tc_persistent"
+    # the persistent kernel streams the widest channel block, whatever a halo
+    # sizing (two CTAs per SM) would have chosen
+    want_bk = 64 if conv.Cin % 64 == 0 else (32 if conv.Cin % 32 == 0 else 16)
+    assert plan.tiling["k_block"] == want_bk
+
+
+def test_plan_tiling_reports():
+    halo = ccv3d.Plan(ccv3d.desc_for(workloads.C3))
+    assert halo.kernel == "tc_pair_halo"
+    assert halo.tiling["k_block"] in (16, 32) and halo.tiling["stages"] >= 2
+    assert halo.tiling["workspace_pairs"] == 0
+    simt = ccv3d.Plan(ccv3d.desc_for(workloads.C1))
+    assert simt.tiling == {"k_block": 0, "stages": 0, "workspace_pairs": 0}
+    assert ccv3d.lib.ccv3d_plan_tiling(None, None, None, None) == ccv3d.CCV3D_ERR_INVALID

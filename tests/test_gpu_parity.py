@@ -78,7 +78,8 @@ def test_config1_fp32_exact_workload():
     assert call.plan.stats()["simt_path"] == 1
 
 
-KERNELS = {"persistent": {"CCV3D_PERSIST": 1}, "pair": {}, "single": {"CCV3D_PAIR": 0}}
+KERNELS = {"persistent": {"CCV3D_PERSIST": 1}, "pair": {"CCV3D_PERSIST": 0},
+           "single": {"CCV3D_PAIR": 0, "CCV3D_PERSIST": 0}}
 
 
 @pytest.mark.parametrize("kernel", sorted(KERNELS))
@@ -128,7 +129,7 @@ HALO = [
 @pytest.mark.parametrize("halo", [1, 0], ids=["halo", "no_halo"])
 @pytest.mark.parametrize("c", HALO, ids=lambda c: c.name)
 def test_small_halo_strips(c, halo):
-    call, _ = _run_small(c, env={"CCV3D_HALO": halo})
+    call, _ = _run_small(c, env={"CCV3D_HALO": halo, "CCV3D_PERSIST": 0})
     assert (call.plan.kernel == "tc_pair_halo") == bool(halo), call.plan.kernel
 
 
