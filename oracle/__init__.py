@@ -36,7 +36,7 @@ class OracleParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "N", "Cin", "Cout", "kt", "kh", "kw", "H", "W", "T_x", "cache_len",
         "pad_t_base", "cache_keep", "s_h", "s_w", "p_h", "p_w", "d_t", "d_h",
-        "d_w")]
+        "d_w", "s_t")]
 
 
 def build(src: str = _SRC, out: str = _LIB_PATH, force: bool = False) -> str:
@@ -83,9 +83,10 @@ def _bind(lib):
 
 def params(N, Cin, Cout, H, W, T_x, cache_len, *, kt=3, kh=3, kw=3,
            pad_t_base=None, cache_keep=None, stride=(1, 1), pad=(1, 1),
-           dilation=(1, 1, 1)) -> OracleParams:
+           dilation=(1, 1, 1), stride_t=1) -> OracleParams:
     """Build an OracleParams.  pad_t_base defaults to d_t*(kt-1) and
-    cache_keep to pad_t_base."""
+    cache_keep to pad_t_base; stride is (s_h, s_w), stride_t the temporal
+    stride."""
     d_t, d_h, d_w = dilation
     if pad_t_base is None:
         pad_t_base = d_t * (kt - 1)
@@ -93,7 +94,7 @@ def params(N, Cin, Cout, H, W, T_x, cache_len, *, kt=3, kh=3, kw=3,
         cache_keep = pad_t_base
     return OracleParams(N, Cin, Cout, kt, kh, kw, H, W, T_x, cache_len,
                         pad_t_base, cache_keep, stride[0], stride[1], pad[0],
-                        pad[1], d_t, d_h, d_w)
+                        pad[1], d_t, d_h, d_w, stride_t)
 
 
 def _dptr(a):

@@ -13,11 +13,14 @@
  *   Zp = p_l zero frames followed by Z        (p_l >= 0)
  *      = Z with its first -p_l frames dropped (p_l <  0)
  *   out[n,o,y,x,co] = bias[co] + sum_{k,r,s,ci}
- *        Zp[n, o + k*d_t, y*s_h + r*d_h - p_h, x*s_w + s*d_w - p_w, ci]
+ *        Zp[n, o*s_t + k*d_t, y*s_h + r*d_h - p_h, x*s_w + s*d_w - p_w, ci]
  *        * W[co, k, r, s, ci]
  *
- * which is PyTorch's cross-correlation convention with unit temporal stride
- * and one group; spatial positions outside [0,H)x[0,W) read zero.  Sums are
+ * which is PyTorch's cross-correlation convention with one group; spatial
+ * positions outside [0,H)x[0,W) read zero.  The paper's lowering covers unit
+ * temporal stride (s_t = 1); s_t > 1 (the encoders' temporal downsampling,
+ * which the paper leaves on native Conv3D) is the same definition with the
+ * output frames s_t apart on Zp.  Sums are
  * accumulated in double starting from 0 and the bias is added last, once.
  * new_cache holds the last min(cache_keep, |Z|) frames of Z (the plain reading
  * of "the cache carries the trailing frames of the cache-augmented input").
@@ -25,7 +28,8 @@
  * This is the DEFINITION, not the paper's lowering: Z is materialised, the
  * causal pad is materialised as zero frames, every (k, r, s) term is visited
  * and no interval arithmetic is used.  Output sizes come from the usual
- * convolution length formula applied to the padded sequence.
+ * convolution length formula (stride s_t, no right pad) applied to the padded
+ * sequence.
  *
  * Layouts (all row-major, channels innermost, "NTHWC"):
  *   x         [N, T_x, H, W, Cin]
@@ -51,6 +55,7 @@ typedef struct {
     int s_h, s_w;
     int p_h, p_w;
     int d_t, d_h, d_w;
+    int s_t;        /* temporal stride (1 in the paper's supported contract) */
 } oracle_params;
 
 /* Output extents of the convolution over the padded sequence Zp.
@@ -61,14 +66,15 @@ int oracle_shape(const oracle_params* p, int* T_o, int* H_o, int* W_o,
         p->kw <= 0 || p->H <= 0 || p->W <= 0 || p->T_x < 0 ||
         p->cache_len < 0 || p->pad_t_base < 0 || p->cache_keep < 0 ||
         p->s_h <= 0 || p->s_w <= 0 || p->p_h < 0 || p->p_w < 0 ||
-        p->d_t <= 0 || p->d_h <= 0 || p->d_w <= 0)
+        p->d_t <= 0 || p->d_h <= 0 || p->d_w <= 0 || p->s_t <= 0)
         return -1;
     int z_len = p->cache_len + p->T_x;
     int p_l = p->pad_t_base - p->cache_len;
     int zp_len = z_len + p_l; /* pad in front, or crop when p_l < 0 */
     if (zp_len < 0) zp_len = 0;
-    /* standard length formula, stride 1, no right pad */
-    *T_o = zp_len - p->d_t * (p->kt - 1);
+    /* standard length formula, stride s_t, no right pad */
+    int tn = zp_len - p->d_t * (p->kt - 1) - 1;
+    *T_o = tn < 0 ? 0 : tn / p->s_t + 1;
     *H_o = (p->H + 2 * p->p_h - p->d_h * (p->kh - 1) - 1) / p->s_h + 1;
     *W_o = (p->W + 2 * p->p_w - p->d_w * (p->kw - 1) - 1) / p->s_w + 1;
     if (p->H + 2 * p->p_h - p->d_h * (p->kh - 1) - 1 < 0) *H_o = 0;
@@ -144,7 +150,7 @@ int oracle_forward(const oracle_params* p, const double* x, const double* cache,
                 for (int k = 0; k < kt; ++k)
                     for (int r = 0; r < kh; ++r)
                         for (int s = 0; s < kw; ++s) {
-                            int t = o + k * p->d_t;
+                            int t = o * p->s_t + k * p->d_t;
                             int yi = y * p->s_h + r * p->d_h - p->p_h;
                             int xi = xo * p->s_w + s * p->d_w - p->p_w;
                             if (yi < 0 || yi >= H || xi < 0 || xi >= Wd) continue;
@@ -209,7 +215,7 @@ int oracle_points(const oracle_params* p, const double* x, const double* cache,
         for (int k = 0; k < p->kt; ++k)
             for (int r = 0; r < p->kh; ++r)
                 for (int s = 0; s < p->kw; ++s) {
-                    int i = o + k * p->d_t;
+                    int i = o * p->s_t + k * p->d_t;
                     int yi = y * p->s_h + r * p->d_h - p->p_h;
                     int xi = xo * p->s_w + s * p->d_w - p->p_w;
                     const double* wrow =
@@ -224,7 +230,7 @@ int oracle_points(const oracle_params* p, const double* x, const double* cache,
 }
 
 /* Brute-force temporal tap scan.  For each tap k and each output frame o,
- * position o + k*d_t of Zp is a real frame of Z exactly when it is not one of
+ * position o*s_t + k*d_t of Zp is a real frame of Z exactly when it is not one of
  * the p_l pad frames and not past the end of Z.  The scan records, per tap,
  * the frame of Z read at output 0 (delta[k]), the smallest and one past the
  * largest output frame whose tap is real (o_l, o_h), and whether any is
@@ -240,7 +246,7 @@ int oracle_tap_scan(const oracle_params* p, int* T_o_out, int* delta, int* o_l,
     for (int k = 0; k < p->kt; ++k) {
         int first = -1, last = -1, count = 0;
         for (int o = 0; o < T_o; ++o) {
-            int zframe = (o + k * p->d_t) - p_l; /* Zp position -> Z frame */
+            int zframe = (o * p->s_t + k * p->d_t) - p_l; /* Zp position -> Z frame */
             if (zframe >= 0 && zframe < z_len) {
                 if (first < 0) first = o;
                 last = o;

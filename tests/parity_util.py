@@ -22,7 +22,7 @@ def oracle_params(c):
     return oracle.params(c.N, c.Cin, c.Cout, c.H, c.W, c.T_x, c.cache_len, kt=c.kt,
                          kh=c.kh, kw=c.kw, pad_t_base=c.pad_t_base,
                          cache_keep=c.cache_keep, stride=c.stride, pad=c.pad,
-                         dilation=c.dilation)
+                         dilation=c.dilation, stride_t=c.stride_t)
 
 
 def inputs_for(c, stream_base=0):

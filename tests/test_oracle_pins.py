@@ -34,7 +34,7 @@ def _params_from(d):
         d["N"], d["Cin"], d["Cout"], d["kt"], d["kh"], d["kw"], d["H"], d["W"],
         d["T_x"], d["cache_len"], d["pad_t_base"], d["cache_keep"],
         d["stride"][0], d["stride"][1], d["pad"][0], d["pad"][1],
-        d["dilation"][0], d["dilation"][1], d["dilation"][2])
+        d["dilation"][0], d["dilation"][1], d["dilation"][2], d.get("stride_t", 1))
 
 
 def _rand(shape, seed, stream):
@@ -59,7 +59,7 @@ def _torch_reference(p, x, cache, w, bias):
         z = F.pad(z[:, :, -p_l:], (p.p_w, p.p_w, p.p_h, p.p_h, 0, 0))
     wt = torch.from_numpy(w).permute(0, 4, 1, 2, 3)
     b = torch.from_numpy(bias) if bias is not None else None
-    y = F.conv3d(z, wt, b, stride=(1, p.s_h, p.s_w), padding=0,
+    y = F.conv3d(z, wt, b, stride=(p.s_t, p.s_h, p.s_w), padding=0,
                  dilation=(p.d_t, p.d_h, p.d_w))
     return y.permute(0, 2, 3, 4, 1).contiguous().numpy()
 
@@ -94,12 +94,23 @@ TORCH_CASES = [
     (1, 2, 3, 7, 5, 2, 1, 3, 3, 2, (1, 2), (2, 0), (1, 1, 2), None),
     (1, 3, 2, 5, 5, 2, 0, 3, 3, 3, (1, 1), (1, 1), (1, 1, 1), 1),   # p_base < d_t(kt-1)
 ]
+# temporal stride (the encoders' downsampling): same columns + s_t
+TORCH_CASES_ST = [
+    (1, 3, 4, 5, 6, 4, 2, 3, 3, 3, (1, 1), (1, 1), (1, 1, 1), None, 2),
+    (1, 2, 3, 4, 5, 5, 0, 3, 3, 3, (1, 1), (1, 1), (1, 1, 1), None, 2),   # odd |Z|
+    (2, 3, 2, 6, 5, 3, 1, 3, 3, 3, (2, 2), (1, 1), (1, 1, 1), None, 2),
+    (1, 2, 3, 5, 4, 6, 4, 3, 3, 3, (1, 1), (1, 1), (2, 1, 1), None, 2),   # d_t = 2
+    (1, 4, 4, 3, 3, 7, 2, 3, 1, 1, (1, 1), (0, 0), (1, 1, 1), None, 3),   # s_t = 3, 3x1x1
+    (1, 2, 2, 4, 4, 3, 0, 3, 3, 3, (1, 1), (1, 1), (1, 1, 1), 0, 2),      # p_base 0
+]
 
 
 def _case(ci):
-    N, Cin, Cout, H, W, T_x, cl, kt, kh, kw, st, pd, dl, pb = TORCH_CASES[ci]
+    row = (TORCH_CASES + TORCH_CASES_ST)[ci]
+    N, Cin, Cout, H, W, T_x, cl, kt, kh, kw, st, pd, dl, pb = row[:14]
+    s_t = row[14] if len(row) > 14 else 1
     p = oracle.params(N, Cin, Cout, H, W, T_x, cl, kt=kt, kh=kh, kw=kw,
-                      stride=st, pad=pd, dilation=dl, pad_t_base=pb)
+                      stride=st, pad=pd, dilation=dl, pad_t_base=pb, stride_t=s_t)
     x = _rand((N, T_x, H, W, Cin), ci, 1)
     cache = _rand((N, cl, H, W, Cin), ci, 2) if cl else None
     w = _rand((Cout, kt, kh, kw, Cin), ci, 3)
@@ -108,7 +119,7 @@ def _case(ci):
 
 
 def _run_pins_torch(lib):
-    for ci in range(len(TORCH_CASES)):
+    for ci in range(len(TORCH_CASES) + len(TORCH_CASES_ST)):
         p, x, cache, w, b = _case(ci)
         out, nc = oracle.forward(p, x, cache, w, b, lib=lib)
         ref = _torch_reference(p, x, cache, w, b)
@@ -130,7 +141,8 @@ def test_matches_torch_conv3d_float64(oracle_lib):
 
 def test_points_match_torch(oracle_lib):
     rng = np.random.default_rng(5)
-    for ci in (0, 1, 4, 5, 6, 9):
+    for ci in (0, 1, 4, 5, 6, 9, len(TORCH_CASES), len(TORCH_CASES) + 2,
+               len(TORCH_CASES) + 4):
         p, x, cache, w, b = _case(ci)
         ref = _torch_reference(p, x, cache, w, b)
         idx = np.stack([rng.integers(0, s, 64) for s in ref.shape], axis=1)
@@ -288,6 +300,55 @@ def test_chunked_equals_whole(oracle_lib, d_t, chunks):
     assert np.array_equal(np.concatenate(outs, axis=1), whole)
 
 
+@pytest.mark.parametrize("s_t,d_t,chunks", [(2, 1, (2, 2, 2, 2)), (2, 1, (4, 2, 6)),
+                                             (2, 2, (2, 4, 2, 4)), (3, 1, (3, 6, 3))])
+def test_chunked_equals_whole_temporal_stride(oracle_lib, s_t, d_t, chunks):
+    """With a temporal stride, threading the cache (the last p_l^base frames)
+    reproduces the whole-sequence call when every chunk boundary falls on a
+    multiple of s_t frames: the next chunk's first window then starts on the
+    stride grid of the whole sequence.  Bit-identical on integer data."""
+    rng = np.random.default_rng(8)
+    T = sum(chunks)
+    frames = _ints((1, T, 4, 5, 2), rng)
+    w = _ints((3, 3, 3, 3, 2), rng)
+    b = _ints((3,), rng, -9, 9)
+    mk = lambda n, cl: oracle.params(1, 2, 3, 4, 5, n, cl, dilation=(d_t, 1, 1), stride_t=s_t)
+    whole, _ = oracle.forward(mk(T, 0), frames, None, w, b, lib=oracle_lib)
+    outs, cache, t0 = [], None, 0
+    for n in chunks:
+        cl = 0 if cache is None else cache.shape[1]
+        out, cache = oracle.forward(mk(n, cl), frames[:, t0:t0 + n], cache, w, b, lib=oracle_lib)
+        outs.append(out)
+        t0 += n
+    assert np.array_equal(np.concatenate(outs, axis=1), whole)
+
+
+def test_temporal_stride_scan_matches_conv_support(oracle_lib):
+    """With s_t > 1 the scan's [o_l, o_h) per tap is still exactly the set of
+    output frames a tap's weight reaches (perturbation on the conv)."""
+    for cl, T_x, d_t, pb, s_t in itertools.product(range(0, 5), range(1, 7), (1, 2), (0, 2, 4),
+                                                   (2, 3)):
+        p = oracle.params(1, 1, 1, 1, 1, T_x, cl, kh=1, kw=1, pad=(0, 0),
+                          dilation=(d_t, 1, 1), pad_t_base=pb, stride_t=s_t)
+        T_o, _, _, _ = oracle.shape(p)
+        if T_o <= 0:
+            continue
+        T_s, delta, o_l, o_h, active = oracle.tap_scan(p, lib=oracle_lib)
+        assert T_s == T_o
+        x = np.ones((1, T_x, 1, 1, 1))
+        cache = np.ones((1, cl, 1, 1, 1)) if cl else None
+        for k in range(3):
+            w = np.zeros((1, 3, 1, 1, 1))
+            w[0, k] = 1.0
+            out, _ = oracle.forward(p, x, cache, w, None, lib=oracle_lib)
+            support = [o for o in range(T_o) if out[0, o, 0, 0, 0] != 0]
+            if active[k]:
+                assert support == list(range(o_l[k], o_h[k]))
+                assert 0 <= o_l[k] * s_t + delta[k] and (o_h[k] - 1) * s_t + delta[k] < cl + T_x
+            else:
+                assert support == [] and o_l[k] == o_h[k] == 0
+
+
 def test_intervals_equal_length_exhaustive(oracle_lib):
     for cl, T_x, d_t, pb in itertools.product(range(0, 7), range(1, 7), (1, 2, 3), range(0, 7)):
         p = oracle.params(1, 1, 1, 1, 1, T_x, cl, kh=1, kw=1, pad=(0, 0),
@@ -307,8 +368,14 @@ def test_intervals_equal_length_exhaustive(oracle_lib):
 MUTANTS = {
     "channel_reversed": ("acc += zrow[ci] * wrow[ci];",
                          "acc += zrow[ci] * wrow[Cin - 1 - ci];"),
-    "taps_flipped": ("int t = o + k * p->d_t;",
-                     "int t = o + (kt - 1 - k) * p->d_t;"),
+    "taps_flipped": ("int t = o * p->s_t + k * p->d_t;",
+                     "int t = o * p->s_t + (kt - 1 - k) * p->d_t;"),
+    "temporal_stride_dropped": ("int t = o * p->s_t + k * p->d_t;",
+                                "int t = o + k * p->d_t;"),
+    # (a mutant that over-counts outputs would read past Zp; this one loses
+    # the last output whenever tn is a multiple of s_t, e.g. |Zp| = 7, s_t = 2)
+    "temporal_stride_length": ("*T_o = tn < 0 ? 0 : tn / p->s_t + 1;",
+                               "*T_o = tn < 0 ? 0 : (tn + 1) / p->s_t;"),
     "pad_sign": ("int yi = y * p->s_h + r * p->d_h - p->p_h;",
                  "int yi = y * p->s_h + r * p->d_h + p->p_h;"),
     "bias_twice": ("if (bias) acc += bias[co];\n                out[",
