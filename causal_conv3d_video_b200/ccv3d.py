@@ -225,7 +225,7 @@ def desc_for(conv) -> ccv3d_desc:
                      T_x=conv.T_x, cache_len=conv.cache_len, kt=conv.kt, kh=conv.kh,
                      kw=conv.kw, pad_t_base=conv.pad_t_base, cache_keep=conv.cache_keep,
                      stride=conv.stride, pad=conv.pad, dilation=conv.dilation,
-                     dtype=conv.dtype, has_bias=conv.has_bias)
+                     dtype=conv.dtype, has_bias=conv.has_bias, stride_t=conv.stride_t)
 
 
 class Plan:

@@ -3,9 +3,11 @@
 // The planner computes the temporal bookkeeping of "Cache-Aware Conv3D
 // Lowering Across Embedded World-Model Decoders" (Sec. 4) in integer
 // arithmetic: |Z| = |C| + T_x, p_l = p_l^base - |C|,
-// T_o = |Z| + p_l - d_t (k_t - 1), delta_k = k d_t - p_l and the valid output
-// interval [o_l, o_h) = [max(0, -delta_k), min(T_o, |Z| - delta_k)) of every
-// tap (the intersection of 0 <= o < T_o and 0 <= o + delta_k < |Z|).  Nothing
+// T_o = floor((|Z| + p_l - d_t (k_t - 1) - 1) / s_t) + 1, delta_k = k d_t - p_l
+// and the valid output interval of every tap, [o_l, o_h) =
+// [max(0, ceil(-delta_k / s_t)), min(T_o, ceil((|Z| - delta_k) / s_t))) (the
+// intersection of 0 <= o < T_o and 0 <= o s_t + delta_k < |Z|; s_t = 1 in the
+// paper, s_t > 1 for the encoders' temporal downsampling).  Nothing
 // concatenates C and X: the kernels pick each source frame from one or the
 // other.
 #include <cuda.h>
@@ -74,6 +76,11 @@ EncodeTiledFn encode_fn() {
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// ceil(a / b) for b > 0 and any sign of a.
+int ceil_div_floor0(long long a, long long b) {
+    return a >= 0 ? (int)((a + b - 1) / b) : -(int)((-a) / b);
+}
+
 // Planner: the paper's closed forms.  Returns CCV3D_OK or the refusal code.
 ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
     if (d.N < 0 || d.Cin <= 0 || d.Cout <= 0 || d.kt <= 0 || d.kh <= 0 || d.kw <= 0 ||
@@ -82,12 +89,14 @@ ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
         d.pad_h < 0 || d.pad_w < 0 || d.dil_t <= 0 || d.dil_h <= 0 || d.dil_w <= 0 ||
         d.groups <= 0)
         return CCV3D_ERR_INVALID;
-    if (d.stride_t != 1 || d.groups != 1 || d.kt != 3 ||
-        (d.dtype != CCV3D_BF16 && d.dtype != CCV3D_FP32))
+    if (d.groups != 1 || d.kt != 3 || (d.dtype != CCV3D_BF16 && d.dtype != CCV3D_FP32))
         return CCV3D_ERR_UNSUPPORTED;
+    const int s_t = d.stride_t;
     p->z_len = d.cache_len + d.T_x;
     p->p_l = d.pad_t_base - d.cache_len;
-    p->T_o = p->z_len + p->p_l - d.dil_t * (d.kt - 1);
+    // output o's tap k reads frame o*s_t + delta_k of Z; no right pad
+    const long long tn = (long long)p->z_len + p->p_l - (long long)d.dil_t * (d.kt - 1) - 1;
+    p->T_o = tn < 0 ? 0 : (int)(tn / s_t + 1);
     const long long hn = (long long)d.H + 2LL * d.pad_h - (long long)d.dil_h * (d.kh - 1) - 1;
     const long long wn = (long long)d.W + 2LL * d.pad_w - (long long)d.dil_w * (d.kw - 1) - 1;
     p->H_o = hn < 0 ? 0 : (int)(hn / d.stride_h + 1);
@@ -97,8 +106,9 @@ ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
         p->delta[k] = p->o_l[k] = p->o_h[k] = 0;
         if (k >= d.kt) continue;
         const int delta = k * d.dil_t - p->p_l;
-        const int lo = std::max(0, -delta);
-        const int hi = std::min(p->T_o, p->z_len - delta);
+        // o*s_t + delta in [0, |Z|)  <=>  ceil(-delta/s_t) <= o < ceil((|Z|-delta)/s_t)
+        const int lo = std::max(0, ceil_div_floor0(-delta, s_t));
+        const int hi = std::min(p->T_o, ceil_div_floor0(p->z_len - delta, s_t));
         p->delta[k] = delta;
         if (hi > lo) {
             p->o_l[k] = lo;
@@ -448,6 +458,7 @@ CopyJob make_copy(const ccv3d_plan_s* p, const void* x, const void* cache, void*
 Taps make_taps(const ccv3d_plan_s* p) {
     Taps t;
     t.kt = p->d.kt;
+    t.s_t = p->d.stride_t;
     for (int k = 0; k < kMaxTaps; ++k) {
         t.delta[k] = p->delta[k];
         t.o_l[k] = p->o_l[k];

@@ -4,7 +4,7 @@
 //
 // Each thread owns one output pixel and CO_T consecutive output channels and
 // walks the active taps only: for output frame o, tap k is skipped unless
-// o_l[k] <= o < o_h[k] (paper, Sec. 4), and its source frame o + delta_k is
+// o_l[k] <= o < o_h[k] (paper, Sec. 4), and its source frame o*s_t + delta_k is
 // read from the cache or the input by pointer select.  Blocks past
 // conv_blocks write new_cache.
 #pragma once
@@ -67,7 +67,7 @@ conv_simt_kernel(const __grid_constant__ SimtParams p) {
 
     for (int k = 0; k < p.taps.kt; ++k) {
         if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
-        const int t = o + p.taps.delta[k];
+        const int t = o * p.taps.s_t + p.taps.delta[k];
         const T* frame = t < p.cache_len
                              ? cache + ((long long)n * p.cache_len + t) * p.H * p.W * p.Cin
                              : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * p.W * p.Cin;

@@ -5,7 +5,7 @@
 // (n, o, y, x) of one output frame, columns = Cout, reduction over
 // (active tap k, r, s, ci).  A tile of 128 output pixels is a box_h x box_w
 // spatial box of frame o.  For every active tap k the source frame
-// t = o + delta_k is picked from the cache or the input tensor map (no
+// t = o*s_t + delta_k is picked from the cache or the input tensor map (no
 // concatenation), and for every spatial tap (r, s) one TMA box load brings the
 // shifted, strided box of BK input channels, zero-filled outside the image.
 // Weights W[co, k, r, s, ci] are read in place (K-major rows).

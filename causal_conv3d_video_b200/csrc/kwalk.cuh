@@ -52,7 +52,7 @@ struct KWalk {
 };
 
 // Source of one temporal tap of output frame o (paper, Sec. 4): frame
-// t = o + delta_k of Z, taken from the cache when t < |C|, else from x.
+// t = o*s_t + delta_k of Z, taken from the cache when t < |C|, else from x.
 struct TapSrc {
     const CUtensorMap* map;
     int frame;  // frame coordinate in that tensor map (n * T + t)
@@ -61,7 +61,7 @@ struct TapSrc {
 
 __device__ __forceinline__ TapSrc tap_source(const TcParams& p, int k, int n, int o) {
     TapSrc ts;
-    const int t = o + p.taps.delta[k];
+    const int t = o * p.taps.s_t + p.taps.delta[k];
     if (t < p.cache_len) {
         ts.map = &p.tmap_c;
         ts.frame = n * p.cache_len + t;

@@ -25,6 +25,7 @@ struct CopyJob {
 // reads frame o + delta[k] of Z, and is active iff o_l[k] <= o < o_h[k].
 struct Taps {
     int kt;
+    int s_t;                // temporal stride: output o's tap k reads frame o*s_t + delta[k]
     int delta[kMaxTaps];
     int o_l[kMaxTaps];
     int o_h[kMaxTaps];

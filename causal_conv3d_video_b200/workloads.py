@@ -28,13 +28,14 @@ class Conv:
     kw: int = 3
     pad_t_base: int | None = None
     cache_keep: int | None = None
-    stride: tuple = (1, 1)
+    stride: tuple = (1, 1)          # (s_h, s_w)
     pad: tuple = (1, 1)
     dilation: tuple = (1, 1, 1)
     dtype: str = "bf16"
     sigma_b: float = 0.02
     has_bias: bool = True
     seed: int = 0
+    stride_t: int = 1               # temporal stride (> 1: encoder downsampling)
 
     def __post_init__(self):
         if self.pad_t_base is None:
@@ -85,9 +86,16 @@ C4_STRIDE = Conv("bf16_192ch_s2_360x640_c2_t1", 192, 192, 360, 640, T_x=1,
                  cache_len=2, stride=(2, 2))
 C4_C1 = C2.replace(name="bf16_384ch_90x160_c1_t1", cache_len=1)
 C4_ODD = Conv("bf16_192ch_89x157_c2_t1", 192, 192, 89, 157, T_x=1, cache_len=2)
+# encoder-side temporal downsampling (stride 2 in time; the paper leaves these
+# calls on native Conv3D): a 3x1x1 time conv and a 3x3x3 conv, 4-frame chunks
+C6_ST2_TIME = Conv("bf16_3x1x1_384ch_st2_180x320_c2_t4", 384, 384, 180, 320, T_x=4,
+                   cache_len=2, kh=1, kw=1, pad=(0, 0), stride_t=2)
+C6_ST2 = Conv("bf16_192ch_st2_180x320_c2_t4", 192, 192, 180, 320, T_x=4, cache_len=2,
+              stride_t=2)
 
 WORKLOADS = {c.name: c for c in (
-    C1, C2, C2_EMPTY, C3, C3B, C4_TIME, C4_DIL, C4_STRIDE, C4_C1, C4_ODD)}
+    C1, C2, C2_EMPTY, C3, C3B, C4_TIME, C4_DIL, C4_STRIDE, C4_C1, C4_ODD, C6_ST2_TIME,
+    C6_ST2)}
 # cache-length sweep {0,1,2} on the bottleneck and on the stride-2 signature
 for _base in (C2, C4_STRIDE):
     for _c in (0, 1, 2):
@@ -168,4 +176,4 @@ def decode17_schedule(scale_hw: tuple | None = None):
 
 def signature(c: Conv):
     return (c.Cin, c.Cout, c.kt, c.kh, c.kw, c.H, c.W, c.T_x, c.cache_len,
-            c.stride, c.pad, c.dilation, c.dtype)
+            c.stride, c.pad, c.dilation, c.dtype, c.stride_t)

@@ -3,17 +3,23 @@
  *
  * The operator ("Cache-Aware Conv3D Lowering Across Embedded World-Model
  * Decoders", Sec. 4): a temporal cache C and the current frames X form the
- * cache-augmented input Z = [C; X]_T.  With unit temporal stride, one group,
- * temporal kernel k_t = 3 and effective left pad p_l = p_l^base - |C|_T,
- * output frame o of tap k reads frame o + delta_k of Z, delta_k = k*d_t - p_l;
- * frames outside Z contribute zero.  The output is the sum over taps of a
- * spatial cross-correlation with W_k = W[:, :, k, :, :] (PyTorch convention,
- * spatial stride s, padding p, dilation d), plus the bias exactly once.
- * Tap k is active on the output interval [o_l, o_h) where
- *   o_l = max(0, -delta_k),  o_h = min(T_o, |Z|_T - delta_k),
- * and reads the equally long source interval [o_l + delta_k, o_h + delta_k).
+ * cache-augmented input Z = [C; X]_T.  With one group, temporal kernel k_t = 3
+ * and effective left pad p_l = p_l^base - |C|_T, output frame o of tap k reads
+ * frame o*s_t + delta_k of Z, delta_k = k*d_t - p_l; frames outside Z
+ * contribute zero.  The paper's lowering has unit temporal stride (s_t = 1);
+ * s_t > 1 (the encoders' temporal downsampling, which the paper leaves on
+ * native Conv3D) is the same sum with output frames s_t apart, and
+ * T_o = floor((|Z| + p_l - d_t*(k_t-1) - 1) / s_t) + 1.  The output is the sum
+ * over taps of a spatial cross-correlation with W_k = W[:, :, k, :, :]
+ * (PyTorch convention, spatial stride s, padding p, dilation d), plus the bias
+ * exactly once.  Tap k is active on the output interval [o_l, o_h) where
+ *   o_l = max(0, ceil(-delta_k / s_t)),  o_h = min(T_o, ceil((|Z|_T - delta_k) / s_t)),
+ * and reads the source frames o_l*s_t + delta_k, ..., (o_h-1)*s_t + delta_k
+ * (for s_t = 1 the equally long interval [o_l + delta_k, o_h + delta_k)).
  * Each call also writes new_cache = the last min(cache_keep, |Z|_T) frames of
- * Z, ready to be passed as the next call's cache.
+ * Z, ready to be passed as the next call's cache.  (With s_t > 1, threading
+ * the cache this way reproduces one whole-sequence call when every chunk
+ * boundary falls on a multiple of s_t frames.)
  *
  * Memory layout (every tensor dense, row-major, channels innermost -- the
  * physical order of PyTorch's channels_last_3d):
@@ -64,8 +70,8 @@ typedef enum {
     CCV3D_ERR_INVALID = 1,      /* bad or inconsistent argument (NULL plan or
                                    pointer, negative size, forward's
                                    stride/pad/dilation differ from the plan) */
-    CCV3D_ERR_UNSUPPORTED = 2,  /* outside the contract: stride_t != 1,
-                                   groups != 1, k_t != 3, unknown dtype */
+    CCV3D_ERR_UNSUPPORTED = 2,  /* outside the contract: groups != 1,
+                                   k_t != 3, unknown dtype */
     CCV3D_ERR_EMPTY_OUTPUT = 3, /* T_o, H_o or W_o would be <= 0, or N == 0 */
     CCV3D_ERR_ALIGNMENT = 4,    /* a pointer is not 16-byte aligned */
     CCV3D_ERR_ALIAS = 5,        /* new_cache overlaps x or cache, or out
@@ -85,7 +91,7 @@ typedef struct {
     int cache_len;        /* |C|_T, frames in cache, >= 0 */
     int pad_t_base;       /* p_l^base, causal left pad with an empty cache */
     int cache_keep;       /* frames of Z kept in new_cache (usually p_l^base) */
-    int stride_t;         /* must be 1 */
+    int stride_t;         /* temporal stride s_t >= 1 (1: the paper's decoder calls) */
     int stride_h, stride_w;
     int pad_h, pad_w;     /* symmetric zero padding */
     int dil_t, dil_h, dil_w;

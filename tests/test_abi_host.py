@@ -40,13 +40,15 @@ def _plan(**kw):
     return ccv3d.ccv3d_plan(ccv3d.make_desc(**kw))
 
 
+@pytest.mark.parametrize("s_t", [1, 2, 3])
 @pytest.mark.parametrize("d_t", [1, 2, 3])
-def test_planner_matches_oracle_scan_exhaustive(d_t):
+def test_planner_matches_oracle_scan_exhaustive(d_t, s_t):
     """Intervals of the closed forms == brute-force scan, bit for bit."""
     for cl, T_x, pb in itertools.product(range(0, 7), range(1, 7), range(0, 7)):
         kw = dict(N=1, Cin=16, Cout=16, H=4, W=4, T_x=T_x, cache_len=cl,
-                  dilation=(d_t, 1, 1), pad_t_base=pb)
-        op = oracle.params(1, 16, 16, 4, 4, T_x, cl, dilation=(d_t, 1, 1), pad_t_base=pb)
+                  dilation=(d_t, 1, 1), pad_t_base=pb, stride_t=s_t)
+        op = oracle.params(1, 16, 16, 4, 4, T_x, cl, dilation=(d_t, 1, 1), pad_t_base=pb,
+                           stride_t=s_t)
         T_o, H_o, W_o, keep = oracle.shape(op)
         if T_o <= 0:
             with pytest.raises(ccv3d.CCV3DError) as e:
@@ -70,7 +72,7 @@ def test_planner_shapes_match_oracle_on_workloads(name):
     c = workloads.WORKLOADS[name]
     op = oracle.params(c.N, c.Cin, c.Cout, c.H, c.W, c.T_x, c.cache_len, kt=c.kt,
                        kh=c.kh, kw=c.kw, pad_t_base=c.pad_t_base, cache_keep=c.cache_keep,
-                       stride=c.stride, pad=c.pad, dilation=c.dilation)
+                       stride=c.stride, pad=c.pad, dilation=c.dilation, stride_t=c.stride_t)
     plan = ccv3d.Plan(ccv3d.desc_for(c))
     T_o, H_o, W_o, keep = oracle.shape(op)
     _, delta, o_l, o_h, _ = oracle.tap_scan(op)
@@ -84,7 +86,8 @@ def test_planner_shapes_match_oracle_on_workloads(name):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(kt=2), ccv3d.CCV3D_ERR_UNSUPPORTED),
-    (dict(stride_t=2), ccv3d.CCV3D_ERR_UNSUPPORTED),
+    (dict(stride_t=0), ccv3d.CCV3D_ERR_INVALID),
+    (dict(stride_t=2, T_x=2, cache_len=0, pad_t_base=0), ccv3d.CCV3D_ERR_EMPTY_OUTPUT),  # |Zp| = 2 < 3
     (dict(groups=2), ccv3d.CCV3D_ERR_UNSUPPORTED),
     (dict(Cin=0), ccv3d.CCV3D_ERR_INVALID),
     (dict(T_x=0), ccv3d.CCV3D_ERR_INVALID),

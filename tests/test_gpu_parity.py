@@ -133,6 +133,45 @@ def test_small_halo_strips(c, halo):
     assert (call.plan.kernel == "tc_pair_halo") == bool(halo), call.plan.kernel
 
 
+SMALL_ST = [
+    # temporal stride (the encoders' downsampling): output frames s_t apart on Zp
+    Conv("st2_c2_t4", 64, 64, 20, 37, T_x=4, cache_len=2, stride_t=2),
+    Conv("st2_c0_t5", 64, 96, 12, 20, T_x=5, cache_len=0, stride_t=2),      # odd |Zp|
+    Conv("st2_3x1x1", 128, 384, 10, 16, T_x=4, cache_len=2, kh=1, kw=1, pad=(0, 0),
+         stride_t=2),
+    Conv("st2_dt2_c4", 64, 64, 18, 32, T_x=2, cache_len=4, dilation=(2, 1, 1), stride_t=2),
+    Conv("st3_c1_t6", 32, 48, 10, 12, T_x=6, cache_len=1, stride_t=3),
+    Conv("st2_s2", 64, 64, 36, 64, T_x=2, cache_len=2, stride=(2, 2), stride_t=2),
+    Conv("st2_batch2", 32, 48, 10, 12, T_x=4, cache_len=2, N=2, stride_t=2),
+]
+
+
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+@pytest.mark.parametrize("c", SMALL_ST, ids=lambda c: c.name)
+def test_small_temporal_stride(c, kernel):
+    call, _ = _run_small(c, env=KERNELS[kernel])
+    assert call.plan.path["tc"] is True
+
+
+@pytest.mark.parametrize("pairs", [2, 3])
+def test_small_temporal_stride_split_tiles(pairs):
+    _run_small(SMALL_ST[0], env={"CCV3D_PERSIST": 1, "CCV3D_SK_PAIRS": pairs})
+
+
+def test_small_temporal_stride_halo():
+    c = Conv("st2_halo", 96, 96, 3, 384, T_x=4, cache_len=2, stride_t=2)
+    call, _ = _run_small(c, env={"CCV3D_HALO": 1, "CCV3D_PERSIST": 0})
+    assert call.plan.kernel == "tc_pair_halo"
+
+
+@pytest.mark.parametrize("c", [SMALL_ST[0], SMALL_ST[4],
+                               Conv("st2_f32", 8, 12, 13, 17, T_x=3, cache_len=1, stride_t=2,
+                                    dtype="fp32")], ids=lambda c: c.name)
+def test_small_temporal_stride_simt(c):
+    call, _ = _run_small(c, force_simt=c.dtype == "bf16")
+    assert call.plan.path["tc"] is False
+
+
 @pytest.mark.parametrize("c", SMALL[:4] + SMALL[12:15] + SMALL[19:21], ids=lambda c: c.name)
 def test_small_simt_bf16(c):
     call, _ = _run_small(c, force_simt=True)

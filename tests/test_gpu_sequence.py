@@ -122,3 +122,35 @@ def test_decode17_full_size_sampled(call):
     ref = oracle.points(oracle_params(c), inp["x"], inp["cache"], inp["w"], inp["bias"], idx)
     got = out[tuple(torch.from_numpy(idx.T).cuda())].double().cpu().numpy()
     assert_close(got, ref, c.dtype, c.name)
+
+
+@pytest.mark.parametrize("s_t,chunks", [(2, (2, 4, 2, 4)), (2, (4, 2, 2)), (3, (3, 6, 3))])
+def test_temporal_stride_chunked_equals_whole(s_t, chunks):
+    """Encoder-style temporal downsampling: with chunk boundaries on multiples
+    of s_t, threading new_cache reproduces one whole-sequence call."""
+    base = workloads.Conv("st", 64, 64, 16, 32, T_x=1, cache_len=0, stride_t=s_t)
+    w_np, b_np = _module_weights(base, 90 + s_t)
+    w, b = to_device(w_np, base.dtype), to_device(b_np, base.dtype)
+    T = sum(chunks)
+    frames = synth.tensor((1, T, base.H, base.W, base.Cin), 1.0, 9100 + s_t, synth.STREAM_X,
+                          base.dtype)
+    outs, cache_np, cache_dev, t0 = [], None, None, 0
+    for i, n in enumerate(chunks):
+        cl = 0 if cache_np is None else cache_np.shape[1]
+        c = base.replace(name=f"st{s_t}_k{i}", T_x=n, cache_len=cl)
+        x_np = frames[:, t0:t0 + n]
+        out, nc = _run(c, to_device(x_np, c.dtype), cache_dev, w, b)
+        torch.cuda.synchronize()
+        if i < 2:
+            ref, _ = oracle.forward(oracle_params(c), x_np, cache_np, w_np, b_np)
+            assert_close(out.double().cpu().numpy(), ref, c.dtype, c.name)
+        outs.append(out)
+        cache_np, cache_dev = nc.double().cpu().numpy().astype(np.float32), nc
+        t0 += n
+    whole, _ = _run(base.replace(name="whole", T_x=T), to_device(frames, base.dtype), None, w, b)
+    torch.cuda.synchronize()
+    chunked = torch.cat(outs, dim=1)
+    assert chunked.shape == whole.shape
+    g, r = chunked.double().cpu().numpy(), whole.double().cpu().numpy()
+    rms = float(np.sqrt(np.mean(r * r)))
+    assert float(np.max(np.abs(g - r))) <= TOL[base.dtype] * rms
