@@ -75,6 +75,8 @@ def _bind(lib):
     lib.oracle_tap_scan.argtypes = [P, ip, ip, ip, ip, ip]
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
+    lib.oracle_quantize_u8.argtypes = [dp, ctypes.c_longlong, ctypes.POINTER(ctypes.c_uint8)]
+    lib.oracle_quantize_u8.restype = ctypes.c_int
     for f in (lib.oracle_shape, lib.oracle_forward, lib.oracle_points,
               lib.oracle_tap_scan):
         f.restype = ctypes.c_int
@@ -179,6 +181,17 @@ def _check(p, x, cache, w, bias):
         raise ValueError(f"w shape {w.shape}")
     if bias is not None and bias.shape != (p.Cout,):
         raise ValueError("bias shape")
+
+
+def quantize_u8(values, lib=None) -> np.ndarray:
+    """uint8 frames from decoded values (fp32 or bf16 numbers given as any
+    float array): trunc(clamp(fp32(v) * 255, 0, 255)), NaN -> 0."""
+    v = np.ascontiguousarray(np.asarray(values, np.float64))
+    out = np.zeros(v.shape, np.uint8)
+    (lib or load()).oracle_quantize_u8(
+        v.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), v.size,
+        out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out
 
 
 def threads(lib=None) -> int:

@@ -268,6 +268,26 @@ int oracle_tap_scan(const oracle_params* p, int* T_o_out, int* delta, int* o_l,
     return 0;
 }
 
+/* Post-decode uint8 quantisation of decoded frames (FastVideo pull request
+ * "Quantize frames to uint8 on-device before the post-decode D->H copy",
+ * Summary and Correctness): each value is multiplied by 255, clamped to
+ * [0, 255] and cast to uint8, the cast truncating toward zero as PyTorch's
+ * float -> uint8 conversion does.  The product is taken in fp32, the decoded
+ * video's precision on that page, for fp32 and bf16 inputs alike (a bf16
+ * input is widened to fp32 first, exactly).  A NaN clamps to 0 (C's fmaxf
+ * returns the non-NaN operand).  `in` holds the input values widened to
+ * double (exact for fp32/bf16 values).  Returns 0. */
+int oracle_quantize_u8(const double* in, long long n, uint8_t* out) {
+    for (long long i = 0; i < n; ++i) {
+        float v = (float)in[i];          /* the fp32 value, exactly */
+        float y = v * 255.0f;            /* one fp32 multiply */
+        y = fmaxf(y, 0.0f);              /* NaN -> 0 */
+        y = fminf(y, 255.0f);
+        out[i] = (uint8_t)(int)y;        /* truncation toward zero */
+    }
+    return 0;
+}
+
 /* Threads an OpenMP region of this library uses (1 without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

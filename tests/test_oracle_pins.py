@@ -364,6 +364,35 @@ def test_intervals_equal_length_exhaustive(oracle_lib):
                 assert 0 <= src_l < src_h <= cl + T_x
 
 
+# ---- post-decode uint8 quantisation ---------------------------------------
+def _run_pins_quantize(lib):
+    """trunc(clamp(fp32(v) * 255, 0, 255)) -- the page's expression
+    (x * 255).clamp_(0, 255).to(uint8) -- pinned by closed forms, by torch's
+    CPU evaluation of that expression, and exhaustively over bf16."""
+    # closed forms: truncation (0.5 -> 127, not 128), clamping (no wraparound)
+    special = np.array([0.0, 1.0, 0.5, 0.25, -0.1, 1.2, -3.0, 7.5, np.inf, -np.inf, np.nan,
+                        254.5 / 255, 1e-30, -0.0], np.float32)
+    want = np.array([0, 255, 127, 63, 0, 255, 0, 255, 255, 0, 0, 254, 0, 0], np.uint8)
+    got = oracle.quantize_u8(special.astype(np.float64), lib=lib)
+    assert np.array_equal(got, want), (got, want)
+    # torch on random fp32 values around [0, 1], and on exact k/255 grid points
+    rng = np.random.default_rng(17)
+    v = np.concatenate([rng.uniform(-0.1, 1.1, 20000), np.arange(256) / 255.0,
+                        (np.arange(256) + 0.5) / 255.0]).astype(np.float32)
+    ref = (torch.from_numpy(v) * 255).clamp_(0, 255).to(torch.uint8).numpy()
+    assert np.array_equal(oracle.quantize_u8(v.astype(np.float64), lib=lib), ref)
+    # every finite bf16 value, widened exactly to fp32, multiplied in fp32
+    bits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    f = bits.float()
+    f = f[torch.isfinite(f)]
+    ref = (f * 255).clamp_(0, 255).to(torch.uint8).numpy()
+    assert np.array_equal(oracle.quantize_u8(f.double().numpy(), lib=lib), ref)
+
+
+def test_quantize_u8_pins(oracle_lib):
+    _run_pins_quantize(oracle_lib)
+
+
 # ---- planted mistakes: each mutant of the oracle must fail a pin ----------
 MUTANTS = {
     "channel_reversed": ("acc += zrow[ci] * wrow[ci];",
@@ -385,6 +414,8 @@ MUTANTS = {
     "dilation_dropped": ("int xi = xo * p->s_w + s * p->d_w - p->p_w;\n                            if",
                          "int xi = xo * p->s_w + s - p->p_w;\n                            if"),
     "oldest_frames_kept": ("(z_len - keep)) * frame", "0) * frame"),
+    "quantize_rounds": ("out[i] = (uint8_t)(int)y;", "out[i] = (uint8_t)(int)(y + 0.5f);"),
+    "quantize_unclamped": ("y = fminf(y, 255.0f);", "y = y;"),
 }
 
 
@@ -400,7 +431,7 @@ def test_planted_mistake_is_caught(tmp_path, name):
                            str(mut), "-o", so, "-lm"])
     lib = oracle.load(so)
     caught = False
-    for pin in (_run_pins_hand, _run_pins_torch):
+    for pin in (_run_pins_hand, _run_pins_torch, _run_pins_quantize):
         try:
             pin(lib)
         except AssertionError:
