@@ -330,7 +330,7 @@ def run_gpu(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) activations, N(0,1/(Cin*27)) weights)",
         "config": {
             "workload": conv.name, "N": conv.N, "Cin": conv.Cin, "Cout": conv.Cout,
-            "kernel": [conv.kt, conv.kh, conv.kw], "H": conv.H, "W": conv.W,
+            "ksize": [conv.kt, conv.kh, conv.kw], "H": conv.H, "W": conv.W,
             "T_x": conv.T_x, "cache_len": conv.cache_len, "stride": list(conv.stride),
             "pad": list(conv.pad), "dilation": list(conv.dilation),
             "gflop_per_call": round(flops / 1e9, 3), "mb_per_call": round(nbytes / 1e6, 2),
@@ -363,7 +363,17 @@ def run_gpu(args, rank, world, local_rank):
                         "over upload/compute/download streams"},
         "gpu_launches": int(launches),
         "clocks": csum,
+        "memory": {
+            "device_workspace_bytes": int(plan.stats()["workspace_bytes"]),
+            "status_block_bytes": 256,
+            "intermediate_tensors": 0,
+            "what": "device memory the library holds besides the caller's x, cache, W, bias, "
+                    "out and new_cache: no concatenated [C;X], no per-tap weight slices, no "
+                    "accumulation buffer",
+        },
     }
+    if world == 1:
+        line["quantize_u8"] = run_quantize(dev)
     if args.sequence:
         line["decode17"] = run_sequence(args, dev)
     if not args.no_cpu_baseline and world == 1:
@@ -372,6 +382,70 @@ def run_gpu(args, rank, world, local_rank):
 
 
 # ------------------------------------------------- decode-sequence leg
+def run_quantize(dev, steps=200):
+    """The post-decode step: uint8 frames from a decoded 17-frame 720x1280
+    RGB fp32 video (47 M values, 235 MB moved per call), timed with CUDA
+    events over two rotating buffers (2 x 188 MB > L2); plus the device-to-host
+    copy of the frames, fp32 as decoded vs quantised on the device first."""
+    import torch
+    from causal_conv3d_video_b200 import ccv3d
+
+    shape = (1, 17, 720, 1280, 3)
+    n = 1
+    for d in shape:
+        n *= d
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3)
+    xs = [torch.rand(shape, generator=gen, device=dev) for _ in range(2)]
+    outs = [torch.empty(shape, dtype=torch.uint8, device=dev) for _ in range(2)]
+    stream = torch.cuda.current_stream(dev)
+    for i in range(6):
+        ccv3d.ccv3d_quantize_u8(xs[i % 2], outs[i % 2], stream)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        ccv3d.ccv3d_quantize_u8(xs[i % 2], outs[i % 2], stream)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    us = statistics.median([ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(steps)])
+    nbytes = 5 * n
+    peaks = load_peaks()
+    h32 = torch.empty(shape, dtype=torch.float32, pin_memory=True)
+    h8 = torch.empty(shape, dtype=torch.uint8, pin_memory=True)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        best = float("inf")
+        for _ in range(3):
+            torch.cuda.synchronize()
+            ea.record(stream)
+            fn()
+            eb.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, ea.elapsed_time(eb))
+        return best
+
+    d2h_fp32 = timed(lambda: h32.copy_(xs[0], non_blocking=True))
+
+    def quant_then_copy():
+        ccv3d.ccv3d_quantize_u8(xs[0], outs[0], stream)
+        h8.copy_(outs[0], non_blocking=True)
+
+    d2h_u8 = timed(quant_then_copy)
+    ok = torch.equal(h8.to(dev), outs[0])
+    return {"values": n, "us_per_call_median": round(us, 2),
+            "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+            "roofline": {"bound": "hbm", "achieved": round(nbytes / (us * 1e-6) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                         "bytes_per_value": 5},
+            "d2h_fp32_ms": round(d2h_fp32, 3), "quantize_plus_d2h_u8_ms": round(d2h_u8, 3),
+            "copied_back_ok": bool(ok),
+            "what": "ccv3d_quantize_u8 on a decoded 17x720x1280x3 fp32 video; D2H into pinned "
+                    "host memory of the fp32 video vs quantise-on-device + uint8 copy"}
+
+
 def run_sequence(args, dev):
     """Time the synthetic 17-frame decode: 164 calls over 28 signatures, each
     module's cache threaded from chunk to chunk (ping-pong buffers), all on one

@@ -25,7 +25,7 @@ CCV3D_MAX_KT = 3
 EXPORTED = ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_plan_path", "ccv3d_forward",
             "ccv3d_get_stats", "ccv3d_get_status", "ccv3d_destroy", "ccv3d_strerror",
             "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout", "ccv3d_forward_noalloc",
-            "ccv3d_plan_kernel", "ccv3d_plan_tiling")
+            "ccv3d_plan_kernel", "ccv3d_plan_tiling", "ccv3d_quantize_u8")
 CCV3D_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -72,6 +72,8 @@ def _load():
     lib.ccv3d_plan_sizes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t),
                                      ctypes.POINTER(ctypes.c_size_t), ip]
     lib.ccv3d_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.ccv3d_quantize_u8.argtypes = [vp, ctypes.c_int, vp, ctypes.c_longlong, vp]
+    lib.ccv3d_quantize_u8.restype = ctypes.c_int
     lib.ccv3d_forward_noalloc.argtypes = [ctypes.POINTER(ccv3d_desc), vp, vp, vp, vp, vp, vp,
                                           ip, ip, ip, vp]
     for f in ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_forward", "ccv3d_get_stats",
@@ -198,6 +200,23 @@ def ccv3d_get_status(plan) -> int:
 
 def ccv3d_destroy(plan) -> None:
     lib.ccv3d_destroy(plan)
+
+
+def ccv3d_quantize_u8(x, out, stream=None, check: bool = True) -> int:
+    """uint8 frames from decoded values on the device: out = trunc(clamp(
+    fp32(x) * 255, 0, 255)), NaN -> 0.  x: a float32 or bfloat16 device
+    tensor (any shape, contiguous); out: a uint8 device tensor of as many
+    elements.  Raises CCV3DError on a refused call unless check=False."""
+    import torch
+    dt = {torch.float32: CCV3D_FP32, torch.bfloat16: CCV3D_BF16}.get(x.dtype)
+    if dt is None or out.dtype != torch.uint8 or out.numel() != x.numel():
+        raise ValueError("ccv3d_quantize_u8: x float32/bfloat16, out uint8 of x.numel()")
+    if not (x.is_contiguous() and out.is_contiguous()):
+        raise ValueError("ccv3d_quantize_u8: contiguous tensors only")
+    rc = lib.ccv3d_quantize_u8(_ptr(x), dt, _ptr(out), x.numel(), _stream(stream))
+    if rc != 0 and check:
+        raise CCV3DError(rc, "ccv3d_quantize_u8")
+    return rc
 
 
 def ccv3d_selftest_wait_timeout(limit_ns: int, stream=None) -> int:

@@ -27,6 +27,7 @@
 #include "conv_tc2h.cuh"
 #include "conv_tcp.cuh"
 #include "params.h"
+#include "quantize.cuh"
 
 using namespace ccv3d;
 
@@ -782,6 +783,27 @@ const char* ccv3d_strerror(ccv3d_status s) {
             return "call needs more device scratch than the no-allocation entry point holds";
     }
     return "unknown status";
+}
+
+ccv3d_status ccv3d_quantize_u8(const void* in, ccv3d_dtype dtype, void* out, long long n,
+                               cudaStream_t stream) {
+    if (n < 0 || (dtype != CCV3D_FP32 && dtype != CCV3D_BF16)) return CCV3D_ERR_INVALID;
+    if (n == 0) return CCV3D_OK;
+    if (in == nullptr || out == nullptr) return CCV3D_ERR_INVALID;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(in), b = reinterpret_cast<uintptr_t>(out);
+    if ((a | b) & 15u) return CCV3D_ERR_ALIGNMENT;
+    const uintptr_t a_end = a + (uintptr_t)n * (dtype == CCV3D_FP32 ? 4u : 2u);
+    if (a < b + (uintptr_t)n && b < a_end) return CCV3D_ERR_ALIAS;
+    const long long units = n / 16;  // 16 values per thread step
+    const int blocks = (int)std::min<long long>(std::max<long long>(1, (units + 255) / 256),
+                                                (long long)kSmCount * 8);
+    if (dtype == CCV3D_FP32)
+        quantize_u8_f32_kernel<<<blocks, 256, 0, stream>>>(static_cast<const float*>(in),
+                                                            static_cast<uint8_t*>(out), n);
+    else
+        quantize_u8_bf16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(in),
+                                                             static_cast<uint8_t*>(out), n);
+    return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
 }
 
 ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {

@@ -184,6 +184,21 @@ CCV3D_API ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t plan, size_t* out_bytes,
  * (a defect), or CCV3D_ERR_CUDA. */
 CCV3D_API ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
 
+/* Post-decode uint8 quantisation of decoded frames, the step after the
+ * decoder (FastVideo pull request "Quantize frames to uint8 on-device before
+ * the post-decode D->H copy", Summary and Correctness):
+ *   out[i] = trunc(clamp(fp32(in[i]) * 255, 0, 255)),  NaN -> 0,
+ * the multiply in fp32 for both input types, the cast truncating toward zero
+ * (PyTorch's float -> uint8).  Elementwise over n values in any layout; the
+ * caller copies `out` to the host (n bytes instead of 4n or 2n).
+ *   in     n values of `dtype` (CCV3D_FP32 or CCV3D_BF16), device memory
+ *   out    n bytes, device memory; must not overlap `in`
+ * Both pointers 16-byte aligned.  Asynchronous on `stream`; no allocation.
+ * Errors: INVALID (n < 0, unknown dtype, NULL pointer with n > 0), ALIGNMENT,
+ * ALIAS (the buffers overlap), CUDA (launch failure).  n == 0 does nothing. */
+CCV3D_API ccv3d_status ccv3d_quantize_u8(const void* in, ccv3d_dtype dtype, void* out,
+                                         long long n, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Forward call that allocates nothing.
  *

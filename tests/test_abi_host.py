@@ -202,3 +202,16 @@ def test_plan_tiling_reports():
     simt = ccv3d.Plan(ccv3d.desc_for(workloads.C1))
     assert simt.tiling == {"k_block": 0, "stages": 0, "workspace_pairs": 0}
     assert ccv3d.lib.ccv3d_plan_tiling(None, None, None, None) == ccv3d.CCV3D_ERR_INVALID
+
+
+def test_quantize_validation_without_gpu():
+    """Argument checks of ccv3d_quantize_u8 run before any device work."""
+    lib = ccv3d.lib
+    A = 1 << 20
+    assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_FP32, 2 * A, -1, None) == ccv3d.CCV3D_ERR_INVALID
+    assert lib.ccv3d_quantize_u8(A, 9, 2 * A, 16, None) == ccv3d.CCV3D_ERR_INVALID
+    assert lib.ccv3d_quantize_u8(None, ccv3d.CCV3D_FP32, 2 * A, 16, None) == ccv3d.CCV3D_ERR_INVALID
+    assert lib.ccv3d_quantize_u8(A + 4, ccv3d.CCV3D_FP32, 2 * A, 16, None) == ccv3d.CCV3D_ERR_ALIGNMENT
+    assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_FP32, A + 48, 16, None) == ccv3d.CCV3D_ERR_ALIAS
+    assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_BF16, A + 16, 16, None) == ccv3d.CCV3D_ERR_ALIAS
+    assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_FP32, 2 * A, 0, None) == ccv3d.CCV3D_OK
