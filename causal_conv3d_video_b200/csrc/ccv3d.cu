@@ -24,6 +24,7 @@
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
 #include "conv_tc2.cuh"
+#include "conv_tc2f.cuh"
 #include "conv_tc2h.cuh"
 #include "conv_tcp.cuh"
 #include "params.h"
@@ -42,6 +43,7 @@ struct ccv3d_plan_s {
     int persist;  // 1: persistent stream-K pair kernel
     int halo;     // 1: pair kernel loading each input row strip once per (tap, channel block)
     int halo_w;   // halo: pixels per strip
+    int fused;    // 1: halo pair kernel computing two output frames per tile
     int G, n_acc;  // persistent: CTA pairs launched, TMEM accumulator buffers
     long long frame_start[kMaxFrames + 1], sk_total;
     size_t smem_bytes;
@@ -130,6 +132,14 @@ size_t smem_for(int kind, int bn, int stages) {
                      : (kind == 1 ? tc2_smem_bytes<BK>(bn, stages) : tc_smem_bytes<BK>(bn, stages));
 }
 
+size_t fused_smem_for(int bk, int bn, int stages, int kh, int kw, int halo_w) {
+    switch (bk) {
+        case 64: return tc2f_smem_bytes<64>(bn, stages, kh, kw, halo_w);
+        case 32: return tc2f_smem_bytes<32>(bn, stages, kh, kw, halo_w);
+        default: return tc2f_smem_bytes<16>(bn, stages, kh, kw, halo_w);
+    }
+}
+
 size_t halo_smem_for(int bk, int bn, int stages, int kh, int kw, int halo_w) {
     switch (bk) {
         case 64: return tc2h_smem_bytes<64>(bn, stages, kh, kw, halo_w);
@@ -163,6 +173,8 @@ void set_smem_attrs() {
         cudaFuncSetAttribute(conv_tcp_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaFuncSetAttribute(conv_tc2h_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
+        cudaFuncSetAttribute(conv_tc2f_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaGetLastError();
     });
@@ -225,6 +237,7 @@ bool setup_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->sk_total = acc;
     p->BK = bk;
     p->halo = 0;
+    p->fused = 0;
     p->persist = 1;
     return true;
 }
@@ -276,6 +289,36 @@ void setup_halo(const ccv3d_desc& d, ccv3d_plan_s* p) {
         p->BK = bk;
         p->stages = s;
         p->smem_bytes = halo_smem_for(bk, p->BN, s, d.kh, d.kw, halo_w);
+        return;
+    }
+}
+
+// Two output frames per tile on the halo kernel (conv_tc2f.cuh): with unit
+// temporal stride and dilation, frames o and o+1 share their source frames,
+// so one MMA of N = 2 Cout covers both, with 1.5x fewer MMAs and strip loads
+// per output frame for thin Cout (<= 128).  Sized like the halo kernel (two
+// CTAs per SM).  Opt-in (CCV3D_FUSE=1): measured on the 96-channel 720x1280
+// calls it runs at the speed of the halo kernel (2433 vs 2409 us), so those
+// calls are bound by neither the MMA count nor the strip traffic.
+void setup_fused(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    p->fused = 0;
+    if (env_int("CCV3D_FUSE") <= 0) return;
+    if (!p->halo || d.stride_t != 1 || d.dil_t != 1 || p->T_o < 2) return;
+    if (p->tiles_n != 1 || p->n_sub != 1 || 2 * p->BN > 256) return;
+    const size_t budget = kSmemBudget / 2;  // two CTAs per SM
+    const int want_s = env_int("CCV3D_STAGES");
+    for (int bk : {64, 32, 16}) {
+        if (d.Cin % bk != 0) continue;
+        int s = want_s >= 2 ? want_s : 8;
+        const size_t cap = want_s >= 2 ? kSmemBudget : budget;
+        while (s >= 2 && fused_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w) > cap) --s;
+        if (s < 2) continue;
+        p->fused = 1;
+        p->BK = bk;
+        p->stages = s;
+        p->smem_bytes = fused_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w);
+        p->tmem_cols = 32;
+        while (p->tmem_cols < 2 * p->BN) p->tmem_cols *= 2;
         return;
     }
 }
@@ -341,6 +384,7 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->persist = 0;
     size_tc(d, p);
     setup_halo(d, p);
+    setup_fused(d, p);
     const char* ps = std::getenv("CCV3D_PERSIST");
     const bool persist = ps != nullptr ? std::atoi(ps) > 0 : prefer_persistent(d, *p);
     if (persist && setup_persistent(d, p)) size_tc(d, p);
@@ -471,7 +515,9 @@ Taps make_taps(const ccv3d_plan_s* p) {
 template <int BK>
 cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s) {
     set_smem_attrs<BK>();
-    if (kind == 3)
+    if (kind == 4)
+        conv_tc2f_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
+    else if (kind == 3)
         conv_tc2h_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
     else if (kind == 2)
         conv_tcp_kernel<BK><<<grid, kTcpThreads, smem, s>>>(prm);
@@ -513,6 +559,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     long long grid =
         p->pair ? 2LL * d.N * p->T_o * prm.pairs_per_frame * p->tiles_n
                 : (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
+    if (p->fused) grid = 2LL * d.N * ((p->T_o + 1) / 2) * prm.pairs_per_frame;  // frame pairs
     if (p->persist) {
         if (p->scratch == nullptr) return CCV3D_ERR_CUDA;
         grid = 2LL * p->G;
@@ -534,7 +581,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
     const long long units = p->pair ? grid / 2 : grid;
     const long long wave = p->pair ? kSmCount / 2 : kSmCount;
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
-    const int kind = p->halo ? 3 : (p->persist ? 2 : p->pair);
+    const int kind = p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair));
     prm.halo_w = p->halo_w;
     cudaError_t e;
     switch (p->BK) {
@@ -543,6 +590,15 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const voi
         default: e = launch_tc<16>(prm, kind, (int)grid, p->smem_bytes, stream); break;
     }
     return e == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+// SIMT variant: one warp per (pixel, 4-channel group) when one thread per
+// unit would leave the SMs under 128 threads each (the calls are latency
+// bound, so parallelism over the reduction wins); otherwise one thread.
+bool simt_uses_warps(const ccv3d_plan_s& p) {
+    const long long units =
+        (long long)p.d.N * p.T_o * p.H_o * p.W_o * ceil_div(p.d.Cout, kSimtCoT);
+    return units < (long long)kSmCount * kSimtThreads;
 }
 
 ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const void* cache, const void* w,
@@ -562,14 +618,19 @@ ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const void* cache, const v
     prm.cache_len = d.cache_len; prm.T_x = d.T_x;
     prm.co_groups = ceil_div(d.Cout, kSimtCoT);
     prm.conv_threads = (long long)d.N * p->T_o * p->H_o * p->W_o * prm.co_groups;
-    const long long cb = (prm.conv_threads + kSimtThreads - 1) / kSimtThreads;
+    const bool warp = simt_uses_warps(*p);
+    const long long cb = (prm.conv_threads * (warp ? 32 : 1) + kSimtThreads - 1) / kSimtThreads;
     const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
     const long long kb = copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 32767) / 32768) : 0;
     if (cb + kb > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
     prm.conv_blocks = (int)cb;
     prm.copy_blocks = (int)kb;
     const int grid = (int)(cb + kb);
-    if (d.dtype == CCV3D_FP32)
+    if (warp && d.dtype == CCV3D_FP32)
+        conv_simt_warp_kernel<float><<<grid, kSimtThreads, 0, stream>>>(prm);
+    else if (warp)
+        conv_simt_warp_kernel<__nv_bfloat16><<<grid, kSimtThreads, 0, stream>>>(prm);
+    else if (d.dtype == CCV3D_FP32)
         conv_simt_kernel<float><<<grid, kSimtThreads, 0, stream>>>(prm);
     else
         conv_simt_kernel<__nv_bfloat16><<<grid, kSimtThreads, 0, stream>>>(prm);
@@ -691,7 +752,8 @@ int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
 
 const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
     if (p == nullptr) return "";
-    if (!p->path_tc) return "simt";
+    if (!p->path_tc) return simt_uses_warps(*p) ? "simt_warp" : "simt";
+    if (p->fused) return "tc_pair_fused";
     if (p->halo) return "tc_pair_halo";
     if (p->persist) return "tc_persistent";
     return p->pair ? "tc_pair" : "tc_single";

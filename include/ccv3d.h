@@ -134,7 +134,9 @@ CCV3D_API ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t plan, int* T_o, int* H_
 CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
 
 /* Name of the kernel the plan launches: "tc_pair_halo", "tc_pair",
- * "tc_single", "tc_persistent" or "simt" (static string; "" for NULL). */
+ * "tc_single", "tc_persistent", "simt" (one thread per pixel and 4 output
+ * channels) or "simt_warp" (one warp per pixel and 4 output channels, for
+ * calls too small to fill the SMs otherwise) (static string; "" for NULL). */
 CCV3D_API const char* ccv3d_plan_kernel(ccv3d_plan_t plan);
 
 /* Reduction tiling of a tensor-core plan (inspection; no counterpart in the

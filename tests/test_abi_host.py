@@ -195,7 +195,7 @@ def test_kernel_choice(conv, kernel, monkeypatch):
 
 
 def test_plan_tiling_reports():
-    halo = ccv3d.Plan(ccv3d.desc_for(workloads.C3))
+    halo = ccv3d.Plan(ccv3d.desc_for(workloads.C3.replace(T_x=1)))
     assert halo.kernel == "tc_pair_halo"
     assert halo.tiling["k_block"] in (16, 32) and halo.tiling["stages"] >= 2
     assert halo.tiling["workspace_pairs"] == 0
@@ -215,3 +215,11 @@ def test_quantize_validation_without_gpu():
     assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_FP32, A + 48, 16, None) == ccv3d.CCV3D_ERR_ALIAS
     assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_BF16, A + 16, 16, None) == ccv3d.CCV3D_ERR_ALIAS
     assert lib.ccv3d_quantize_u8(A, ccv3d.CCV3D_FP32, 2 * A, 0, None) == ccv3d.CCV3D_OK
+
+
+def test_simt_variant_choice():
+    """Calls too small for one thread per (pixel, 4 channels) to fill the SMs
+    run one warp per unit (the lanes split the reduction)."""
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
+    big = workloads.Conv("f32_big", 32, 32, 64, 64, T_x=4, cache_len=2, dtype="fp32")
+    assert ccv3d.Plan(ccv3d.desc_for(big)).kernel == "simt"

@@ -75,6 +75,7 @@ def _run_small(c, force_simt=False, env=None):
 def test_config1_fp32_exact_workload():
     call, m = _run_small(workloads.C1)
     assert call.plan.path["tc"] is False
+    assert call.plan.kernel == "simt_warp"
     assert call.plan.stats()["simt_path"] == 1
 
 
@@ -129,8 +130,50 @@ HALO = [
 @pytest.mark.parametrize("halo", [1, 0], ids=["halo", "no_halo"])
 @pytest.mark.parametrize("c", HALO, ids=lambda c: c.name)
 def test_small_halo_strips(c, halo):
-    call, _ = _run_small(c, env={"CCV3D_HALO": halo, "CCV3D_PERSIST": 0})
+    call, _ = _run_small(c, env={"CCV3D_HALO": halo, "CCV3D_PERSIST": 0, "CCV3D_FUSE": 0})
     assert (call.plan.kernel == "tc_pair_halo") == bool(halo), call.plan.kernel
+
+
+FUSED = [
+    # two output frames per tile, sharing source frames (unit temporal stride)
+    Conv("f96_t4_c2", 96, 96, 3, 256, T_x=4, cache_len=2, sigma_b=0.1),
+    Conv("f64_t3_c0", 64, 64, 4, 256, T_x=3, cache_len=0),            # odd T_o, warm-up taps
+    Conv("f32to48_t5_c1", 32, 48, 3, 200, T_x=5, cache_len=1),        # ragged row, odd T_o
+    Conv("f64_biasonly", 64, 64, 2, 256, T_x=3, cache_len=0, pad_t_base=4, cache_keep=2),
+    Conv("f64_crop", 64, 64, 2, 256, T_x=2, cache_len=3),              # |C| > p_l^base
+    Conv("f128_k311", 128, 128, 2, 256, T_x=4, cache_len=2, kh=1, kw=1, pad=(0, 0)),
+    Conv("f64_n2", 64, 64, 2, 256, T_x=2, cache_len=2, N=2),
+    Conv("f96_dilw2", 96, 96, 2, 256, T_x=2, cache_len=2, pad=(2, 2), dilation=(1, 2, 2)),
+    Conv("f128_s2h", 128, 128, 9, 256, T_x=2, cache_len=1, stride=(2, 1)),
+    Conv("f192to96_t4", 192, 96, 2, 384, T_x=4, cache_len=2, sigma_b=0.1),
+]
+
+
+@pytest.mark.parametrize("c", FUSED, ids=lambda c: c.name)
+def test_small_fused_frame_pairs(c):
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1})
+    assert call.plan.kernel == "tc_pair_fused", call.plan.kernel
+
+
+@pytest.mark.parametrize("c", FUSED[:3], ids=lambda c: c.name)
+def test_small_fused_off_is_halo(c):
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0})
+    assert call.plan.kernel == "tc_pair_halo", call.plan.kernel
+
+
+def test_full_size_fused_sampled():
+    """The 96-channel 720x1280 four-frame call on the frame-pair kernel."""
+    c = workloads.C3
+    inp = inputs_for(c)
+    call = GpuCall(c, inp, env={"CCV3D_FUSE": 1}).run()
+    torch.cuda.synchronize()
+    assert call.plan.kernel == "tc_pair_fused"
+    idx = sample_indices(tuple(call.out.shape), call.plan, n_random=2000)
+    ref = oracle.points(oracle_params(c), inp["x"], inp["cache"], inp["w"], inp["bias"], idx)
+    got = call.out[tuple(torch.from_numpy(idx.T).cuda())].double().cpu().numpy()
+    assert_close(got, ref, c.dtype, c.name)
+    assert np.array_equal(call.nc_f64(), expected_new_cache(c, inp))
+    assert call.guards_intact() and call.plan.status() == ccv3d.CCV3D_OK
 
 
 SMALL_ST = [
@@ -172,10 +215,15 @@ def test_small_temporal_stride_simt(c):
     assert call.plan.path["tc"] is False
 
 
-@pytest.mark.parametrize("c", SMALL[:4] + SMALL[12:15] + SMALL[19:21], ids=lambda c: c.name)
+@pytest.mark.parametrize("c", SMALL[:4] + SMALL[8:9] + SMALL[12:15] + SMALL[19:21],
+                         ids=lambda c: c.name)
 def test_small_simt_bf16(c):
     call, _ = _run_small(c, force_simt=True)
     assert call.plan.path["tc"] is False
+    # one warp per (pixel, 4 channels) below 148 x 128 such units, else one thread
+    iv = call.plan.intervals
+    units = c.N * iv["T_o"] * iv["H_o"] * iv["W_o"] * -(-c.Cout // 4)
+    assert call.plan.kernel == ("simt_warp" if units < 148 * 128 else "simt")
 
 
 @pytest.mark.parametrize("c", [
