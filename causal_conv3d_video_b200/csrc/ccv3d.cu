@@ -296,23 +296,26 @@ void setup_halo(const ccv3d_desc& d, ccv3d_plan_s* p) {
 // Two output frames per tile on the halo kernel (conv_tc2f.cuh): with unit
 // temporal stride and dilation, frames o and o+1 share their source frames,
 // so one MMA of N = 2 Cout covers both, with 1.5x fewer MMAs and strip loads
-// per output frame for thin Cout (<= 128).  Sized like the halo kernel (two
-// CTAs per SM).  Opt-in (CCV3D_FUSE=1): measured on the 96-channel 720x1280
-// calls it runs at the speed of the halo kernel (2433 vs 2409 us), so those
-// calls are bound by neither the MMA count nor the strip traffic.
+// per output frame for thin Cout (<= 128).  Stages of one kernel row keep 4
+// in flight per CTA at two CTAs per SM.  Measured on the 720x1280 four-frame
+// calls: 2068 vs 2405 us (96 channels) and 3631 vs 4315 us (192 -> 96)
+// against the halo kernel.  CCV3D_FUSE=0 disables it.
 void setup_fused(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->fused = 0;
-    if (env_int("CCV3D_FUSE") <= 0) return;
+    const char* fe = std::getenv("CCV3D_FUSE");
+    if (fe != nullptr && std::atoi(fe) == 0) return;
     if (!p->halo || d.stride_t != 1 || d.dil_t != 1 || p->T_o < 2) return;
     if (p->tiles_n != 1 || p->n_sub != 1 || 2 * p->BN > 256) return;
     const size_t budget = kSmemBudget / 2;  // two CTAs per SM
     const int want_s = env_int("CCV3D_STAGES");
+    // the widest channel block that keeps 4 stages per CTA, else 2
+    for (int min_s : {4, 2})
     for (int bk : {64, 32, 16}) {
         if (d.Cin % bk != 0) continue;
         int s = want_s >= 2 ? want_s : 8;
         const size_t cap = want_s >= 2 ? kSmemBudget : budget;
         while (s >= 2 && fused_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w) > cap) --s;
-        if (s < 2) continue;
+        if (s < (want_s >= 2 ? 2 : min_s)) continue;
         p->fused = 1;
         p->BK = bk;
         p->stages = s;

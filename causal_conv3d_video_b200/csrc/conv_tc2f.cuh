@@ -4,15 +4,17 @@
 // With unit temporal stride and dilation, output frames o and o+1 read the
 // same source frame t through adjacent temporal taps: k = t - o + p_l for
 // frame o and k - 1 for frame o+1 (Sec. 4's per-tap decomposition, regrouped
-// by source frame).  So one pipeline stage per (source frame t, channel block)
-// holds the kh input strips of frame t and, per spatial tap (r, s), the weight
-// rows of both temporal taps stacked along N:
+// by source frame).  A pipeline stage is (source frame t, channel block,
+// kernel row r): the input strip of row r of frame t and, per kernel column
+// s, the weight rows of both temporal taps stacked along N:
 //     N rows [0, BN)      tap k   (frame o,   TMEM columns [0, BN))
 //     N rows [BN, 2 BN)   tap k-1 (frame o+1, TMEM columns [BN, 2 BN))
 // and one MMA of N = 2 BN accumulates both frames.  In the CTA pair the N rows
 // split by halves, so the even CTA holds tap k's rows and the odd CTA tap
 // k-1's.  A source frame that only one of the two frames reads is a stage of
 // N = BN aimed at that frame's columns (each CTA holding half its rows).
+// Stages this small fit four per CTA at two CTAs per SM, so the loads of the
+// next stages stay in flight while an MMA group runs.
 //
 // Thin channel counts (BN <= 128) are where this pays: a tcgen05 MMA has a
 // floor of about 125 cycles whatever its N, so N = 96 instructions run at
@@ -24,8 +26,8 @@
 // zeroes each region), then the shared stages; otherwise the first stage
 // (shared, or the only kind) zeroes what it writes.
 //
-// Halo strips, pair barriers, epilogue and bounded waits are those of
-// conv_tc2h.cuh.
+// Halo strips (one per stage here), pair barriers, epilogue and bounded waits
+// are those of conv_tc2h.cuh.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -39,12 +41,11 @@
 
 namespace ccv3d {
 
-// One stage (per CTA): kh strips + kh*kw weight areas of bn rows (two taps'
-// halves, or one tap's half in the first bn/2 rows).
+// One stage (per CTA): one strip + kw weight areas of bn rows (two taps'
+// rows, or one tap's half in the first bn/2 rows).
 template <int BK>
 __host__ __device__ constexpr size_t tc2f_stage_bytes(int bn, int kh, int kw, int halo_w) {
-    return (size_t)kh * halo_strip_bytes<BK>(halo_w) +
-           (size_t)kh * kw * bn * TcSmem<BK>::kRowBytes;
+    return (void)kh, halo_strip_bytes<BK>(halo_w) + (size_t)kw * bn * TcSmem<BK>::kRowBytes;
 }
 
 template <int BK>
@@ -127,8 +128,8 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
     const int kWt = BN * kRow;        // weight area per (r, s), per CTA
     const int halo_w = p.halo_w;
     const int kStrip = (int)halo_strip_bytes<BK>(halo_w);
-    const int kAst = p.kh * kStrip;
-    const int kStage = kAst + p.kh * p.kw * kWt;
+    const int kAst = kStrip;                 // the stage's strip
+    const int kStage = kAst + p.kw * kWt;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(
         smem + ring_bytes((size_t)stages * kStage, BN));
     uint64_t* empty_bar = full_bar + stages;
@@ -155,7 +156,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
         ty = box / p.tiles_x;
     }
     const FusedSrc src = fused_sources(p, o0);
-    const int iters = src.n * p.n_cb;  // stages of this tile: (source frame, channel block)
+    const int iters = src.n * p.n_cb * p.kh;  // stages: (source frame, channel block, row r)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -188,11 +189,11 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
     if (warp == 0) {
         if (lane == 0 && iters > 0) {
             // ------------------------------- TMA producer (both CTAs)
-            const uint32_t strip_bytes = 2u * (uint32_t)(p.kh * halo_w * kRow);
+            const uint32_t strip_bytes = 2u * (uint32_t)(halo_w * kRow);
             const int xs = tx * p.box_w - p.p_w;  // first pixel of the strip (s_w = 1)
             const int y_out = ty * p.box_h;
             Ring ring;
-            int si = 0, cb = 0;
+            int si = 0, cb = 0, r = 0;
             for (int it = 0; it < iters; ++it) {
                 if (it >= stages && !mbar_wait(smem_u32(&empty_bar[ring.st]), ring.ph ^ 1u,
                                                p.status, p.wait_limit_ns))
@@ -203,7 +204,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 // this CTA's rows: both -> all BN rows of its tap (even CTA tap ka, odd
                 // CTA tap kb); one frame -> its half (hB rows) of the single tap
                 const int my_tap = both ? (leader ? ka : kb) : (ka >= 0 ? ka : kb);
-                const int wbytes_cta = p.kh * p.kw * (both ? BN : hB) * kRow;
+                const int wbytes_cta = p.kw * (both ? BN : hB) * kRow;
                 uint8_t* st_base = smem + (size_t)ring.st * kStage;
                 const uint32_t fb_local = smem_u32(&full_bar[ring.st]);
                 if (leader) mbar_arrive_expect_tx(fb_local, strip_bytes + 2u * (uint32_t)wbytes_cta);
@@ -211,26 +212,28 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 const CUtensorMap* map = t < p.cache_len ? &p.tmap_c : &p.tmap_x;
                 const int frame = t < p.cache_len ? n * p.cache_len + t
                                                   : n * p.T_x + (t - p.cache_len);
-                for (int r = 0; r < p.kh; ++r)
-                    tma_load_4d_pair(smem_u32(st_base + r * kStrip), map, fb, cb * BK, xs,
-                                     y_out * p.s_h + r * p.d_h - p.p_h, frame);
+                tma_load_4d_pair(smem_u32(st_base), map, fb, cb * BK, xs,
+                                 y_out * p.s_h + r * p.d_h - p.p_h, frame);
                 uint8_t* b_base = st_base + kAst;
-                const int wtap = my_tap * p.kh * p.kw;
-                for (int rs = 0; rs < p.kh * p.kw; ++rs) {
+                const int wrow = my_tap * p.kh * p.kw + r * p.kw;
+                for (int sx = 0; sx < p.kw; ++sx) {
                     if (both) {
-                        tma_load_3d_pair(smem_u32(b_base + rs * kWt), &p.tmap_w, fb, cb * BK,
-                                         wtap + rs, 0);
-                        tma_load_3d_pair(smem_u32(b_base + rs * kWt + hB * kRow), &p.tmap_w, fb,
-                                         cb * BK, wtap + rs, hB);
+                        tma_load_3d_pair(smem_u32(b_base + sx * kWt), &p.tmap_w, fb, cb * BK,
+                                         wrow + sx, 0);
+                        tma_load_3d_pair(smem_u32(b_base + sx * kWt + hB * kRow), &p.tmap_w, fb,
+                                         cb * BK, wrow + sx, hB);
                     } else {
-                        tma_load_3d_pair(smem_u32(b_base + rs * kWt), &p.tmap_w, fb, cb * BK,
-                                         wtap + rs, (int)rank * hB);
+                        tma_load_3d_pair(smem_u32(b_base + sx * kWt), &p.tmap_w, fb, cb * BK,
+                                         wrow + sx, (int)rank * hB);
                     }
                 }
                 ring.next(stages);
-                if (++cb == p.n_cb) {
-                    cb = 0;
-                    ++si;
+                if (++r == p.kh) {
+                    r = 0;
+                    if (++cb == p.n_cb) {
+                        cb = 0;
+                        ++si;
+                    }
                 }
             }
         }
@@ -241,7 +244,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
             const uint32_t idesc_two = idesc_bf16_m256((uint32_t)(2 * BN));
             const uint64_t d0 = smem_desc_kmajor(smem_u32(smem), kRow);
             Ring ring;
-            int si = 0, cb = 0;
+            int si = 0, cb = 0, r = 0;
             for (int it = 0; it < iters; ++it) {
                 if (!mbar_wait(smem_u32(&full_bar[ring.st]), ring.ph, p.status, p.wait_limit_ns))
                     break;
@@ -249,25 +252,26 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 const bool both = src.k0[si] >= 0 && src.k1[si] >= 0;
                 const uint32_t idesc = both ? idesc_two : idesc_one;
                 const uint32_t d_tmem = tmem_base + (src.k0[si] >= 0 ? 0u : (uint32_t)BN);
-                const bool zero = src.zero[si] && cb == 0;
+                const bool zero = src.zero[si] && cb == 0 && r == 0;
                 const uint32_t st_off = (uint32_t)ring.st * (uint32_t)kStage;
-                for (int r = 0; r < p.kh; ++r)
-                    for (int s = 0; s < p.kw; ++s) {
-                        const uint64_t a_desc =
-                            d0 + (uint64_t)((st_off + r * kStrip + s * p.d_w * kRow) >> 4);
-                        const uint64_t b_desc =
-                            d0 + (uint64_t)((st_off + kAst + (r * p.kw + s) * kWt) >> 4);
-                        const bool first = zero && r == 0 && s == 0;
+                for (int sx = 0; sx < p.kw; ++sx) {
+                    // A: the strip shifted by sx*d_w pixels (rows)
+                    const uint64_t a_desc = d0 + (uint64_t)((st_off + sx * p.d_w * kRow) >> 4);
+                    const uint64_t b_desc = d0 + (uint64_t)((st_off + kAst + sx * kWt) >> 4);
+                    const bool first = zero && sx == 0;
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            umma_bf16_pair(d_tmem, a_desc + 2u * kk, b_desc + 2u * kk, idesc,
-                                           (first && kk == 0) ? 0u : 1u);
-                    }
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, a_desc + 2u * kk, b_desc + 2u * kk, idesc,
+                                       (first && kk == 0) ? 0u : 1u);
+                }
                 umma_commit_pair(smem_u32(&empty_bar[ring.st]), (uint16_t)0x3);
                 ring.next(stages);
-                if (++cb == p.n_cb) {
-                    cb = 0;
-                    ++si;
+                if (++r == p.kh) {
+                    r = 0;
+                    if (++cb == p.n_cb) {
+                        cb = 0;
+                        ++si;
+                    }
                 }
             }
             umma_commit_pair(smem_u32(acc_bar), (uint16_t)0x3);

@@ -169,7 +169,7 @@ def test_tile_choice_on_bottleneck():
 
 @pytest.mark.parametrize("conv,kernel", [
     (workloads.C2, "tc_pair"),                      # 0.8 wave of pair tiles
-    (workloads.C3, "tc_pair_halo"),                 # thin 720x1280: halo strips
+    (workloads.C3, "tc_pair_fused"),                # thin 720x1280, 4 frames: frame pairs
     (workloads.C4_TIME, "tc_persistent"),           # 6.1 waves, ragged last wave
     (workloads.C4_STRIDE, "tc_persistent"),         # 3.04 waves
     (workloads.C4_DIL, "tc_persistent"),

@@ -157,7 +157,7 @@ def test_small_fused_frame_pairs(c):
 
 @pytest.mark.parametrize("c", FUSED[:3], ids=lambda c: c.name)
 def test_small_fused_off_is_halo(c):
-    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0})
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 0})
     assert call.plan.kernel == "tc_pair_halo", call.plan.kernel
 
 
