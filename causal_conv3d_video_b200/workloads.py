@@ -177,3 +177,18 @@ def decode17_schedule(scale_hw: tuple | None = None):
 def signature(c: Conv):
     return (c.Cin, c.Cout, c.kt, c.kh, c.kw, c.H, c.W, c.T_x, c.cache_len,
             c.stride, c.pad, c.dilation, c.dtype, c.stride_t)
+
+
+def decode17_records(scale_hw: tuple | None = None):
+    """The 164-call schedule as plain records (the content of
+    configs/decode17.json): one dict per call, in call order."""
+    out = []
+    for c in decode17_schedule(scale_hw):
+        v = c.conv
+        out.append({"call": len(out), "module": c.module, "group": c.group, "chunk": c.chunk,
+                    "Cin": v.Cin, "Cout": v.Cout, "kernel": [v.kt, v.kh, v.kw], "H": v.H,
+                    "W": v.W, "T_x": v.T_x, "cache_len": v.cache_len,
+                    "pad_t_base": v.pad_t_base, "cache_keep": v.cache_keep,
+                    "stride": list(v.stride), "pad": list(v.pad),
+                    "dilation": list(v.dilation), "dtype": v.dtype})
+    return out

@@ -2,6 +2,7 @@
 import collections
 
 import numpy as np
+import pytest
 
 from causal_conv3d_video_b200 import synth, workloads
 
@@ -52,3 +53,52 @@ def test_bf16_rounding_is_rne():
     ref = torch.from_numpy(a).to(torch.bfloat16).float().numpy()
     assert np.array_equal(synth.round_to_bf16(a), ref)
     assert np.array_equal(synth.normal((1 << 16,), 3.0, 4, 1, bf16=True), ref)
+
+
+def test_decode17_json_matches_schedule():
+    """configs/decode17.json is the committed form of decode17_schedule()."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "configs", "decode17.json")
+    doc = json.load(open(path))
+    assert doc["calls"] == workloads.decode17_records()
+    assert len(doc["calls"]) == 164
+    sigs = {json.dumps({k: v for k, v in r.items() if k not in ("call", "module", "group",
+                                                                 "chunk")}, sort_keys=True)
+            for r in doc["calls"]}
+    assert len(sigs) == 28
+
+
+# per-call effective GFLOP and algorithmic MB of the decoder workloads, as the
+# measurement plan tabulates them from the formulas (active taps only; Z and W
+# read once, out and new_cache written once)
+_TABLE = {"bf16_384ch_90x160_c2_t1": (114.7, 74.3), "bf16_384ch_90x160_c0_t1": (38.2, 41.1),
+          "bf16_96ch_720x1280_c2_t4": (1834.6, 2124), "bf16_192to96_720x1280_c2_t4": (3669.2, 3540),
+          "bf16_3x1x1_384to768_180x320_c2_t1": (101.9, 311),
+          "bf16_192ch_dt2_180x320_c4_t1": (114.7, 223), "bf16_192ch_s2_360x640_c2_t1": (114.7, 466),
+          "bf16_384ch_90x160_c1_t1": (76.4, 63.3), "bf16_192ch_89x157_c2_t1": (27.8, 34.2)}
+
+
+@pytest.mark.parametrize("name", sorted(_TABLE))
+def test_bench_algorithmic_flops_and_bytes(name):
+    """bench.algorithmic() against the tabulated figures, and its FLOP count
+    against a brute-force count of the (output frame, tap) pairs whose source
+    frame lies in Z (the oracle's scan)."""
+    import bench
+    import oracle
+    c = workloads.WORKLOADS[name]
+    op = oracle.params(c.N, c.Cin, c.Cout, c.H, c.W, c.T_x, c.cache_len, kt=c.kt, kh=c.kh,
+                       kw=c.kw, pad_t_base=c.pad_t_base, cache_keep=c.cache_keep,
+                       stride=c.stride, pad=c.pad, dilation=c.dilation, stride_t=c.stride_t)
+    T_o, H_o, W_o, _ = oracle.shape(op)
+    _, delta, o_l, o_h, _ = oracle.tap_scan(op)
+    iv = {"T_o": T_o, "H_o": H_o, "W_o": W_o, "o_l": o_l, "o_h": o_h}
+    flops, nbytes = bench.algorithmic(c, iv)
+    z = c.cache_len + c.T_x
+    pairs = sum(1 for o in range(T_o) for k in range(c.kt)
+                if 0 <= o * c.stride_t + k * c.dilation[0] - (c.pad_t_base - c.cache_len) < z)
+    assert flops == 2.0 * c.N * c.Cout * H_o * W_o * c.Cin * c.kh * c.kw * pairs
+    gf, mb = _TABLE[name]
+    assert abs(flops / 1e9 - gf) <= 0.051 * max(1.0, gf / 100), (flops / 1e9, gf)
+    assert abs(nbytes / 1e6 - mb) <= 0.6 + 0.001 * mb, (nbytes / 1e6, mb)
