@@ -133,10 +133,14 @@ CCV3D_API ccv3d_status ccv3d_plan_intervals(ccv3d_plan_t plan, int* T_o, int* H_
  * when a CTA pair shares each MMA (cta_group::2), else 128 (may be NULL). */
 CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
 
-/* Name of the kernel the plan launches: "tc_pair_halo", "tc_pair",
- * "tc_single", "tc_persistent", "simt" (one thread per pixel and 4 output
- * channels) or "simt_warp" (one warp per pixel and 4 output channels, for
- * calls too small to fill the SMs otherwise) (static string; "" for NULL). */
+/* Name of the kernel the plan launches (static string; "" for NULL):
+ *   "tc_pair"        CTA-pair implicit GEMM (cta_group::2)
+ *   "tc_pair_halo"   CTA pair, one input row strip per (tap, channel block)
+ *   "tc_pair_fused"  CTA pair with row strips, two output frames per tile
+ *   "tc_persistent"  persistent stream-K over all SM pairs
+ *   "tc_single"      one CTA per tile
+ *   "simt"           FFMA, one thread per pixel and 4 output channels
+ *   "simt_warp"      FFMA, one warp per pixel and 4 output channels (small calls) */
 CCV3D_API const char* ccv3d_plan_kernel(ccv3d_plan_t plan);
 
 /* Reduction tiling of a tensor-core plan (inspection; no counterpart in the
