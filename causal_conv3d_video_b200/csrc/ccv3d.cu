@@ -99,11 +99,19 @@ ccv3d_status compute_intervals(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->p_l = d.pad_t_base - d.cache_len;
     // output o's tap k reads frame o*s_t + delta_k of Z; no right pad
     const long long tn = (long long)p->z_len + p->p_l - (long long)d.dil_t * (d.kt - 1) - 1;
-    p->T_o = tn < 0 ? 0 : (int)(tn / s_t + 1);
     const long long hn = (long long)d.H + 2LL * d.pad_h - (long long)d.dil_h * (d.kh - 1) - 1;
     const long long wn = (long long)d.W + 2LL * d.pad_w - (long long)d.dil_w * (d.kw - 1) - 1;
-    p->H_o = hn < 0 ? 0 : (int)(hn / d.stride_h + 1);
-    p->W_o = wn < 0 ? 0 : (int)(wn / d.stride_w + 1);
+    const long long T_o = tn < 0 ? 0 : tn / s_t + 1;
+    const long long H_o = hn < 0 ? 0 : hn / d.stride_h + 1;
+    const long long W_o = wn < 0 ? 0 : wn / d.stride_w + 1;
+    // extents the kernels index with 32-bit integers (tiles, frames, pixels of a frame)
+    constexpr long long kMax = 0x7fffffffLL;
+    if ((long long)p->z_len > kMax || T_o > kMax || H_o * W_o > kMax ||
+        (long long)d.H * d.W > kMax || (long long)d.N * (T_o > p->z_len ? T_o : p->z_len) > kMax)
+        return CCV3D_ERR_UNSUPPORTED;
+    p->T_o = (int)T_o;
+    p->H_o = (int)H_o;
+    p->W_o = (int)W_o;
     p->keep = std::min(d.cache_keep, p->z_len);
     for (int k = 0; k < kMaxTaps; ++k) {
         p->delta[k] = p->o_l[k] = p->o_h[k] = 0;

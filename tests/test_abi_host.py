@@ -223,3 +223,16 @@ def test_simt_variant_choice():
     assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
     big = workloads.Conv("f32_big", 32, 32, 64, 64, T_x=4, cache_len=2, dtype="fp32")
     assert ccv3d.Plan(ccv3d.desc_for(big)).kernel == "simt"
+
+
+@pytest.mark.parametrize("kw", [
+    dict(H=1 << 30, pad=(1 << 30, 1)),            # H_o past 2^31
+    dict(H=1 << 16, W=1 << 16),                   # one frame of 2^32 pixels
+    dict(N=1 << 20, T_x=1 << 12),                 # N * frames past 2^31
+])
+def test_plan_refuses_extents_past_32_bit_indexing(kw):
+    base = dict(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2)
+    base.update(kw)
+    with pytest.raises(ccv3d.CCV3DError) as e:
+        ccv3d.Plan(ccv3d.make_desc(**base))
+    assert e.value.status == ccv3d.CCV3D_ERR_UNSUPPORTED
