@@ -431,16 +431,27 @@ def run_gpu(args, rank, world, local_rank):
                     "accumulation buffer",
         },
     }
+    # side measurements: a failure here is reported in the line, never raised
     if world == 1:
-        line["quantize_u8"] = run_quantize(dev)
+        line["quantize_u8"] = _guarded(run_quantize, dev)
     if args.sequence:
-        line["decode17"] = run_sequence(args, dev)
+        line["decode17"] = _guarded(run_sequence, args, dev)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(conv, args.cpu_seconds)
     return line
 
 
 # ------------------------------------------------- decode-sequence leg
+def _guarded(fn, *a):
+    """fn(*a), or {"error": ...} if it raised (the headline line still prints)."""
+    try:
+        return fn(*a)
+    except Exception as e:  # noqa: BLE001 -- recorded, not swallowed silently
+        import traceback
+        traceback.print_exc()
+        return {"error": f"{type(e).__name__}: {e}"}
+
+
 def run_quantize(dev, steps=200):
     """The post-decode step: uint8 frames from a decoded 17-frame 720x1280
     RGB fp32 video (47 M values, 235 MB moved per call), timed with CUDA
