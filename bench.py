@@ -625,7 +625,8 @@ class OracleSampler:
         self.op = oracle.params(conv.N, conv.Cin, conv.Cout, conv.H, conv.W, conv.T_x,
                                 conv.cache_len, kt=conv.kt, kh=conv.kh, kw=conv.kw,
                                 pad_t_base=conv.pad_t_base, cache_keep=conv.cache_keep,
-                                stride=conv.stride, pad=conv.pad, dilation=conv.dilation)
+                                stride=conv.stride, pad=conv.pad, dilation=conv.dilation,
+                                stride_t=conv.stride_t)
         inp = synth.conv_inputs(**conv.synth_kwargs())
         f64 = lambda a: None if a is None else a.astype(np.float64)
         self.x, self.cache, self.w, self.b = (f64(inp["x"]), f64(inp["cache"]),
@@ -668,7 +669,27 @@ def cpu_baseline(conv, seconds):
     n = int(max(256, min(smp.n_out, smp.points_per_s() * seconds)))
     dt = smp.run(n)
     return {"value": round(smp.tflops(n, dt), 6), "unit": "TFLOP/s", "cores": smp.cores,
-            "kind": "oracle", "sample": smp.describe(n, dt)}
+            "kind": "oracle", "sample": smp.describe(n, dt),
+            "single_thread": _single_thread_baseline(conv, min(4.0, seconds / 3))}
+
+
+def _single_thread_baseline(conv, seconds):
+    """The same oracle on one host core (OpenMP pinned to one thread in a
+    child process, since the thread count is fixed when the library loads)."""
+    code = ("import json, sys; sys.path.insert(0, sys.argv[1]); import bench; "
+            "from causal_conv3d_video_b200 import workloads; "
+            "smp = bench.OracleSampler(workloads.WORKLOADS[sys.argv[2]]); "
+            "n = int(max(64, min(smp.n_out, smp.points_per_s() * float(sys.argv[3])))); "
+            "dt = smp.run(n); "
+            "print(json.dumps({'value': round(smp.tflops(n, dt), 6), 'unit': 'TFLOP/s', "
+            "'cores': smp.cores, 'sample': smp.describe(n, dt)}))")
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", code, ROOT, conv.name, str(seconds)], env=env,
+                           capture_output=True, text=True, timeout=120 + 4 * seconds)
+        return json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception as e:  # noqa: BLE001 -- reported in the line
+        return {"error": f"{type(e).__name__}: {e}"}
 
 
 def run_reference(args, rank, world):
