@@ -105,6 +105,7 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.stamps = []  # host time each sample line arrived
 
     def __enter__(self):
         try:
@@ -125,6 +126,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
+            self.stamps.append(time.time())
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
@@ -136,10 +138,15 @@ class ClockSampler:
                 self.proc.kill()
             self.t.join(timeout=2)
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock, max clock and active throttle reasons of the samples
+        (only those that arrived between host times t0 and t1, when given)."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lines = self.lines
+        if t0 is not None:
+            lines = [l for l, t in zip(list(self.lines), list(self.stamps)) if t0 <= t <= t1]
+        for line in lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 8:
                 continue
@@ -434,11 +441,157 @@ def run_gpu(args, rank, world, local_rank):
     # side measurements: a failure here is reported in the line, never raised
     if world == 1:
         line["quantize_u8"] = _guarded(run_quantize, dev)
-    if args.sequence:
-        line["decode17"] = _guarded(run_sequence, args, dev)
+        if not args.no_workloads:
+            line["workloads"] = run_workloads(dev, peaks)
+        if not args.no_sequence:
+            line["decode17"] = _guarded(run_sequence, args, dev)
+        line["noalloc"] = _guarded(run_noalloc, conv, dev)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(conv, args.cpu_seconds)
     return line
+
+
+# ------------------------------------------------------ per-workload legs
+# FP32 FFMA peak of the SIMT path, from unit counts and the maximum clock:
+# 148 SMs x 128 FP32 lanes x 2 FLOP per FMA x 1.965 GHz.
+FP32_FFMA_TFLOPS = round(148 * 128 * 2 * 1.965e9 / 1e12, 2)
+FLUSH_BYTES = 256 * 1024 * 1024   # written between calls whose operands fit in L2 many times
+
+
+def bench_legs():
+    """(leg name, Conv, ring) for every config reported beside the headline:
+    the fp32 contract call, the bottleneck call and its cache sweep, the two
+    720x1280 calls, the edge sweep, the stride-2 cache sweep, the encoder
+    stride-2 calls, the decoder's thin RGB output conv, and the ring-buffer
+    variants of the bottleneck and stride-2 calls."""
+    W = workloads
+    legs = [(c.name, c, False) for c in (
+        W.C1, W.C2, W.C2_EMPTY, W.C4_C1, W.C3, W.C3B, W.C4_TIME, W.C4_DIL, W.C4_STRIDE,
+        W.C4_ODD, W.C6_ST2_TIME, W.C6_ST2, W.C_RGB)]
+    for name in sorted(W.WORKLOADS):
+        if name.startswith("bf16_192ch_s2_360x640_c") and name != W.C4_STRIDE.name:
+            legs.append((name, W.WORKLOADS[name], False))
+    legs += [(W.C2.name + "+ring", W.C2, True), (W.C4_STRIDE.name + "+ring", W.C4_STRIDE, True)]
+    return legs
+
+
+def ring_algorithmic_bytes(conv, intervals, nbytes):
+    """A ring-buffer call writes only the arriving frames of the new cache."""
+    z = conv.cache_len + conv.T_x
+    keep = min(conv.cache_keep, z)
+    e = 2 if conv.dtype == "bf16" else 4
+    return nbytes - e * conv.N * (keep - min(keep, conv.T_x)) * conv.H * conv.W * conv.Cin
+
+
+def time_leg(conv, ring, dev, peaks, sampler, seconds=0.6, min_calls=20, max_calls=4000):
+    """Median device time of one call of `conv` (CUDA events on the launching
+    stream, one event pair per call), operands cold in L2: rotated over sets
+    whose total exceeds twice the L2, or, for calls under 36 MB, a 256 MB
+    buffer written between calls.  Inputs are seeded N(0,1) activations and
+    N(0, 1/(Cin*kt*kh*kw)) weights drawn on the device."""
+    import torch
+    from causal_conv3d_video_b200 import ccv3d
+
+    plan = ccv3d.Plan(ccv3d.desc_for(conv))
+    flops, nbytes = algorithmic(conv, plan.intervals)
+    if ring:
+        nbytes = ring_algorithmic_bytes(conv, plan.intervals, nbytes)
+    dt = torch.bfloat16 if conv.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(hash(conv.name) & 0xFFFF)
+    flush = nbytes < 36e6
+    n_sets = 1 if flush else max(2, int(np.ceil(2.0 * L2_BYTES / nbytes)) + 1)
+    rnd = lambda shape, sigma: (sigma * torch.randn(shape, generator=gen, device=dev)).to(dt)
+    slots = conv.cache_len + plan.ring_writes()
+    sets = []
+    for _ in range(n_sets):
+        x = rnd((conv.N, conv.T_x, conv.H, conv.W, conv.Cin), 1.0)
+        w = rnd((conv.Cout, conv.kt, conv.kh, conv.kw, conv.Cin),
+                1.0 / np.sqrt(conv.Cin * conv.kt * conv.kh * conv.kw))
+        b = rnd((conv.Cout,), conv.sigma_b) if conv.has_bias else None
+        out, nc = plan.alloc_outputs(dev)
+        if ring:
+            cache = rnd((conv.N, slots, conv.H, conv.W, conv.Cin), 1.0)
+            nc = None
+        else:
+            cache = (rnd((conv.N, conv.cache_len, conv.H, conv.W, conv.Cin), 1.0)
+                     if conv.cache_len > 0 else None)
+        sets.append([x, cache, w, b, out, nc, 0])
+    scratch = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
+    stream = torch.cuda.current_stream(dev)
+
+    def call(i):
+        st = sets[i % n_sets]
+        x, cache, w, b, out, nc, head = st
+        if ring:
+            st[6] = plan.forward_ring(x, cache, slots, head, w, b, out, stream)
+        else:
+            plan.forward(x, cache, w, b, out, nc, stream)
+
+    def run(n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for i in range(n):
+            if flush:
+                scratch.fill_(float(i & 7))
+            evs[i][0].record(stream)
+            call(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) * 1e3 for a, b in evs]
+
+    run(3)  # warm-up
+    if plan.status() != 0:
+        raise RuntimeError(f"{conv.name}: device status {plan.status()} after warm-up")
+    est_us = statistics.median(run(3))
+    n = int(min(max_calls, max(min_calls, seconds / (est_us * 1e-6 + (4e-5 if flush else 0)))))
+    t0 = time.time()
+    per = run(n)
+    t1 = time.time()
+    if plan.status() != 0:
+        raise RuntimeError(f"{conv.name}: device status {plan.status()} after timing")
+    us = statistics.median(per)
+    if conv.dtype == "bf16":
+        peak, bound_unit = peaks["bf16_tflops"], "bf16 tensor (measured burst)"
+    else:
+        peak, bound_unit = FP32_FFMA_TFLOPS, "fp32 FFMA (derived: 148 SMs x 128 lanes x 2 x 1.965 GHz)"
+    t_flop = flops / (peak * 1e12) * 1e6
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_star = max(t_flop, t_hbm)
+    line = {
+        "kernel": plan.kernel, "calls": n, "us_per_call_median": round(us, 2),
+        "us_per_call_min": round(min(per), 2),
+        "gflop": round(flops / 1e9, 3), "mb": round(nbytes / 1e6, 2),
+        "tflops": round(flops / (us * 1e-6) / 1e12, 2),
+        "roofline": {
+            "bound": ("tensor" if conv.dtype == "bf16" else "alu") if t_flop >= t_hbm else "hbm",
+            "t_star_us": round(t_star, 2), "frac": round(t_star / us, 4),
+            "peak_flop": peak, "peak_flop_kind": bound_unit, "peak_hbm_gbs": peaks["hbm_gbs"],
+            "traffic": traffic_from_profiles(conv.name + ("+ring" if ring else "")),
+        },
+        "tensor_frac": round(t_flop / us, 4) if conv.dtype == "bf16" else None,
+        "hbm_frac": round(t_hbm / us, 4),
+        "l2": ("256 MB buffer written between calls" if flush
+               else f"rotating {n_sets} operand sets ({n_sets * nbytes / 1e6:.0f} MB)"),
+        "clocks": sampler.summary(t0, t1),
+    }
+    if ring:
+        line["ring_slots"] = slots
+    del sets, scratch
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_workloads(dev, peaks):
+    """One timed leg per config; a leg that fails reports its error."""
+    import torch
+
+    out = {}
+    with ClockSampler(dev.index or 0) as sampler:
+        for name, conv, ring in bench_legs():
+            out[name] = _guarded(time_leg, conv, ring, dev, peaks, sampler)
+            torch.cuda.synchronize()
+    return out
 
 
 # ------------------------------------------------- decode-sequence leg
@@ -450,6 +603,48 @@ def _guarded(fn, *a):
         import traceback
         traceback.print_exc()
         return {"error": f"{type(e).__name__}: {e}"}
+
+
+def run_noalloc(conv, dev, calls=50):
+    """ccv3d_forward_noalloc on the headline signature: the host time of one
+    call (it plans on the host stack every time) and its device time."""
+    import torch
+    from causal_conv3d_video_b200 import ccv3d
+
+    desc = ccv3d.desc_for(conv)
+    plan = ccv3d.Plan(desc)
+    dt = torch.bfloat16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    rnd = lambda shape, sigma: (sigma * torch.randn(shape, generator=gen, device=dev)).to(dt)
+    x = rnd((conv.N, conv.T_x, conv.H, conv.W, conv.Cin), 1.0)
+    cache = rnd((conv.N, conv.cache_len, conv.H, conv.W, conv.Cin), 1.0)
+    w = rnd((conv.Cout, conv.kt, conv.kh, conv.kw, conv.Cin), 1.0 / np.sqrt(conv.Cin * 27))
+    b = rnd((conv.Cout,), conv.sigma_b)
+    out, nc = plan.alloc_outputs(dev)
+    stream = torch.cuda.current_stream(dev)
+    f = lambda: ccv3d.ccv3d_forward_noalloc(desc, x, cache, w, b, out, nc, conv.stride,
+                                            conv.pad, conv.dilation, stream)
+    for _ in range(3):
+        f()
+    torch.cuda.synchronize()
+    host, dev_us = [], []
+    for _ in range(calls):
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        t = time.perf_counter()
+        f()
+        host.append((time.perf_counter() - t) * 1e6)
+        eb.record(stream)
+        torch.cuda.synchronize()
+        dev_us.append(ea.elapsed_time(eb) * 1e3)
+    status = ccv3d.ccv3d_noalloc_get_status(stream)
+    return {"host_us_per_call_median": round(statistics.median(host), 1),
+            "device_us_per_call_median": round(statistics.median(dev_us), 2),
+            "status": ccv3d.STATUS.get(status, status),
+            "what": "ccv3d_forward_noalloc on the headline signature (persistent kernel, "
+                    "scratch in the library's static array): host time of the call, which "
+                    "plans on the host stack, and device time"}
 
 
 def run_quantize(dev, steps=200):
@@ -529,13 +724,17 @@ def run_sequence(args, dev):
     gen.manual_seed(0)
     plans, frames, outs, mods = {}, {}, {}, {}
     flops = 0.0
+    t_star_us = 0.0  # sum over the calls of max(F/P, B/BW) at the measured peaks
+    peaks = load_peaks()
     for call in calls:
         c = call.conv
         sig = workloads.signature(c)
         if sig not in plans:
             plans[sig] = ccv3d.Plan(ccv3d.desc_for(c))
         plan = plans[sig]
-        flops += algorithmic(c, plan.intervals)[0]
+        f_i, b_i = algorithmic(c, plan.intervals)
+        flops += f_i
+        t_star_us += max(f_i / (peaks["bf16_tflops"] * 1e12), b_i / (peaks["hbm_gbs"] * 1e9)) * 1e6
         xs = (1, c.T_x, c.H, c.W, c.Cin)
         if xs not in frames:
             frames[xs] = torch.randn(xs, generator=gen, device=dev).to(torch.bfloat16)
@@ -600,16 +799,73 @@ def run_sequence(args, dev):
         if plan.status() != 0:
             raise RuntimeError("device status after the graph-replayed decode sequence")
     del graph
+
+    # the same pass with every module's cache in a ring buffer (only the
+    # arriving frames of each new cache are written)
+    rings = {}
+    for call in calls:
+        c = call.conv
+        m = call.module
+        plan = plans[workloads.signature(c)]
+        need = c.cache_len + plan.ring_writes()
+        if m not in rings or rings[m][1] < need:
+            rings[m] = [None, max(need, rings.get(m, [None, 0])[1]), 0]
+    for m, r in rings.items():
+        c = next(call.conv for call in calls if call.module == m)
+        r[0] = torch.randn((1, r[1], c.H, c.W, c.Cin), generator=gen, device=dev).to(torch.bfloat16)
+
+    def ring_pass(stream=stream):
+        for call in calls:
+            c = call.conv
+            plan = plans[workloads.signature(c)]
+            w, b = mods[call.module][0], mods[call.module][1]
+            ring = rings[call.module]
+            ring[2] = plan.forward_ring(frames[(1, c.T_x, c.H, c.W, c.Cin)], ring[0], ring[1],
+                                        ring[2], w, b, outs[plan.out_shape()], stream)
+
+    for _ in range(2):
+        ring_pass()
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(passes):
+        ring_pass()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    ms_ring = ea.elapsed_time(eb) / passes
+    graph = torch.cuda.CUDAGraph()
+    cap.wait_stream(stream)
+    with torch.cuda.graph(graph, stream=cap):
+        ring_pass(cap)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(passes):
+        graph.replay()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    ms_ring_graph = ea.elapsed_time(eb) / passes
+    for plan in plans.values():
+        if plan.status() != 0:
+            raise RuntimeError("device status after the ring-buffer decode sequence")
+    del graph
     kernels = sorted({p.kernel for p in plans.values()})
     return {"calls": len(calls), "signatures": len(plans), "ms_per_sequence": round(ms, 3),
             "tflops": round(flops / (ms / 1e3) / 1e12, 2), "gflop_per_sequence": round(flops / 1e9, 1),
             "ms_per_sequence_graph": round(ms_graph, 3),
             "tflops_graph": round(flops / (ms_graph / 1e3) / 1e12, 2),
+            "ms_per_sequence_ring": round(ms_ring, 3),
+            "ms_per_sequence_ring_graph": round(ms_ring_graph, 3),
+            "tflops_ring_graph": round(flops / (ms_ring_graph / 1e3) / 1e12, 2),
+            "t_star_ms": round(t_star_us / 1e3, 3),
+            "frac_of_roofline_graph": round(t_star_us / 1e3 / ms_graph, 4),
             "passes": passes, "kernels": kernels,
             "kernel_per_signature": {f"{k[0]}->{k[1]} k{k[2]}{k[3]}{k[4]} {k[5]}x{k[6]} T{k[7]} C{k[8]}":
                                      p.kernel for k, p in plans.items()},
             "what": "164-call synthetic 17-frame decode, caches threaded, one stream; "
-                    "eager launches, and the same pass captured as one CUDA graph"}
+                    "eager launches, and the same pass captured as one CUDA graph; then "
+                    "the pass with ring-buffer caches (ccv3d_forward_ring), eager and graph"}
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -735,8 +991,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sequence", action="store_true",
-                    help="also time the 164-call synthetic decode sequence")
+    ap.add_argument("--no-sequence", action="store_true",
+                    help="skip the 164-call synthetic decode sequence leg")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload legs")
     ap.add_argument("--sequence-passes", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:

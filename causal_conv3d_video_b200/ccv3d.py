@@ -11,12 +11,16 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "_lib", "libccv3d.so")
+# CCV3D_LIBRARY=checked loads the bounds-checked build (libccv3d_checked.so:
+# the same ABI, every computed device address range-checked); the tests use it
+LIB_PATH = os.path.join(_HERE, "_lib", "libccv3d_checked.so"
+                        if os.environ.get("CCV3D_LIBRARY") == "checked" else "libccv3d.so")
 
 CCV3D_BF16, CCV3D_FP32 = 0, 1
 STATUS = {0: "CCV3D_OK", 1: "CCV3D_ERR_INVALID", 2: "CCV3D_ERR_UNSUPPORTED",
           3: "CCV3D_ERR_EMPTY_OUTPUT", 4: "CCV3D_ERR_ALIGNMENT", 5: "CCV3D_ERR_ALIAS",
-          6: "CCV3D_ERR_CUDA", 7: "CCV3D_ERR_TIMEOUT", 8: "CCV3D_ERR_SCRATCH_LIMIT"}
+          6: "CCV3D_ERR_CUDA", 7: "CCV3D_ERR_TIMEOUT", 8: "CCV3D_ERR_SCRATCH_LIMIT",
+          9: "CCV3D_ERR_BOUNDS"}
 for _code, _name in STATUS.items():
     globals()[_name] = _code
 CCV3D_MAX_KT = 3
@@ -25,7 +29,9 @@ CCV3D_MAX_KT = 3
 EXPORTED = ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_plan_path", "ccv3d_forward",
             "ccv3d_get_stats", "ccv3d_get_status", "ccv3d_destroy", "ccv3d_strerror",
             "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout", "ccv3d_forward_noalloc",
-            "ccv3d_plan_kernel", "ccv3d_plan_tiling", "ccv3d_quantize_u8")
+            "ccv3d_plan_kernel", "ccv3d_plan_tiling", "ccv3d_quantize_u8",
+            "ccv3d_get_status_stream", "ccv3d_noalloc_get_status", "ccv3d_forward_ring",
+            "ccv3d_selftest_bounds")
 CCV3D_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -38,7 +44,8 @@ class ccv3d_desc(ctypes.Structure):
 
 class ccv3d_stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
-        "calls", "tc_path", "simt_path", "unsupported", "errors", "workspace_bytes")]
+        "calls", "tc_path", "simt_path", "unsupported", "errors", "workspace_bytes",
+        "plans_unsupported")]
 
 
 class CCV3DError(RuntimeError):
@@ -76,9 +83,16 @@ def _load():
     lib.ccv3d_quantize_u8.restype = ctypes.c_int
     lib.ccv3d_forward_noalloc.argtypes = [ctypes.POINTER(ccv3d_desc), vp, vp, vp, vp, vp, vp,
                                           ip, ip, ip, vp]
+    lib.ccv3d_get_status_stream.argtypes = [vp, vp]
+    lib.ccv3d_selftest_bounds.argtypes = [vp]
+    lib.ccv3d_selftest_bounds.restype = ctypes.c_int
+    lib.ccv3d_noalloc_get_status.argtypes = [vp]
+    lib.ccv3d_forward_ring.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                                       ip, ip, ip, vp, ip]
     for f in ("ccv3d_plan", "ccv3d_plan_intervals", "ccv3d_forward", "ccv3d_get_stats",
               "ccv3d_get_status", "ccv3d_plan_sizes", "ccv3d_selftest_wait_timeout",
-              "ccv3d_forward_noalloc"):
+              "ccv3d_forward_noalloc", "ccv3d_get_status_stream", "ccv3d_noalloc_get_status",
+              "ccv3d_forward_ring"):
         getattr(lib, f).restype = ctypes.c_int
     del i3
     return lib
@@ -170,6 +184,24 @@ def ccv3d_forward(plan, x, cache, w, bias, out, new_cache, stride, pad, dilation
     return rc
 
 
+def ccv3d_forward_ring(plan, x, ring, ring_slots: int, head: int, w, bias, out, stride, pad,
+                       dilation, stream=None, check: bool = True):
+    """The call with its cache in a ring buffer of ring_slots frames per batch
+    entry (cache frame t at slot (head + t) % ring_slots).  Writes only the
+    arriving frames of the new cache into the ring.  Returns (status,
+    next_head); raises CCV3DError on a refused call unless check=False."""
+    s = (ctypes.c_int * 2)(*stride)
+    p = (ctypes.c_int * 2)(*pad)
+    d = (ctypes.c_int * 3)(*dilation)
+    nh = ctypes.c_int(-1)
+    rc = lib.ccv3d_forward_ring(plan, _ptr(x), _ptr(ring), int(ring_slots), int(head), _ptr(w),
+                                _ptr(bias), _ptr(out), s, p, d, _stream(stream),
+                                ctypes.byref(nh))
+    if rc != 0 and check:
+        raise CCV3DError(rc, "ccv3d_forward_ring")
+    return rc, nh.value
+
+
 def ccv3d_forward_noalloc(desc: ccv3d_desc, x, cache, w, bias, out, new_cache, stride, pad,
                           dilation, stream=None, check: bool = True) -> int:
     """The no-allocation variant of ccv3d_forward: no plan, no device memory
@@ -198,6 +230,14 @@ def ccv3d_get_status(plan) -> int:
     return lib.ccv3d_get_status(plan)
 
 
+def ccv3d_get_status_stream(plan, stream=None) -> int:
+    return lib.ccv3d_get_status_stream(plan, _stream(stream))
+
+
+def ccv3d_noalloc_get_status(stream=None) -> int:
+    return lib.ccv3d_noalloc_get_status(_stream(stream))
+
+
 def ccv3d_destroy(plan) -> None:
     lib.ccv3d_destroy(plan)
 
@@ -221,6 +261,10 @@ def ccv3d_quantize_u8(x, out, stream=None, check: bool = True) -> int:
 
 def ccv3d_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     return lib.ccv3d_selftest_wait_timeout(int(limit_ns), _stream(stream))
+
+
+def ccv3d_selftest_bounds(stream=None) -> int:
+    return lib.ccv3d_selftest_bounds(_stream(stream))
 
 
 # ---------------------------------------------------------------- helpers
@@ -283,6 +327,15 @@ class Plan:
         return ccv3d_forward(self.handle, x, cache, w, bias, out, new_cache, self.stride,
                              self.pad, self.dilation, stream)
 
+    def forward_ring(self, x, ring, ring_slots, head, w, bias, out, stream=None):
+        """Ring-buffer cache call; returns the head of the new cache."""
+        return ccv3d_forward_ring(self.handle, x, ring, ring_slots, head, w, bias, out,
+                                  self.stride, self.pad, self.dilation, stream)[1]
+
+    def ring_writes(self):
+        """Frames of x a ring-buffer call writes into the ring."""
+        return min(self.sizes["new_cache_frames"], self.desc.T_x)
+
     def alloc_outputs(self, device="cuda"):
         import torch
         dt = torch.bfloat16 if self.desc.dtype == CCV3D_BF16 else torch.float32
@@ -296,6 +349,9 @@ class Plan:
 
     def status(self):
         return ccv3d_get_status(self.handle)
+
+    def status_stream(self, stream=None):
+        return ccv3d_get_status_stream(self.handle, stream)
 
     def close(self):
         if getattr(self, "handle", None) is not None:

@@ -3,13 +3,14 @@
 // Z is cache[t] when t < |C|, else x[t - |C|] (the paper's cache-augmented
 // input, Sec. 4; the cache carries Z's trailing frames to the next call).
 #pragma once
+#include "checked.cuh"
 #include "params.h"
 
 namespace ccv3d {
 
 __device__ __forceinline__ const uint8_t* z_frame(const CopyJob& c, int n, int t) {
     return t < c.cache_len
-               ? c.cache + ((long long)n * c.cache_len + t) * c.frame_bytes
+               ? c.cache + (long long)ring_frame(n, t, c.cache_slots, c.cache_head) * c.frame_bytes
                : c.x + ((long long)n * c.T_x + (t - c.cache_len)) * c.frame_bytes;
 }
 
@@ -33,8 +34,15 @@ __device__ __forceinline__ void copy_new_cache(const CopyJob& c, long long part,
         const long long lo = begin > f * per_frame ? begin - f * per_frame : 0;
         const long long hi = end < (f + 1) * per_frame ? end - f * per_frame : per_frame;
         const int n = (int)(f / c.keep), j = (int)(f % c.keep);
-        const uint8_t* src = z_frame(c, n, c.z_len - c.keep + j);
-        uint8_t* dst = c.dst + f * c.frame_bytes;
+        const int t = c.z_len - c.keep + j;
+        const uint8_t* src = z_frame(c, n, t);
+        uint8_t* dst = c.dst + (long long)ring_frame(n, j, c.dst_slots, c.dst_head) * c.frame_bytes;
+        // checked build: this slice's loop reads and writes exactly these ranges
+        if (!in_bounds(c.status, src + lo * vb, (hi - lo) * vb,
+                       t < c.cache_len ? c.cache : c.x,
+                       t < c.cache_len ? c.cache_bytes : c.x_bytes) ||
+            !in_bounds(c.status, dst + lo * vb, (hi - lo) * vb, c.dst, c.dst_bytes))
+            continue;
         if (vb == 16) {
             // kU independent 16-byte loads in flight per thread before their
             // stores (source and destination never overlap: checked on host)

@@ -21,6 +21,7 @@
 #include <new>
 
 #include "ccv3d.h"
+#include "checked.cuh"
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
 #include "conv_tc2.cuh"
@@ -44,6 +45,9 @@ struct ccv3d_plan_s {
     int halo;     // 1: pair kernel loading each input row strip once per (tap, channel block)
     int halo_w;   // halo: pixels per strip
     int fused;    // 1: halo pair kernel computing two output frames per tile
+    int simt_kind;  // SIMT plans: 0 thread per unit, 1 warp per unit, 2 shared-memory blocks
+    int simt_band_h, simt_rows_in, simt_threads;
+    size_t simt_smem;
     int G, n_acc;  // persistent: CTA pairs launched, TMEM accumulator buffers
     long long frame_start[kMaxFrames + 1], sk_total;
     size_t smem_bytes;
@@ -56,6 +60,10 @@ struct ccv3d_plan_s {
 };
 
 namespace {
+
+// ccv3d_plan calls refused as outside the contract, over the whole process
+// (a refused signature never gets a plan whose counters could hold it).
+std::atomic<uint64_t> g_plans_unsupported{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -170,10 +178,23 @@ int pick_stages(int kind, int bn, int want) {
     return s;
 }
 
+// Function attributes belong to each device's context: set them once per
+// device (the current one).
+constexpr int kMaxDevices = 64;
+
 template <int BK>
 void set_smem_attrs() {
-    static std::once_flag once;
-    std::call_once(once, [] {
+    static std::atomic<bool> done[kMaxDevices];
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    if (dev < 0 || dev >= kMaxDevices || done[dev].load(std::memory_order_acquire)) return;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev].load(std::memory_order_relaxed)) return;
+    {
         cudaFuncSetAttribute(conv_tc_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaFuncSetAttribute(conv_tc2_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -185,12 +206,35 @@ void set_smem_attrs() {
         cudaFuncSetAttribute(conv_tc2f_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaGetLastError();
-    });
+    }
+    done[dev].store(true, std::memory_order_release);
 }
 
-// CTA pairs of the persistent kernel that can be resident at once.
+// CTA pairs of the persistent kernel that can be resident at once.  The
+// occupancy query costs milliseconds of host time, so its answer is kept per
+// (device, channel block, shared memory) for the life of the process.
+struct ResidentEntry {
+    int dev, bk, pairs;
+    size_t smem;
+};
+constexpr int kResidentEntries = 64;
+std::mutex g_resident_mu;
+ResidentEntry g_resident[kResidentEntries];
+int g_resident_n = 0;
+
 template <int BK>
 int resident_pairs(size_t smem) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_resident_mu);
+        for (int i = 0; i < g_resident_n; ++i)
+            if (g_resident[i].dev == dev && g_resident[i].bk == BK && g_resident[i].smem == smem)
+                return g_resident[i].pairs;
+    }
     set_smem_attrs<BK>();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
@@ -201,17 +245,30 @@ int resident_pairs(size_t smem) {
         cudaGetLastError();
         return 0;
     }
+    std::lock_guard<std::mutex> lock(g_resident_mu);
+    if (g_resident_n < kResidentEntries) g_resident[g_resident_n++] = {dev, BK, n, smem};
     return n;
 }
 
+// Planner overrides (kernel form, tiling, ring depth) for tests and tuning
+// sweeps.  They are read only when CCV3D_TEST_OVERRIDES=1 is also set, so a
+// deployment's environment cannot change the kernel, the reduction order or
+// the performance behind the ABI; without the gate every plan is the
+// planner's own choice.
+const char* override_env(const char* name) {
+    const char* gate = std::getenv("CCV3D_TEST_OVERRIDES");
+    if (gate == nullptr || std::strcmp(gate, "1") != 0) return nullptr;
+    return std::getenv(name);
+}
+
 bool force_simt() {
-    const char* e = std::getenv("CCV3D_FORCE_PATH");
+    const char* e = override_env("CCV3D_FORCE_PATH");
     return e != nullptr && std::strcmp(e, "simt") == 0;
 }
 
-// Tiling overrides for tuning sweeps (0 = the planner's choice).
+// Integer override (0 = the planner's choice).
 int env_int(const char* name) {
-    const char* e = std::getenv(name);
+    const char* e = override_env(name);
     return e != nullptr ? std::atoi(e) : 0;
 }
 
@@ -278,7 +335,7 @@ void size_tc(const ccv3d_desc& d, ccv3d_plan_s* p) {
 // CCV3D_STAGES override its channel block and depth.
 void setup_halo(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->halo = 0;
-    const char* he = std::getenv("CCV3D_HALO");
+    const char* he = override_env("CCV3D_HALO");
     if (he != nullptr && std::atoi(he) == 0) return;
     if (!p->pair || p->persist) return;
     if (p->box_w != 128 || p->box_h != 1 || d.stride_w != 1) return;
@@ -310,7 +367,7 @@ void setup_halo(const ccv3d_desc& d, ccv3d_plan_s* p) {
 // against the halo kernel.  CCV3D_FUSE=0 disables it.
 void setup_fused(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->fused = 0;
-    const char* fe = std::getenv("CCV3D_FUSE");
+    const char* fe = override_env("CCV3D_FUSE");
     if (fe != nullptr && std::atoi(fe) == 0) return;
     if (!p->halo || d.stride_t != 1 || d.dil_t != 1 || p->T_o < 2) return;
     if (p->tiles_n != 1 || p->n_sub != 1 || 2 * p->BN > 256) return;
@@ -388,7 +445,7 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     if (p->n_sub == 2 && p->BN % 32 != 0) p->BN = ((p->BN + 31) / 32) * 32;
     p->BK = widest_bk(d.Cin);
     // CTA pairs whenever every pair MMA has N >= 32 (16 weight rows per CTA)
-    const char* pe = std::getenv("CCV3D_PAIR");
+    const char* pe = override_env("CCV3D_PAIR");
     p->pair = (p->BN / p->n_sub) >= 32 ? 1 : 0;
     if (pe != nullptr) p->pair = std::atoi(pe) != 0 && (p->BN / p->n_sub) >= 32;
     p->path_tc_candidate = 1;
@@ -396,7 +453,7 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     size_tc(d, p);
     setup_halo(d, p);
     setup_fused(d, p);
-    const char* ps = std::getenv("CCV3D_PERSIST");
+    const char* ps = override_env("CCV3D_PERSIST");
     const bool persist = ps != nullptr ? std::atoi(ps) > 0 : prefer_persistent(d, *p);
     if (persist && setup_persistent(d, p)) size_tc(d, p);
     p->path_tc = 1;
@@ -497,17 +554,51 @@ ccv3d_status encode_out(CUtensorMap* m, void* base, const ccv3d_desc& d, const c
     return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
 }
 
-CopyJob make_copy(const ccv3d_plan_s* p, const void* x, const void* cache, void* nc) {
+// Where one call reads its cached frames and writes the frames it keeps.
+struct CacheIO {
+    const void* cache;            // [N, cache_slots, H, W, Cin]
+    int cache_slots, cache_head;  // cache frame t at slot (cache_head + t) mod cache_slots
+    void* dst;                    // [N, dst_slots, H, W, Cin]
+    int dst_slots, dst_head;      // kept frame j at slot (dst_head + j) mod dst_slots
+    int copy_frames;              // frames written per batch entry: the last ones of Z
+};
+
+// ccv3d_forward: a dense cache in, a dense new_cache of K' frames out.
+CacheIO dense_io(const ccv3d_plan_s* p, const void* cache, void* nc) {
+    CacheIO io;
+    io.cache = cache;
+    io.cache_slots = p->d.cache_len;
+    io.cache_head = 0;
+    io.dst = nc;
+    io.dst_slots = p->keep;
+    io.dst_head = 0;
+    io.copy_frames = nc != nullptr ? p->keep : 0;
+    return io;
+}
+
+// Frames of x a ring-buffer call writes: those of the new cache that arrive
+// with this call (the others are already in the ring).
+int ring_writes(const ccv3d_plan_s* p) { return std::min(p->keep, p->d.T_x); }
+
+CopyJob make_copy(const ccv3d_plan_s* p, const void* x, const CacheIO& io) {
     CopyJob c;
     c.x = static_cast<const uint8_t*>(x);
-    c.cache = static_cast<const uint8_t*>(cache);
-    c.dst = static_cast<uint8_t*>(nc);
+    c.cache = static_cast<const uint8_t*>(io.cache);
+    c.dst = static_cast<uint8_t*>(io.dst);
     c.frame_bytes = (long long)p->d.H * p->d.W * p->d.Cin * (long long)elt(p->d);
-    c.keep = nc != nullptr ? p->keep : 0;
+    c.keep = io.dst != nullptr ? io.copy_frames : 0;
     c.cache_len = p->d.cache_len;
     c.T_x = p->d.T_x;
     c.z_len = p->z_len;
     c.N = p->d.N;
+    c.cache_slots = io.cache_slots;
+    c.cache_head = io.cache_head;
+    c.dst_slots = io.dst_slots;
+    c.dst_head = io.dst_head;
+    c.x_bytes = (long long)p->d.N * p->d.T_x * c.frame_bytes;
+    c.cache_bytes = io.cache != nullptr ? (long long)p->d.N * io.cache_slots * c.frame_bytes : 0;
+    c.dst_bytes = io.dst != nullptr ? (long long)p->d.N * io.dst_slots * c.frame_bytes : 0;
+    c.status = p->d_status;
     return c;
 }
 
@@ -539,27 +630,31 @@ cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cuda
     return cudaGetLastError();
 }
 
-ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const void* cache, const void* w,
-                    const void* bias, void* out, void* nc, cudaStream_t stream) {
+ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const void* w,
+                    const void* bias, void* out, cudaStream_t stream) {
     if (encode_fn() == nullptr) return CCV3D_ERR_CUDA;
     const ccv3d_desc& d = p->d;
     TcParams prm;
     std::memset(&prm, 0, sizeof(prm));
     ccv3d_status st = encode_act(&prm.tmap_x, x, d.N * d.T_x, d, p);
-    if (st == CCV3D_OK && d.cache_len > 0) st = encode_act(&prm.tmap_c, cache, d.N * d.cache_len, d, p);
+    if (st == CCV3D_OK && d.cache_len > 0)
+        st = encode_act(&prm.tmap_c, io.cache, d.N * io.cache_slots, d, p);
     if (st == CCV3D_OK) st = encode_w(&prm.tmap_w, w, d, p);
     if (st == CCV3D_OK) st = encode_out(&prm.tmap_out, out, d, p);
     if (st != CCV3D_OK) return st;
     prm.bias = d.has_bias ? static_cast<const uint16_t*>(bias) : nullptr;
     prm.out = static_cast<uint16_t*>(out);
     prm.status = p->d_status;
-    prm.copy = make_copy(p, x, cache, nc);
+    prm.copy = make_copy(p, x, io);
     prm.taps = make_taps(p);
     prm.N = d.N; prm.T_o = p->T_o; prm.H_o = p->H_o; prm.W_o = p->W_o;
     prm.Cin = d.Cin; prm.Cout = d.Cout; prm.kh = d.kh; prm.kw = d.kw;
     prm.s_h = d.stride_h; prm.s_w = d.stride_w; prm.p_h = d.pad_h; prm.p_w = d.pad_w;
     prm.d_h = d.dil_h; prm.d_w = d.dil_w;
     prm.cache_len = d.cache_len; prm.T_x = d.T_x;
+    prm.cache_slots = io.cache_slots; prm.cache_head = io.cache_head;
+    prm.x_frames = d.N * d.T_x;
+    prm.c_frames = d.N * io.cache_slots;
     prm.box_h = p->box_h; prm.box_w = p->box_w;
     prm.tiles_x = p->tiles_x; prm.tiles_y = p->tiles_y; prm.tiles_n = p->tiles_n;
     prm.BN = p->BN; prm.n_sub = p->n_sub; prm.n_cb = ceil_div(d.Cin, p->BK);
@@ -612,15 +707,62 @@ bool simt_uses_warps(const ccv3d_plan_s& p) {
     return units < (long long)kSmCount * kSimtThreads;
 }
 
-ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const void* cache, const void* w,
-                      const void* bias, void* out, void* nc, cudaStream_t stream) {
+constexpr size_t kSimtSmemMax = 96 * 1024;
+
+// Small calls whose weights and a band of input rows fit in shared memory run
+// the shared-memory kernel; its band height aims at ~256 units per block.
+void choose_simt(ccv3d_plan_s* p) {
+    const ccv3d_desc& d = p->d;
+    p->simt_kind = simt_uses_warps(*p) ? 1 : 0;
+    const bool smem_off = override_env("CCV3D_SIMT_SMEM") != nullptr && env_int("CCV3D_SIMT_SMEM") == 0;
+    if (p->simt_kind != 1 || smem_off) return;
+    const long long w_floats = (long long)d.Cout * d.kt * d.kh * d.kw * d.Cin;
+    const int Wp = d.W + 2 * d.pad_w;
+    const long long row_units = (long long)p->W_o * ceil_div(d.Cout, kSimtCoT);
+    int bh = (int)std::max<long long>(1, std::min<long long>(p->H_o, 256 / std::max(1LL, row_units)));
+    for (; bh >= 1; --bh) {
+        const int rows_in = (bh - 1) * d.stride_h + (d.kh - 1) * d.dil_h + 1;
+        const size_t bytes = 4 * (size_t)simt_smem_floats(w_floats, d.kt, rows_in, Wp, d.Cin);
+        if (bytes <= kSimtSmemMax) {
+            p->simt_kind = 2;
+            p->simt_band_h = bh;
+            p->simt_rows_in = rows_in;
+            p->simt_smem = bytes;
+            const long long u = bh * row_units;
+            p->simt_threads = (int)std::min<long long>(256, std::max<long long>(32, (u + 31) / 32 * 32));
+            return;
+        }
+    }
+}
+
+template <typename T>
+void set_simt_smem_attr() {
+    static std::atomic<bool> done[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    if (dev < 0 || dev >= kMaxDevices || done[dev].load(std::memory_order_acquire)) return;
+    cudaFuncSetAttribute(conv_simt_smem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kSimtSmemMax);
+    cudaGetLastError();
+    done[dev].store(true, std::memory_order_release);
+}
+
+ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const CacheIO& io, const void* w,
+                      const void* bias, void* out, cudaStream_t stream) {
     const ccv3d_desc& d = p->d;
     SimtParams prm;
     std::memset(&prm, 0, sizeof(prm));
-    prm.x = x; prm.cache = cache; prm.w = w;
+    prm.x = x; prm.cache = io.cache; prm.w = w;
     prm.bias = d.has_bias ? bias : nullptr;
     prm.out = out;
-    prm.copy = make_copy(p, x, cache, nc);
+    prm.copy = make_copy(p, x, io);
+    prm.cache_slots = io.cache_slots; prm.cache_head = io.cache_head;
+    prm.status = p->d_status;
+    prm.w_floats = (long long)d.Cout * d.kt * d.kh * d.kw * d.Cin;
+    prm.out_elems = (long long)d.N * p->T_o * p->H_o * p->W_o * d.Cout;
     prm.taps = make_taps(p);
     prm.N = d.N; prm.T_o = p->T_o; prm.H_o = p->H_o; prm.W_o = p->W_o;
     prm.Cin = d.Cin; prm.Cout = d.Cout; prm.H = d.H; prm.W = d.W; prm.kh = d.kh; prm.kw = d.kw;
@@ -629,7 +771,29 @@ ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const void* cache, const v
     prm.cache_len = d.cache_len; prm.T_x = d.T_x;
     prm.co_groups = ceil_div(d.Cout, kSimtCoT);
     prm.conv_threads = (long long)d.N * p->T_o * p->H_o * p->W_o * prm.co_groups;
-    const bool warp = simt_uses_warps(*p);
+    if (p->simt_kind == 2) {
+        prm.band_h = p->simt_band_h;
+        prm.bands = ceil_div(p->H_o, p->simt_band_h);
+        prm.rows_in = p->simt_rows_in;
+        prm.Wp = d.W + 2 * d.pad_w;
+        const long long cb = (long long)d.N * p->T_o * prm.bands;
+        const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
+        const long long kb =
+            copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 16383) / 16384) : 0;
+        if (cb + kb > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
+        prm.conv_blocks = (int)cb;
+        prm.copy_blocks = (int)kb;
+        const int grid = (int)(cb + kb);
+        if (d.dtype == CCV3D_FP32) {
+            set_simt_smem_attr<float>();
+            conv_simt_smem_kernel<float><<<grid, p->simt_threads, p->simt_smem, stream>>>(prm);
+        } else {
+            set_simt_smem_attr<__nv_bfloat16>();
+            conv_simt_smem_kernel<__nv_bfloat16><<<grid, p->simt_threads, p->simt_smem, stream>>>(prm);
+        }
+        return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+    }
+    const bool warp = p->simt_kind == 1;
     const long long cb = (prm.conv_threads * (warp ? 32 : 1) + kSimtThreads - 1) / kSimtThreads;
     const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
     const long long kb = copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 32767) / 32768) : 0;
@@ -679,6 +843,67 @@ ccv3d_status check_call(const ccv3d_plan_s* p, const void* x, const void* cache,
     return CCV3D_OK;
 }
 
+// Read a status word after the work already queued on `stream`, and clear
+// it when it holds an error.  Synchronises that stream only; the copy goes to
+// pageable host memory, so nothing is allocated.
+ccv3d_status read_and_clear_status(int* d_status, cudaStream_t stream) {
+    int v = 0;
+    if (cudaMemcpyAsync(&v, d_status, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CCV3D_ERR_CUDA;
+    }
+    if (v != 0 && (cudaMemsetAsync(d_status, 0, sizeof(int), stream) != cudaSuccess ||
+                   cudaStreamSynchronize(stream) != cudaSuccess)) {
+        cudaGetLastError();
+        return CCV3D_ERR_CUDA;
+    }
+    return v == 0 ? CCV3D_OK : (ccv3d_status)v;
+}
+
+// Argument checks of a ring-buffer call against its plan (no device work).
+ccv3d_status check_ring_call(const ccv3d_plan_s* p, const void* x, const void* ring,
+                             int ring_slots, int head, const void* w, const void* bias,
+                             const void* out, const int stride[2], const int pad[2],
+                             const int dilation[3]) {
+    const ccv3d_desc& d = p->d;
+    if (stride == nullptr || pad == nullptr || dilation == nullptr) return CCV3D_ERR_INVALID;
+    if (stride[0] != d.stride_h || stride[1] != d.stride_w || pad[0] != d.pad_h ||
+        pad[1] != d.pad_w || dilation[0] != d.dil_t || dilation[1] != d.dil_h ||
+        dilation[2] != d.dil_w)
+        return CCV3D_ERR_INVALID;
+    const int writes = ring_writes(p);
+    const bool uses_ring = d.cache_len > 0 || writes > 0;
+    // the slots this call writes must not hold a frame it reads
+    if (ring_slots < 1 || head < 0 || head >= ring_slots || d.cache_len + writes > ring_slots)
+        return CCV3D_ERR_INVALID;
+    if (x == nullptr || w == nullptr || out == nullptr || (uses_ring && ring == nullptr) ||
+        (d.has_bias && bias == nullptr))
+        return CCV3D_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out) || (uses_ring && !aligned16(ring)) ||
+        (d.has_bias && (reinterpret_cast<uintptr_t>(bias) % elt(d)) != 0))
+        return CCV3D_ERR_ALIGNMENT;
+    const size_t e = elt(d);
+    const size_t frame = (size_t)d.H * d.W * d.Cin * e;
+    const size_t x_bytes = (size_t)d.N * d.T_x * frame;
+    const size_t r_bytes = uses_ring ? (size_t)d.N * ring_slots * frame : 0;
+    const size_t o_bytes = (size_t)d.N * p->T_o * p->H_o * p->W_o * d.Cout * e;
+    const size_t w_bytes = (size_t)d.Cout * d.kt * d.kh * d.kw * d.Cin * e;
+    if (overlaps(ring, r_bytes, x, x_bytes) || overlaps(out, o_bytes, ring, r_bytes) ||
+        overlaps(out, o_bytes, x, x_bytes) || overlaps(out, o_bytes, w, w_bytes) ||
+        overlaps(ring, r_bytes, w, w_bytes))
+        return CCV3D_ERR_ALIAS;
+    return CCV3D_OK;
+}
+
+// One thread hands the range checks a byte range that ends one byte past its
+// buffer and an index one past its count; nothing is dereferenced.
+__global__ void bounds_selftest_kernel(int* status) {
+    const char* base = reinterpret_cast<const char*>(status);
+    if (in_bounds(status, base, sizeof(int) + 1, base, sizeof(int))) return;
+    index_ok(status, 1, 1);
+}
+
 __global__ void wait_selftest_kernel(int* status, uint64_t limit_ns) {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
@@ -702,10 +927,12 @@ ccv3d_status ccv3d_plan(ccv3d_plan_t* out, const ccv3d_desc* desc) {
     p->d = *desc;
     ccv3d_status st = compute_intervals(*desc, p);
     if (st != CCV3D_OK) {
+        if (st == CCV3D_ERR_UNSUPPORTED) g_plans_unsupported.fetch_add(1, std::memory_order_relaxed);
         delete p;
         return st;
     }
     choose_path(*desc, p);
+    if (!p->path_tc) choose_simt(p);
     // The status block lives on the current device.  Without any CUDA device
     // the plan still serves inspection (intervals, sizes, path) and
     // ccv3d_forward refuses with CCV3D_ERR_CUDA.
@@ -763,7 +990,7 @@ int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
 
 const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
     if (p == nullptr) return "";
-    if (!p->path_tc) return simt_uses_warps(*p) ? "simt_warp" : "simt";
+    if (!p->path_tc) return p->simt_kind == 2 ? "simt_smem" : (p->simt_kind == 1 ? "simt_warp" : "simt");
     if (p->fused) return "tc_pair_fused";
     if (p->halo) return "tc_pair_halo";
     if (p->persist) return "tc_persistent";
@@ -797,7 +1024,8 @@ ccv3d_status ccv3d_forward(ccv3d_plan_t p, const void* x, const void* cache, con
                            const int pad[2], const int dilation[3], cudaStream_t stream) {
     if (p == nullptr) return CCV3D_ERR_INVALID;
     auto refuse = [&](ccv3d_status s) {
-        p->errors.fetch_add(1, std::memory_order_relaxed);
+        (s == CCV3D_ERR_UNSUPPORTED ? p->unsupported : p->errors)
+            .fetch_add(1, std::memory_order_relaxed);
         return s;
     };
     const ccv3d_status chk = check_call(p, x, cache, w, bias, out, nc, stride, pad, dilation);
@@ -805,9 +1033,47 @@ ccv3d_status ccv3d_forward(ccv3d_plan_t p, const void* x, const void* cache, con
     if (p->d_status == nullptr) return refuse(CCV3D_ERR_CUDA);
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return refuse(CCV3D_ERR_INVALID);
-    ccv3d_status st = p->path_tc ? run_tc(p, x, cache, w, bias, out, nc, stream)
-                                 : run_simt(p, x, cache, w, bias, out, nc, stream);
+    const CacheIO io = dense_io(p, cache, nc);
+    ccv3d_status st = p->path_tc ? run_tc(p, x, io, w, bias, out, stream)
+                                 : run_simt(p, x, io, w, bias, out, stream);
     if (st != CCV3D_OK) return refuse(st);
+    p->calls.fetch_add(1, std::memory_order_relaxed);
+    (p->path_tc ? p->tc : p->simt).fetch_add(1, std::memory_order_relaxed);
+    return CCV3D_OK;
+}
+
+ccv3d_status ccv3d_forward_ring(ccv3d_plan_t p, const void* x, void* ring, int ring_slots,
+                                int head, const void* w, const void* bias, void* out,
+                                const int stride[2], const int pad[2], const int dilation[3],
+                                cudaStream_t stream, int* next_head) {
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    auto refuse = [&](ccv3d_status s) {
+        (s == CCV3D_ERR_UNSUPPORTED ? p->unsupported : p->errors)
+            .fetch_add(1, std::memory_order_relaxed);
+        return s;
+    };
+    const ccv3d_status chk =
+        check_ring_call(p, x, ring, ring_slots, head, w, bias, out, stride, pad, dilation);
+    if (chk != CCV3D_OK) return refuse(chk);
+    if (p->d_status == nullptr) return refuse(CCV3D_ERR_CUDA);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return refuse(CCV3D_ERR_INVALID);
+    const ccv3d_desc& d = p->d;
+    const int writes = ring_writes(p);
+    CacheIO io;
+    io.cache = ring;
+    io.cache_slots = ring_slots;
+    io.cache_head = head;
+    io.dst = ring;
+    io.dst_slots = ring_slots;
+    io.dst_head = (head + d.cache_len) % ring_slots;
+    io.copy_frames = writes;
+    ccv3d_status st = p->path_tc ? run_tc(p, x, io, w, bias, out, stream)
+                                 : run_simt(p, x, io, w, bias, out, stream);
+    if (st != CCV3D_OK) return refuse(st);
+    if (next_head != nullptr)
+        *next_head = (int)(((long long)head + d.cache_len + writes - p->keep) % ring_slots +
+                           ring_slots) % ring_slots;
     p->calls.fetch_add(1, std::memory_order_relaxed);
     (p->path_tc ? p->tc : p->simt).fetch_add(1, std::memory_order_relaxed);
     return CCV3D_OK;
@@ -821,6 +1087,7 @@ ccv3d_status ccv3d_get_stats(ccv3d_plan_t p, ccv3d_stats* s) {
     s->unsupported = p->unsupported.load();
     s->errors = p->errors.load();
     s->workspace_bytes = p->scratch_bytes;
+    s->plans_unsupported = g_plans_unsupported.load();
     return CCV3D_OK;
 }
 
@@ -833,6 +1100,12 @@ ccv3d_status ccv3d_get_status(ccv3d_plan_t p) {
         return CCV3D_ERR_CUDA;
     if (v != 0 && cudaMemset(p->d_status, 0, sizeof(int)) != cudaSuccess) return CCV3D_ERR_CUDA;
     return v == 0 ? CCV3D_OK : (ccv3d_status)v;
+}
+
+ccv3d_status ccv3d_get_status_stream(ccv3d_plan_t p, cudaStream_t stream) {
+    if (p == nullptr) return CCV3D_ERR_INVALID;
+    if (p->d_status == nullptr) return CCV3D_ERR_CUDA;
+    return read_and_clear_status(p->d_status, stream);
 }
 
 void ccv3d_destroy(ccv3d_plan_t p) {
@@ -854,6 +1127,8 @@ const char* ccv3d_strerror(ccv3d_status s) {
         case CCV3D_ERR_TIMEOUT: return "bounded device wait timed out";
         case CCV3D_ERR_SCRATCH_LIMIT:
             return "call needs more device scratch than the no-allocation entry point holds";
+        case CCV3D_ERR_BOUNDS:
+            return "bounds-checked build: a kernel computed an address outside its buffer";
     }
     return "unknown status";
 }
@@ -877,6 +1152,22 @@ ccv3d_status ccv3d_quantize_u8(const void* in, ccv3d_dtype dtype, void* out, lon
         quantize_u8_bf16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(in),
                                                              static_cast<uint8_t*>(out), n);
     return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+ccv3d_status ccv3d_selftest_bounds(cudaStream_t stream) {
+    int* d = nullptr;
+    if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) return CCV3D_ERR_CUDA;
+    int v = -1;
+    cudaError_t e = cudaMemsetAsync(d, 0, sizeof(int), stream);
+    if (e == cudaSuccess) {
+        bounds_selftest_kernel<<<1, 1, 0, stream>>>(d);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&v, d, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    cudaFree(d);
+    if (e != cudaSuccess) return CCV3D_ERR_CUDA;
+    return v == kStatusBounds ? CCV3D_ERR_BOUNDS : (v == 0 ? CCV3D_OK : CCV3D_ERR_CUDA);
 }
 
 ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
@@ -960,10 +1251,27 @@ extern "C" ccv3d_status ccv3d_forward_noalloc(const ccv3d_desc* desc, const void
     p.device = dev;
     p.d_status = static_cast<int*>(base);
     p.scratch = static_cast<unsigned char*>(base) + kNoallocStatusBytes;
-    p.epoch.store(g_noalloc_calls[dev].fetch_add(1));
-    if (cudaMemsetAsync(p.d_status, 0, sizeof(int), stream) != cudaSuccess) {
+    // This call's split-tile epoch: the next value of the device's call
+    // counter, skipping 0 ("never published"), so no two calls within 2^32
+    // share one.  run_tc adds 1 to the plan's counter, hence the e - 1.
+    unsigned e;
+    do {
+        e = g_noalloc_calls[dev].fetch_add(1) + 1u;
+    } while (e == 0u);
+    p.epoch.store(e - 1u);
+    // The status word is not cleared here: it keeps the first timeout any
+    // call recorded until ccv3d_noalloc_get_status reads it.
+    return run_tc(&p, x, dense_io(&p, cache, nc), w, bias, out, stream);
+}
+
+extern "C" ccv3d_status ccv3d_noalloc_get_status(cudaStream_t stream) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return CCV3D_ERR_CUDA;
     }
-    return run_tc(&p, x, cache, w, bias, out, nc, stream);
+    void* base = nullptr;
+    const ccv3d_status st = noalloc_scratch(dev, &base);
+    if (st != CCV3D_OK) return st;
+    return read_and_clear_status(static_cast<int*>(base), stream);
 }

@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 
 #include "cache_copy.cuh"
+#include "checked.cuh"
 #include "params.h"
 
 namespace ccv3d {
@@ -68,9 +69,12 @@ conv_simt_kernel(const __grid_constant__ SimtParams p) {
     for (int k = 0; k < p.taps.kt; ++k) {
         if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
         const int t = o * p.taps.s_t + p.taps.delta[k];
-        const T* frame = t < p.cache_len
-                             ? cache + ((long long)n * p.cache_len + t) * p.H * p.W * p.Cin
-                             : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * p.W * p.Cin;
+        const T* frame =
+            t < p.cache_len
+                ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) * p.H * p.W * p.Cin
+                : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * p.W * p.Cin;
+        const void* src_base = t < p.cache_len ? (const void*)cache : (const void*)x;
+        const long long src_bytes = t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes;
         for (int r = 0; r < p.kh; ++r) {
             const int yi = yo * p.s_h + r * p.d_h - p.p_h;
             if (yi < 0 || yi >= p.H) continue;
@@ -80,11 +84,21 @@ conv_simt_kernel(const __grid_constant__ SimtParams p) {
                 const T* zrow = frame + ((long long)yi * p.W + xi) * p.Cin;
                 const T* wrow = w + (((long long)co0 * p.taps.kt + k) * p.kh + r) * p.kw * p.Cin +
                                 (long long)s * p.Cin;
+                // checked build: the input pixel and the weight rows read below
+                if (!in_bounds(p.status, zrow, (long long)p.Cin * sizeof(T), src_base, src_bytes))
+                    continue;
+                bool wok[kSimtCoT];
+#pragma unroll
+                for (int j = 0; j < kSimtCoT; ++j)
+                    wok[j] = co0 + j < p.Cout &&
+                             in_bounds(p.status, wrow + j * w_co_stride,
+                                       (long long)p.Cin * sizeof(T), w,
+                                       p.w_floats * (long long)sizeof(T));
                 for (int ci = 0; ci < p.Cin; ++ci) {
                     const float z = to_f32<T>(zrow[ci]);
 #pragma unroll
                     for (int j = 0; j < kSimtCoT; ++j)
-                        if (co0 + j < p.Cout)
+                        if (wok[j])
                             acc[j] = fmaf(z, to_f32<T>(wrow[j * w_co_stride + ci]), acc[j]);
                 }
             }
@@ -93,9 +107,11 @@ conv_simt_kernel(const __grid_constant__ SimtParams p) {
     const T* bias = static_cast<const T*>(p.bias);
     T* out = static_cast<T*>(p.out) +
              ((((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo) * p.Cout;
+    const long long out_i = (((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo;
 #pragma unroll
     for (int j = 0; j < kSimtCoT; ++j) {
         if (co0 + j >= p.Cout) break;
+        if (!index_ok(p.status, out_i * p.Cout + co0 + j, p.out_elems)) break;
         float v = acc[j];
         if (bias != nullptr) v += to_f32<T>(bias[co0 + j]);
         out[co0 + j] = from_f32<T>(v);
@@ -165,13 +181,20 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
                 const int t = o * p.taps.s_t + p.taps.delta[k];
                 const T* frame =
                     t < p.cache_len
-                        ? cache + ((long long)n * p.cache_len + t) * p.H * p.W * p.Cin
+                        ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) * p.H *
+                                      p.W * p.Cin
                         : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * p.W * p.Cin;
-                z[u] = to_f32<T>(frame[((long long)yi * p.W + xi) * p.Cin + ci]);
+                const T* zp = frame + ((long long)yi * p.W + xi) * p.Cin + ci;
+                if (in_bounds(p.status, zp, sizeof(T), t < p.cache_len ? (const void*)cache : (const void*)x,
+                              t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
+                    z[u] = to_f32<T>(*zp);
                 const T* wcol = w + (long long)co0 * w_co_stride + (long long)tap * p.Cin + ci;
 #pragma unroll
                 for (int j = 0; j < kSimtCoT; ++j)
-                    if (co0 + j < p.Cout) wv[u][j] = to_f32<T>(wcol[j * w_co_stride]);
+                    if (co0 + j < p.Cout &&
+                        in_bounds(p.status, wcol + j * w_co_stride, sizeof(T), w,
+                                  p.w_floats * (long long)sizeof(T)))
+                        wv[u][j] = to_f32<T>(wcol[j * w_co_stride]);
             }
         }
 #pragma unroll
@@ -187,12 +210,186 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
     const T* bias = static_cast<const T*>(p.bias);
     T* out = static_cast<T*>(p.out) +
              ((((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo) * p.Cout;
+    const long long out_i = (((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo;
 #pragma unroll
     for (int j = 0; j < kSimtCoT; ++j) {
         if (co0 + j >= p.Cout) break;
+        if (!index_ok(p.status, out_i * p.Cout + co0 + j, p.out_elems)) break;
         float v = acc[j];
         if (bias != nullptr) v += to_f32<T>(bias[co0 + j]);
         out[co0 + j] = from_f32<T>(v);
+    }
+}
+
+// Small calls (a few thousand (pixel, 4-channel) units, e.g. the 16-channel
+// fp32 contract call): one block per (output frame, band of band_h output
+// rows).  The block first stages, as fp32 in shared memory and with 16-byte
+// global loads where the layout allows, every weight of the call and, for
+// each active tap of its frame, the input rows its band reads (zero rows and
+// columns stand for the spatial padding, so the inner loop has no bounds
+// checks).  Each thread then computes (pixel, 4 output channels) units from
+// shared memory, four input channels per float4 read.  Global memory is read
+// once per block and never in the reduction loop, which removes the load
+// latency chains that bound these calls.
+template <typename T>
+__device__ __forceinline__ void stage_f32(float* dst, const T* src, long long n, bool vec,
+                                          int tid, int nthreads);
+
+template <>
+__device__ __forceinline__ void stage_f32<float>(float* dst, const float* src, long long n,
+                                                 bool vec, int tid, int nthreads) {
+    if (vec) {  // n % 4 == 0, both 16-byte aligned
+        const float4* s4 = reinterpret_cast<const float4*>(src);
+        float4* d4 = reinterpret_cast<float4*>(dst);
+        for (long long i = tid; i < n / 4; i += nthreads) d4[i] = __ldg(s4 + i);
+    } else {
+        for (long long i = tid; i < n; i += nthreads) dst[i] = __ldg(src + i);
+    }
+}
+
+template <>
+__device__ __forceinline__ void stage_f32<__nv_bfloat16>(float* dst, const __nv_bfloat16* src,
+                                                         long long n, bool vec, int tid,
+                                                         int nthreads) {
+    if (vec) {  // n % 8 == 0, src 16-byte and dst 16-byte aligned
+        const uint4* s8 = reinterpret_cast<const uint4*>(src);
+        float4* d4 = reinterpret_cast<float4*>(dst);
+        for (long long i = tid; i < n / 8; i += nthreads) {
+            const uint4 v = __ldg(s8 + i);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // a bf16 is the high half of its fp32
+                f[2 * j] = __uint_as_float(u[j] << 16);
+                f[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+            }
+            d4[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+            d4[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    } else {
+        for (long long i = tid; i < n; i += nthreads) dst[i] = __bfloat162float(src[i]);
+    }
+}
+
+// Offset of the staged input rows after the weights (16-byte aligned), and
+// the kernel's dynamic shared memory, in floats.
+__host__ __device__ inline long long simt_band_offset(long long w_floats) {
+    return (w_floats + 3) / 4 * 4;
+}
+__host__ __device__ inline long long simt_smem_floats(long long w_floats, int kt, int rows_in,
+                                                      int Wp, int Cin) {
+    return simt_band_offset(w_floats) + (long long)kt * rows_in * Wp * Cin;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
+    if ((int)blockIdx.x >= p.conv_blocks) {
+        copy_new_cache(p.copy, blockIdx.x - p.conv_blocks, p.copy_blocks, threadIdx.x,
+                       blockDim.x);
+        return;
+    }
+    extern __shared__ __align__(16) float sm[];
+    float* wsm = sm;                      // [Cout][kt][kh][kw][Cin]
+    float* band = sm + simt_band_offset(p.w_floats);  // [kt][rows_in][Wp = W + 2 p_w][Cin]
+    const int tid = threadIdx.x, nth = blockDim.x;
+    const int frame = blockIdx.x / p.bands;
+    const int bnd = blockIdx.x - frame * p.bands;
+    const int o = frame % p.T_o, n = frame / p.T_o;
+    const int y0 = bnd * p.band_h;
+    const int V = sizeof(T) == 4 ? 4 : 8;  // elements per 16-byte load
+
+    // ---- stage the weights and, per active tap, the band's input rows
+    if (in_bounds(p.status, p.w, p.w_floats * (long long)sizeof(T), p.w,
+                  p.w_floats * (long long)sizeof(T)))
+        stage_f32<T>(wsm, static_cast<const T*>(p.w), p.w_floats, p.w_floats % V == 0, tid, nth);
+    const T* x = static_cast<const T*>(p.x);
+    const T* cache = static_cast<const T*>(p.cache);
+    const long long row_elems = (long long)p.W * p.Cin;
+    const bool row_vec = (row_elems % V == 0) && (p.Cin % 4 == 0);
+    for (int k = 0; k < p.taps.kt; ++k) {
+        if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
+        const int t = o * p.taps.s_t + p.taps.delta[k];
+        const T* fr = t < p.cache_len
+                          ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) *
+                                        p.H * row_elems
+                          : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * row_elems;
+        for (int i = 0; i < p.rows_in; ++i) {
+            float* drow = band + ((long long)k * p.rows_in + i) * p.Wp * p.Cin;
+            const int yi = y0 * p.s_h - p.p_h + i;
+            if (yi < 0 || yi >= p.H) {
+                for (long long e = tid; e < (long long)p.Wp * p.Cin; e += nth) drow[e] = 0.f;
+                continue;
+            }
+            for (long long e = tid; e < (long long)p.p_w * p.Cin; e += nth) {
+                drow[e] = 0.f;                                   // left padding
+                drow[(long long)(p.p_w + p.W) * p.Cin + e] = 0.f;  // right padding
+            }
+            const T* srow = fr + (long long)yi * row_elems;
+            if (in_bounds(p.status, srow, row_elems * (long long)sizeof(T),
+                          t < p.cache_len ? (const void*)cache : (const void*)x,
+                          t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
+                stage_f32<T>(drow + (long long)p.p_w * p.Cin, srow, row_elems, row_vec, tid, nth);
+        }
+    }
+    __syncthreads();
+
+    // ---- one (pixel, 4-channel group) unit per thread step
+    const int units = p.band_h * p.W_o * p.co_groups;
+    const long long w_co = (long long)p.taps.kt * p.kh * p.kw * p.Cin;
+    for (int u = tid; u < units; u += nth) {
+        const int cog = u % p.co_groups;
+        const int px = u / p.co_groups;
+        const int xo = px % p.W_o, yl = px / p.W_o;
+        const int yo = y0 + yl;
+        if (yo >= p.H_o) continue;
+        const int co0 = cog * kSimtCoT;
+        const float* wj[kSimtCoT];
+#pragma unroll
+        for (int j = 0; j < kSimtCoT; ++j)
+            wj[j] = wsm + (long long)min(co0 + j, p.Cout - 1) * w_co;  // rows past Cout unused
+        float acc[kSimtCoT] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < p.taps.kt; ++k) {
+            if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
+            for (int r = 0; r < p.kh; ++r) {
+                const float* zrow = band + ((long long)k * p.rows_in + yl * p.s_h + r * p.d_h) *
+                                               p.Wp * p.Cin;
+                for (int s = 0; s < p.kw; ++s) {
+                    const float* z = zrow + (long long)(xo * p.s_w + s * p.d_w) * p.Cin;
+                    const long long woff = (((long long)k * p.kh + r) * p.kw + s) * p.Cin;
+                    if (p.Cin % 4 == 0) {
+                        for (int ci = 0; ci < p.Cin; ci += 4) {
+                            const float4 z4 = *reinterpret_cast<const float4*>(z + ci);
+#pragma unroll
+                            for (int j = 0; j < kSimtCoT; ++j) {
+                                const float4 w4 =
+                                    *reinterpret_cast<const float4*>(wj[j] + woff + ci);
+                                acc[j] = fmaf(z4.x, w4.x, acc[j]);
+                                acc[j] = fmaf(z4.y, w4.y, acc[j]);
+                                acc[j] = fmaf(z4.z, w4.z, acc[j]);
+                                acc[j] = fmaf(z4.w, w4.w, acc[j]);
+                            }
+                        }
+                    } else {
+                        for (int ci = 0; ci < p.Cin; ++ci)
+#pragma unroll
+                            for (int j = 0; j < kSimtCoT; ++j)
+                                acc[j] = fmaf(z[ci], wj[j][woff + ci], acc[j]);
+                    }
+                }
+            }
+        }
+        const T* bias = static_cast<const T*>(p.bias);
+        const long long out_i = (((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo;
+        T* out = static_cast<T*>(p.out) + out_i * p.Cout;
+#pragma unroll
+        for (int j = 0; j < kSimtCoT; ++j) {
+            if (co0 + j >= p.Cout) break;
+            if (!index_ok(p.status, out_i * p.Cout + co0 + j, p.out_elems)) break;
+            float v = acc[j];
+            if (bias != nullptr) v += to_f32<T>(bias[co0 + j]);
+            out[co0 + j] = from_f32<T>(v);
+        }
     }
 }
 

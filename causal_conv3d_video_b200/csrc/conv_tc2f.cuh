@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 
 #include "cache_copy.cuh"
+#include "checked.cuh"
 #include "conv_tc.cuh"
 #include "conv_tc2h.cuh"
 #include "epilogue.cuh"
@@ -176,7 +177,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
     if (warp >= 2) {
         for (int i = threadIdx.x - 64; i < BN; i += 128) {
             float b = 0.f;
-            if (p.bias != nullptr && i < p.Cout)
+            if (p.bias != nullptr && i < p.Cout && index_ok(p.status, i, p.Cout))
                 b = __bfloat162float(__ushort_as_bfloat16(p.bias[i]));
             bias_s[i] = b;
         }
@@ -210,8 +211,11 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 if (leader) mbar_arrive_expect_tx(fb_local, strip_bytes + 2u * (uint32_t)wbytes_cta);
                 const uint32_t fb = pair_leader_addr(fb_local);
                 const CUtensorMap* map = t < p.cache_len ? &p.tmap_c : &p.tmap_x;
-                const int frame = t < p.cache_len ? n * p.cache_len + t
-                                                  : n * p.T_x + (t - p.cache_len);
+                int frame = t < p.cache_len ? ring_frame(n, t, p.cache_slots, p.cache_head)
+                                            : n * p.T_x + (t - p.cache_len);
+                // checked build: a frame outside the tensor map is recorded and
+                // clamped (the load still completes its barrier)
+                if (!index_ok(p.status, frame, t < p.cache_len ? p.c_frames : p.x_frames)) frame = 0;
                 tma_load_4d_pair(smem_u32(st_base), map, fb, cb * BK, xs,
                                  y_out * p.s_h + r * p.d_h - p.p_h, frame);
                 uint8_t* b_base = st_base + kAst;

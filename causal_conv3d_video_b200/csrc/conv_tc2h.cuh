@@ -114,7 +114,7 @@ conv_tc2h_kernel(const __grid_constant__ TcParams p) {
         for (int i = threadIdx.x - 64; i < BN; i += 128) {
             const int co = n_tile * BN + i;
             float b = 0.f;
-            if (p.bias != nullptr && co < p.Cout)
+            if (p.bias != nullptr && co < p.Cout && index_ok(p.status, co, p.Cout))
                 b = __bfloat162float(__ushort_as_bfloat16(p.bias[co]));
             bias_s[i] = b;
         }

@@ -155,8 +155,12 @@ __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t
     const int row = q * 32 + lane;
     const size_t slot_floats = (size_t)kTileM * BN;
     const int nblk = BN / kCh;
+    // checked build: extent of the partial tiles ([2G][128][BN] fp32)
+    const long long partial_bytes = (long long)2 * p.sk.G * kTileM * BN * 4;
     if (!owner) {
         float* mine = p.sk.partial + (size_t)(2 * g + rank) * slot_floats;
+        if (!in_bounds(p.status, mine, (long long)slot_floats * 4, p.sk.partial, partial_bytes))
+            ok = false;
         for (int b = 0; b < nblk; ++b) {
             uint32_t v[kCh];
 #pragma unroll
@@ -187,6 +191,9 @@ __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t
         const float* src = p.sk.partial + (size_t)(2 * (g + 1 + c) + rank) * slot_floats +
                            (size_t)b * (kTileM * kCh);
         const uint32_t bar = smem_u32(&fetch_bar[buf]);
+        // checked build: an out-of-range piece is recorded and fetched from
+        // the first slot instead (the fetch barrier still completes)
+        if (!in_bounds(p.status, src, kUnit, p.sk.partial, partial_bytes)) src = p.sk.partial;
         mbar_arrive_expect_tx(bar, kUnit);
         bulk_load_g2s(smem_u32(ring + (size_t)buf * kUnit), src, kUnit, bar);
     };
@@ -228,7 +235,9 @@ __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t
         }
         // staging buffer `slot`: its previous tensor store must have read it
         if (etid == 0) bulk_wait_group_read1();
-        epi_bar();  // also: every thread is done with this block's fetch buffers
+        // also: every thread is done with this block's fetch buffers; a fetch
+        // wait that ran out in any thread stops the refills in all of them
+        fetched = epi_bar_and(fetched);
         if (etid == 0 && fetched) {
             fence_proxy_async_smem();
             for (int r = u - ncon; r < u; ++r)
@@ -250,7 +259,7 @@ __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t
         }
         fence_proxy_async_smem();
         epi_bar();
-        if (etid == 0 && store && ok) {
+        if (etid == 0 && store && ok && index_ok(p.status, frame, (long long)p.N * p.T_o)) {
             tma_store_4d(&p.tmap_out, smem_u32(staging + slot * kBuf), co0 + b * kCh, x0, y0, frame);
             bulk_commit_group();
         }
@@ -472,13 +481,16 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
                                  p.wait_limit_ns))
                 ok = false;
             tc_fence_after();
+            // from here on `ok` decides counts and barrier phases (fetch units,
+            // fetch-buffer parities): make it uniform over the epilogue threads
+            ok = epi_bar_and(ok);
             const bool owner = sg.kb0 == 0;
             const bool whole = owner && sg.kb1 == sg.iters;
             if (owner && n_tile != bias_tile) {
                 epi_bar();  // the previous tile's epilogue is done with bias_s
                 for (int i = etid; i < BN; i += 128) {
                     const int co = n_tile * BN + i;
-                    bias_s[i] = (p.bias != nullptr && co < p.Cout)
+                    bias_s[i] = (p.bias != nullptr && co < p.Cout && index_ok(p.status, co, p.Cout))
                                     ? __bfloat162float(__ushort_as_bfloat16(__ldg(p.bias + co)))
                                     : 0.f;
                 }
@@ -489,18 +501,28 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             int g_last = g;
             if (owner && !whole) g_last = sk_owner_of(p, sg.tile_start + sg.iters - 1);
             if (owner && !whole && ok) {
-                // wait until every contributor of this CTA's rank has published
-                for (int gc = g + 1; gc <= g_last && ok; ++gc) {
-                    const unsigned* flag = p.sk.flags + 2 * gc + rank;
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(flag) != p.sk.epoch) {
-                        if (globaltimer_ns() - t0 > p.wait_limit_ns) {
-                            atomicCAS(p.status, 0, kStatusTimeout);
-                            ok = false;
+                // one thread waits until every contributor of this CTA's rank
+                // has published (its acquire orders the fetches it then
+                // issues); the outcome is shared by the barrier below
+                bool got = true;
+                if (etid == 0) {
+                    for (int gc = g + 1; gc <= g_last && got; ++gc) {
+                        if (!index_ok(p.status, 2 * gc + rank, 2LL * p.sk.G)) {
+                            got = false;
                             break;
+                        }
+                        const unsigned* flag = p.sk.flags + 2 * gc + rank;
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_gpu(flag) != p.sk.epoch) {
+                            if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+                                atomicCAS(p.status, 0, kStatusTimeout);
+                                got = false;
+                                break;
+                            }
                         }
                     }
                 }
+                ok = epi_bar_and(got);
             }
             const int fo = n * p.T_o + o;
             const int x0 = tx * p.box_w, y0 = ty * p.box_h, co0 = n_tile * BN;
@@ -516,7 +538,8 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             // replay of the same launch parameters (a captured graph, whose
             // epoch is fixed) waits for fresh pieces again.
             if (owner && !whole && ok && etid == 0)
-                for (int gc = g + 1; gc <= g_last; ++gc) p.sk.flags[2 * gc + rank] = 0u;
+                for (int gc = g + 1; gc <= g_last; ++gc)
+                    if (index_ok(p.status, 2 * gc + rank, 2LL * p.sk.G)) p.sk.flags[2 * gc + rank] = 0u;
             // TMEM buffer b is drained: hand it back to the MMA issuer
             tc_fence_before();
             __syncwarp();
@@ -530,7 +553,8 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
                 // publish this CTA's piece: stores visible before the flag
                 __threadfence();
                 epi_bar();  // all 128 epilogue threads (owner is uniform)
-                if (etid == 0 && ok) st_release_gpu(p.sk.flags + 2 * g + rank, p.sk.epoch);
+                if (etid == 0 && ok && index_ok(p.status, 2 * g + rank, 2LL * p.sk.G))
+                    st_release_gpu(p.sk.flags + 2 * g + rank, p.sk.epoch);
             }
             I = sg.tile_start + sg.kb1;
         }

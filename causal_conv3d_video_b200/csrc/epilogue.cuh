@@ -10,6 +10,7 @@
 #pragma once
 #include <cuda_bf16.h>
 
+#include "checked.cuh"
 #include "params.h"
 #include "ptx.cuh"
 
@@ -42,6 +43,21 @@ __device__ __forceinline__ void bulk_wait_group0() {
 // Named barrier over the four epilogue warps (barrier 1, 128 threads).
 __device__ __forceinline__ void epi_bar() {
     asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// The same barrier, returning the AND of `v` over the 128 epilogue threads,
+// so that decisions taken from bounded waits are uniform across them.
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
 }
 
 // 16-byte chunk c of row `row` inside a block of kRowB-byte rows, swizzled the
@@ -98,7 +114,7 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, uint32_t tmem_
     }
     fence_proxy_async_smem();  // generic-proxy writes -> visible to the TMA unit
     epi_bar();
-    if (etid == 0 && do_store) {
+    if (etid == 0 && do_store && index_ok(p.status, frame, (long long)p.N * p.T_o)) {
         for (int b = 0; b < nblk; ++b)
             tma_store_4d(&p.tmap_out, smem_u32(stage + (size_t)b * (kTileM * kRowB)),
                          co0 + b * kCh, x0, y0, frame);

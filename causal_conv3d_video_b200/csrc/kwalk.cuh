@@ -6,6 +6,7 @@
 // the thin signatures.  These helpers step the ring slot/phase and the
 // (tap, r, s, channel block) coordinates of the reduction incrementally.
 #pragma once
+#include "checked.cuh"
 #include "params.h"
 
 namespace ccv3d {
@@ -64,11 +65,14 @@ __device__ __forceinline__ TapSrc tap_source(const TcParams& p, int k, int n, in
     const int t = o * p.taps.s_t + p.taps.delta[k];
     if (t < p.cache_len) {
         ts.map = &p.tmap_c;
-        ts.frame = n * p.cache_len + t;
+        ts.frame = ring_frame(n, t, p.cache_slots, p.cache_head);
     } else {
         ts.map = &p.tmap_x;
         ts.frame = n * p.T_x + (t - p.cache_len);
     }
+    // checked build: a frame outside the tensor map is recorded and clamped
+    // (the load still completes its barrier, so the call ends promptly)
+    if (!index_ok(p.status, ts.frame, t < p.cache_len ? p.c_frames : p.x_frames)) ts.frame = 0;
     ts.wtap = k * p.kh * p.kw;
     return ts;
 }

@@ -12,13 +12,31 @@ constexpr int kSmCount = 148;        // B200 SMs (scheduling heuristics only)
 constexpr int kTcThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 
-// new_cache = last `keep` frames of Z = [cache; x], copied frame by frame.
+// Frame index, in a cache tensor of `slots` frames per batch entry, of cache
+// frame t (0 <= t < slots) of batch entry n, when frame 0 sits at slot `head`
+// (0 <= head < slots).  A dense cache has slots = |C| and head = 0; a ring
+// buffer wraps around its slots.
+__host__ __device__ __forceinline__ int ring_frame(int n, int t, int slots, int head) {
+    int s = head + t;
+    if (s >= slots) s -= slots;
+    return n * slots + s;
+}
+
+// The cache write of one call: the last `keep` frames of Z = [cache; x],
+// copied frame by frame, Z's frame z_len - keep + j to slot
+// (dst_head + j) mod dst_slots of dst.  Dense new_cache: dst_slots = keep,
+// dst_head = 0.  Ring buffer: only the arriving frames, into the slots that
+// follow the cached ones.
 struct CopyJob {
     const uint8_t* x;       // [N, T_x, frame_bytes]
-    const uint8_t* cache;   // [N, cache_len, frame_bytes]
-    uint8_t* dst;           // [N, keep, frame_bytes]
+    const uint8_t* cache;   // [N, cache_slots, frame_bytes], frame t at ring_frame(n, t, ...)
+    uint8_t* dst;           // [N, dst_slots, frame_bytes]
     long long frame_bytes;
     int keep, cache_len, T_x, z_len, N;
+    int cache_slots, cache_head;
+    int dst_slots, dst_head;
+    long long x_bytes, cache_bytes, dst_bytes;  // buffer extents (checked build)
+    int* status;                                // status word (checked build)
 };
 
 // Temporal bookkeeping of one call (paper, Sec. 4): tap k of output frame o
@@ -58,6 +76,7 @@ struct __align__(64) TcParams {
     int N, T_o, H_o, W_o, Cin, Cout, kh, kw;
     int s_h, s_w, p_h, p_w, d_h, d_w;
     int cache_len, T_x;
+    int cache_slots, cache_head;  // cache frame t of entry n: ring_frame(n, t, cache_slots, cache_head)
     int box_h, box_w, tiles_x, tiles_y, tiles_n;
     int BN, n_sub, n_cb, stages, tmem_cols;
     int pairs_per_frame;     // CTA-pair kernel: ceil(tiles_x * tiles_y / 2)
@@ -65,6 +84,7 @@ struct __align__(64) TcParams {
     int halo_w;              // halo kernel: pixels per input strip (128 + (kw-1)*d_w)
     StreamK sk;
     uint64_t wait_limit_ns;
+    int x_frames, c_frames;  // frames of the x and cache tensor maps (checked build)
 };
 
 struct SimtParams {
@@ -78,9 +98,17 @@ struct SimtParams {
     int N, T_o, H_o, W_o, Cin, Cout, H, W, kh, kw;
     int s_h, s_w, p_h, p_w, d_h, d_w;
     int cache_len, T_x;
+    int cache_slots, cache_head;
     int co_groups;
     long long conv_threads;  // N*T_o*H_o*W_o*co_groups
     int conv_blocks, copy_blocks;
+    // shared-memory kernel (small calls): bands of band_h output rows per
+    // frame, rows_in staged input rows per tap, staged rows padded to Wp
+    // pixels; w_floats = Cout*kt*kh*kw*Cin staged weights
+    int band_h, bands, rows_in, Wp;
+    long long w_floats;
+    long long out_elems;  // buffer extent (checked build; w's is w_floats)
+    int* status;          // status word: bounds violations of the checked build
 };
 
 }  // namespace ccv3d

@@ -93,9 +93,13 @@ C6_ST2_TIME = Conv("bf16_3x1x1_384ch_st2_180x320_c2_t4", 384, 384, 180, 320, T_x
 C6_ST2 = Conv("bf16_192ch_st2_180x320_c2_t4", 192, 192, 180, 320, T_x=4, cache_len=2,
               stride_t=2)
 
+# the decoder's RGB output conv (96 -> 3 channels at 720x1280, 4-frame chunks):
+# too thin in Cout for the tensor-core tiles, it runs on the FFMA path
+C_RGB = Conv("bf16_96to3_720x1280_c2_t4", 96, 3, 720, 1280, T_x=4, cache_len=2, sigma_b=0.1)
+
 WORKLOADS = {c.name: c for c in (
     C1, C2, C2_EMPTY, C3, C3B, C4_TIME, C4_DIL, C4_STRIDE, C4_C1, C4_ODD, C6_ST2_TIME,
-    C6_ST2)}
+    C6_ST2, C_RGB)}
 # cache-length sweep {0,1,2} on the bottleneck and on the stride-2 signature
 for _base in (C2, C4_STRIDE):
     for _c in (0, 1, 2):

@@ -60,7 +60,8 @@
 extern "C" {
 #endif
 
-#define CCV3D_ABI_VERSION 1
+#define CCV3D_ABI_VERSION 2 /* 2: ccv3d_stats.plans_unsupported, stream-scoped status
+                               reads, ring-buffer caches */
 #define CCV3D_MAX_KT 3 /* the contract's temporal kernel size */
 
 typedef enum { CCV3D_BF16 = 0, CCV3D_FP32 = 1 } ccv3d_dtype;
@@ -78,8 +79,12 @@ typedef enum {
                                    overlaps an input */
     CCV3D_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
     CCV3D_ERR_TIMEOUT = 7,      /* a bounded device-side wait ran out */
-    CCV3D_ERR_SCRATCH_LIMIT = 8 /* ccv3d_forward_noalloc: the call needs more
-                                   device scratch than its fixed array holds */
+    CCV3D_ERR_SCRATCH_LIMIT = 8, /* ccv3d_forward_noalloc: the call needs more
+                                    device scratch than its fixed array holds */
+    CCV3D_ERR_BOUNDS = 9         /* bounds-checked build (libccv3d_checked.so)
+                                    only: a kernel computed an address outside
+                                    the buffer it indexes; the access was
+                                    skipped and the output is not valid */
 } ccv3d_status;
 
 /* Conv3D call signature.  Sizes are in elements/frames. */
@@ -104,9 +109,14 @@ typedef struct {
     uint64_t calls;       /* successful ccv3d_forward calls */
     uint64_t tc_path;     /* of which ran the tcgen05 implicit-GEMM kernel */
     uint64_t simt_path;   /* of which ran the FP32 / thin-channel kernel */
-    uint64_t unsupported; /* forward calls refused as outside the contract */
+    uint64_t unsupported; /* forward calls of this plan refused with
+                             CCV3D_ERR_UNSUPPORTED (strict mode: no fallback) */
     uint64_t errors;      /* forward calls refused for any other reason */
-    uint64_t workspace_bytes; /* device scratch used per call (0) */
+    uint64_t workspace_bytes; /* device scratch the plan holds (0 unless the
+                                 persistent stream-K kernel runs it) */
+    uint64_t plans_unsupported; /* process-wide: ccv3d_plan calls refused with
+                                   CCV3D_ERR_UNSUPPORTED (no plan exists to
+                                   count them on) */
 } ccv3d_stats;
 
 typedef struct ccv3d_plan_s* ccv3d_plan_t;
@@ -116,7 +126,23 @@ typedef struct ccv3d_plan_s* ccv3d_plan_t;
  * plan's 256-byte device status block on the current device.  On a host with
  * no CUDA device the plan is still made, for inspection only (intervals,
  * sizes, path); ccv3d_forward then returns CCV3D_ERR_CUDA.  *out is set to
- * NULL on failure.  Errors: INVALID, UNSUPPORTED, EMPTY_OUTPUT, CUDA. */
+ * NULL on failure.  Errors: INVALID, UNSUPPORTED (also counted in
+ * ccv3d_stats.plans_unsupported), EMPTY_OUTPUT, CUDA.
+ *
+ * The kernel and tiling are the planner's own choice.  Environment variables
+ * CCV3D_PERSIST, CCV3D_HALO, CCV3D_FUSE, CCV3D_PAIR, CCV3D_TILE_N,
+ * CCV3D_STAGES, CCV3D_BOX_W, CCV3D_HALO_BK, CCV3D_SK_PAIRS, CCV3D_NO_ROT,
+ * CCV3D_SIMT_SMEM and CCV3D_FORCE_PATH=simt override it for tests and tuning
+ * sweeps, and are read only when CCV3D_TEST_OVERRIDES=1 is also set.
+ *
+ * The persistent stream-K kernel ("tc_persistent") launches one CTA pair per
+ * resident pair slot (the occupancy of an otherwise idle GPU, queried at plan
+ * time) and finishes split tiles from pieces other pairs publish, so it needs
+ * all of its pairs resident at once.  If other work on the GPU keeps some off
+ * the SMs for longer than the 2 s device wait limit, the waiting pairs give
+ * up: the call's output is incomplete and CCV3D_ERR_TIMEOUT is recorded in
+ * the status block (read it with ccv3d_get_status or
+ * ccv3d_get_status_stream).  The kernel never hangs. */
 CCV3D_API ccv3d_status ccv3d_plan(ccv3d_plan_t* out, const ccv3d_desc* desc);
 
 /* The planner's temporal bookkeeping, for inspection and testing.
@@ -140,7 +166,9 @@ CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
  *   "tc_persistent"  persistent stream-K over all SM pairs
  *   "tc_single"      one CTA per tile
  *   "simt"           FFMA, one thread per pixel and 4 output channels
- *   "simt_warp"      FFMA, one warp per pixel and 4 output channels (small calls) */
+ *   "simt_warp"      FFMA, one warp per pixel and 4 output channels (small calls)
+ *   "simt_smem"      FFMA, one block per band of output rows with the weights
+ *                    and input rows staged in shared memory (small calls that fit) */
 CCV3D_API const char* ccv3d_plan_kernel(ccv3d_plan_t plan);
 
 /* Reduction tiling of a tensor-core plan (inspection; no counterpart in the
@@ -163,6 +191,35 @@ CCV3D_API ccv3d_status ccv3d_forward(ccv3d_plan_t plan, const void* x, const voi
                            const int pad[2], const int dilation[3],
                            cudaStream_t stream);
 
+/* The same call with the cache kept in a ring buffer (the cache-augmented
+ * input Z = [C; X] of Sec. 4, with the cache state carried from chunk to
+ * chunk in place).  Instead of rewriting all K' = min(cache_keep, |Z|) frames
+ * of new_cache, a call writes only the frames of the new cache that arrive
+ * with it -- n_w = min(K', T_x) frames of x -- so a streaming decoder
+ * (T_x = 1, K' = 2) writes one frame per call instead of two.
+ *
+ *   ring  [N, ring_slots, H, W, Cin], device memory owned by the caller.
+ *         Cache frame t (0 <= t < |C|, |C| = the plan's cache_len) of batch
+ *         entry n is slot (head + t) mod ring_slots of entry n.  The call
+ *         writes the last n_w frames of x to slots (head + |C| + i) mod
+ *         ring_slots, i < n_w; no other slot changes.
+ *   next_head  (may be NULL) receives (head + |C| + n_w - K') mod ring_slots:
+ *         the head of the new cache, whose K' frames then sit at slots
+ *         (next_head + t) mod ring_slots -- pass it, with cache_len = K', to
+ *         the next call.
+ * Requirements: 0 <= head < ring_slots and ring_slots >= |C| + n_w (so no
+ * slot the call writes holds a frame it reads; ring_slots = cache_keep + T_x
+ * always suffices), ring 16-byte aligned and overlapping neither x, w nor
+ * out.  The first call of a stream uses a plan with cache_len = 0 and any
+ * head.  Outputs, kernels and numerics are those of ccv3d_forward (the same
+ * plan gives bit-identical out).  Errors: INVALID (as ccv3d_forward, or
+ * ring_slots / head out of range), ALIGNMENT, ALIAS, CUDA. */
+CCV3D_API ccv3d_status ccv3d_forward_ring(ccv3d_plan_t plan, const void* x, void* ring,
+                                          int ring_slots, int head, const void* w,
+                                          const void* bias, void* out, const int stride[2],
+                                          const int pad[2], const int dilation[3],
+                                          cudaStream_t stream, int* next_head);
+
 /* Counters since the plan was made (route counters of the paper's acceptance
  * criteria: fast-path hits, refusals). */
 CCV3D_API ccv3d_status ccv3d_get_stats(ccv3d_plan_t plan, ccv3d_stats* stats);
@@ -171,6 +228,13 @@ CCV3D_API ccv3d_status ccv3d_get_stats(ccv3d_plan_t plan, ccv3d_stats* stats);
  * plan's kernels: CCV3D_OK, or CCV3D_ERR_TIMEOUT after a bounded wait ran out.
  * CCV3D_ERR_CUDA when the device reports an error. */
 CCV3D_API ccv3d_status ccv3d_get_status(ccv3d_plan_t plan);
+
+/* As ccv3d_get_status, but ordered on `stream` only: waits for the work
+ * already queued on that stream (not the whole device), then returns and
+ * clears the status the plan's kernels recorded.  Calls of the plan on other
+ * streams are covered only once they have completed.  Allocates nothing.
+ * Errors: INVALID (NULL plan), CUDA. */
+CCV3D_API ccv3d_status ccv3d_get_status_stream(ccv3d_plan_t plan, cudaStream_t stream);
 
 /* Free the plan and its device status block.  NULL is ignored. */
 CCV3D_API void ccv3d_destroy(ccv3d_plan_t plan);
@@ -189,6 +253,15 @@ CCV3D_API ccv3d_status ccv3d_plan_sizes(ccv3d_plan_t plan, size_t* out_bytes,
  * reported it, and the context stays usable), CCV3D_OK if the wait completed
  * (a defect), or CCV3D_ERR_CUDA. */
 CCV3D_API ccv3d_status ccv3d_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+/* Self-test of the range checks: launches one thread that hands the device
+ * check one byte range ending past its buffer and one index past its count
+ * (neither is dereferenced).  Returns CCV3D_ERR_BOUNDS in the bounds-checked
+ * build (libccv3d_checked.so, compiled with -DCCV3D_CHECKED: every computed
+ * global address is checked before use and a violation is recorded, the
+ * access skipped), CCV3D_OK in the normal build, where the checks compile
+ * away; CCV3D_ERR_CUDA on a CUDA failure.  Allocates a 4-byte status word. */
+CCV3D_API ccv3d_status ccv3d_selftest_bounds(cudaStream_t stream);
 
 /* Post-decode uint8 quantisation of decoded frames, the step after the
  * decoder (FastVideo pull request "Quantize frames to uint8 on-device before
@@ -220,16 +293,23 @@ CCV3D_API ccv3d_status ccv3d_quantize_u8(const void* in, ccv3d_dtype dtype, void
  * It runs the persistent stream-K CTA-pair kernel.  That kernel's device
  * scratch -- a status word, the split-tile flags and the fp32 partial tiles --
  * lives in one static array of CCV3D_NOALLOC_SCRATCH_BYTES bytes compiled into
- * this library: every GPU that loads the library holds the array until the
- * process exits, whether or not it calls this function.  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture.
+ * this library: a GPU holds the array, from the moment the CUDA driver loads
+ * this library's device code on it, until the process exits.  Under the
+ * driver's lazy module loading (the default) that load can happen inside the
+ * first call of this function on a device -- the first call also looks up
+ * the array's device address (cudaGetSymbolAddress) with that device current
+ * -- so make one call (or one ccv3d_plan / ccv3d_forward) on each device
+ * before entering the context that may not allocate, and before any stream
+ * capture.
  *
  * All calls share the array and it keeps what the last call left there, so
  * calls that overlap on the GPU (other streams, other host threads) race:
- * the caller must order them.  Each call clears the status word before its
- * launch; the split-tile flags carry a per-device call number, so stale flags
- * from earlier calls are never mistaken for this call's.
+ * the caller must order them.  The split-tile flags carry a per-device call
+ * number, so stale flags from earlier calls are never mistaken for this
+ * call's.  A device-side wait that runs out (see the persistent kernel's
+ * co-residency note at ccv3d_plan) leaves that call's output incomplete and
+ * records CCV3D_ERR_TIMEOUT in the array's status word, which keeps the first
+ * such record until ccv3d_noalloc_get_status reads and clears it.
  *
  * Arguments and layouts are those of ccv3d_forward, with the signature in
  * `desc` instead of a plan.  Covered: bf16 signatures that run on the
@@ -237,15 +317,21 @@ CCV3D_API ccv3d_status ccv3d_quantize_u8(const void* in, ccv3d_dtype dtype, void
  * an active tap; others return CCV3D_ERR_UNSUPPORTED.  A call whose scratch
  * (2 x pairs x 128 x Cout-tile x 4 bytes, plus flags) would not fit returns
  * CCV3D_ERR_SCRATCH_LIMIT before any device work.  Other errors as
- * ccv3d_forward; a device-side wait that runs out is recorded in the shared
- * status word, which this entry point does not read back (it never
- * synchronises the host).  No device memory is allocated or freed. */
+ * ccv3d_forward.  This call never synchronises the host; no device memory is
+ * allocated or freed. */
 #define CCV3D_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 CCV3D_API ccv3d_status ccv3d_forward_noalloc(const ccv3d_desc* desc, const void* x,
                                              const void* cache, const void* w,
                                              const void* bias, void* out, void* new_cache,
                                              const int stride[2], const int pad[2],
                                              const int dilation[3], cudaStream_t stream);
+
+/* Status of the ccv3d_forward_noalloc calls on the current device: waits for
+ * the work queued on `stream`, then returns and clears the status word of the
+ * static array -- CCV3D_OK, or CCV3D_ERR_TIMEOUT when a call's bounded wait
+ * ran out since the last read.  Allocates nothing (the word is copied to
+ * pageable host memory).  Errors: CUDA. */
+CCV3D_API ccv3d_status ccv3d_noalloc_get_status(cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -36,10 +36,13 @@ def to_device(a, dtype):
 
 
 class plan_env:
-    """Temporarily set CCV3D_* planner overrides (read at plan time only)."""
+    """Temporarily set CCV3D_* planner overrides (read at plan time only, and
+    only with CCV3D_TEST_OVERRIDES=1, which this sets too)."""
 
     def __init__(self, env):
-        self.env = env
+        self.env = dict(env)
+        if self.env:
+            self.env["CCV3D_TEST_OVERRIDES"] = 1
 
     def __enter__(self):
         self.old = {k: os.environ.get(k) for k in self.env}

@@ -80,8 +80,9 @@ def test_planner_shapes_match_oracle_on_workloads(name):
     assert (iv["T_o"], iv["H_o"], iv["W_o"]) == (T_o, H_o, W_o)
     assert (iv["delta"], iv["o_l"], iv["o_h"]) == (delta, o_l, o_h)
     assert plan.sizes["new_cache_frames"] == keep
-    # bf16 workloads take the tensor-core path; fp32 the SIMT path
-    assert plan.path["tc"] == (c.dtype == "bf16")
+    # bf16 workloads with 16-multiple channels take the tensor-core path; fp32
+    # and the 3-channel RGB output conv the SIMT path
+    assert plan.path["tc"] == (c.dtype == "bf16" and c.Cin % 16 == 0 and c.Cout % 16 == 0)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -183,6 +184,7 @@ def test_kernel_choice(conv, kernel, monkeypatch):
     CCV3D_PERSIST=0/1 overrides."""
     monkeypatch.delenv("CCV3D_PERSIST", raising=False)
     assert ccv3d.Plan(ccv3d.desc_for(conv)).kernel == kernel
+    monkeypatch.setenv("CCV3D_TEST_OVERRIDES", "1")
     monkeypatch.setenv("CCV3D_PERSIST", "0")
     assert ccv3d.Plan(ccv3d.desc_for(conv)).kernel != "tc_persistent"
     monkeypatch.setenv("CCV3D_PERSIST", "1")
@@ -220,7 +222,13 @@ def test_quantize_validation_without_gpu():
 def test_simt_variant_choice():
     """Calls too small for one thread per (pixel, 4 channels) to fill the SMs
     run one warp per unit (the lanes split the reduction)."""
-    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_smem"
+    from parity_util import plan_env
+    with plan_env({"CCV3D_SIMT_SMEM": 0}):
+        assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
+    # weights of 384 -> 384 x 27 fp32 (15.9 MB) do not fit in shared memory
+    wide = workloads.Conv("f32_wide", 384, 384, 4, 4, T_x=1, cache_len=2, dtype="fp32")
+    assert ccv3d.Plan(ccv3d.desc_for(wide)).kernel == "simt_warp"
     big = workloads.Conv("f32_big", 32, 32, 64, 64, T_x=4, cache_len=2, dtype="fp32")
     assert ccv3d.Plan(ccv3d.desc_for(big)).kernel == "simt"
 
@@ -236,3 +244,76 @@ def test_plan_refuses_extents_past_32_bit_indexing(kw):
     with pytest.raises(ccv3d.CCV3DError) as e:
         ccv3d.Plan(ccv3d.make_desc(**base))
     assert e.value.status == ccv3d.CCV3D_ERR_UNSUPPORTED
+
+
+def test_overrides_need_the_test_gate(monkeypatch):
+    """Without CCV3D_TEST_OVERRIDES=1 the planner ignores every CCV3D_* override:
+    a deployment's environment cannot change the kernel or its tiling."""
+    monkeypatch.delenv("CCV3D_TEST_OVERRIDES", raising=False)
+    want = ccv3d.Plan(ccv3d.desc_for(workloads.C2))
+    assert want.kernel == "tc_pair"
+    for k, v in (("CCV3D_PERSIST", "1"), ("CCV3D_TILE_N", "128"), ("CCV3D_PAIR", "0"),
+                 ("CCV3D_STAGES", "2"), ("CCV3D_FORCE_PATH", "simt")):
+        monkeypatch.setenv(k, v)
+    plan = ccv3d.Plan(ccv3d.desc_for(workloads.C2))
+    assert plan.kernel == want.kernel and plan.path == want.path
+    assert plan.tiling == want.tiling
+    monkeypatch.setenv("CCV3D_TEST_OVERRIDES", "0")
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C2)).kernel == want.kernel
+    monkeypatch.setenv("CCV3D_TEST_OVERRIDES", "1")
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C2)).kernel == "simt"
+
+
+def test_unsupported_counted_apart_from_errors():
+    """Refused plans count in the process-wide plans_unsupported counter (there
+    is no plan to hold them); a plan's own counters keep errors apart."""
+    plan = ccv3d.Plan(ccv3d.make_desc(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2))
+    before = plan.stats()["plans_unsupported"]
+    for kw in (dict(kt=2), dict(groups=2), dict(kt=5)):
+        base = dict(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2)
+        base.update(kw)
+        with pytest.raises(ccv3d.CCV3DError) as e:
+            _plan(**base)
+        assert e.value.status == ccv3d.CCV3D_ERR_UNSUPPORTED
+    with pytest.raises(ccv3d.CCV3DError):
+        _plan(N=1, Cin=0, Cout=16, H=8, W=8, T_x=1, cache_len=2)   # INVALID: not counted
+    st = plan.stats()
+    assert st["plans_unsupported"] == before + 3
+    assert st["unsupported"] == 0 and st["errors"] == 0
+
+
+def test_ring_call_validation_without_gpu():
+    """ccv3d_forward_ring checks its ring arguments before any device work."""
+    plan = ccv3d.Plan(ccv3d.make_desc(N=1, Cin=16, Cout=16, H=8, W=8, T_x=1, cache_len=2))
+    A = 1 << 20
+    frame = 8 * 8 * 16 * 2
+
+    def call(ring=8 * A, slots=3, head=0, x=A, out=5 * A, w=3 * A, bias=4 * A):
+        return ccv3d.ccv3d_forward_ring(plan.handle, x, ring, slots, head, w, bias, out,
+                                        plan.stride, plan.pad, plan.dilation, stream=0,
+                                        check=False)[0]
+
+    assert call(slots=2) == ccv3d.CCV3D_ERR_INVALID       # |C| + 1 written > 2 slots
+    assert call(head=3) == ccv3d.CCV3D_ERR_INVALID        # head outside the ring
+    assert call(head=-1) == ccv3d.CCV3D_ERR_INVALID
+    assert call(ring=None) == ccv3d.CCV3D_ERR_INVALID
+    assert call(ring=8 * A + 8) == ccv3d.CCV3D_ERR_ALIGNMENT
+    assert call(ring=A + frame // 2) == ccv3d.CCV3D_ERR_ALIAS    # ring overlaps x
+    assert call(out=8 * A + frame) == ccv3d.CCV3D_ERR_ALIAS      # out inside the ring
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == ccv3d.CCV3D_ERR_CUDA
+    assert plan.stats()["calls"] == 0 and plan.stats()["errors"] >= 7
+
+
+def test_checked_build_exports_the_same_abi():
+    """libccv3d_checked.so (-DCCV3D_CHECKED) is the same ABI with every kernel
+    address range-checked; it exports every declared symbol too."""
+    from causal_conv3d_video_b200 import build
+    path = build.CHECKED_LIB_PATH
+    if not os.path.exists(path):
+        build.build(checked=True)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", path]).decode()
+    exported = set(re.findall(r"\bT (ccv3d_\w+)", out))
+    assert _declared_symbols() <= exported
+    assert "oracle" not in subprocess.check_output(["nm", "-D", path]).decode()

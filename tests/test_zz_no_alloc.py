@@ -13,7 +13,9 @@ import torch
 
 from causal_conv3d_video_b200 import ccv3d
 from causal_conv3d_video_b200.workloads import Conv
-from parity_util import TOL, inputs_for, plan_env, to_device
+import oracle
+from parity_util import (TOL, assert_close, inputs_for, oracle_params, plan_env,
+                         sample_indices, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -68,6 +70,14 @@ def _noalloc_vs_forward(c, desc, plan, call):
     assert _close(out, out_ref, c.dtype), (c.name, call)
     if nc is not None:
         assert torch.equal(nc, nc_ref)
+    # and against the FP64 oracle, at sampled outputs plus the tile edges
+    inp = inputs_for(c, stream_base=100 * call)
+    idx = sample_indices(tuple(out.shape), plan, n_random=1500)
+    ref = oracle.points(oracle_params(c), inp["x"], inp["cache"], inp["w"], inp["bias"], idx)
+    got = out[tuple(torch.from_numpy(idx.T).cuda())].double().cpu().numpy()
+    assert_close(got, ref, c.dtype, c.name)
+    # the status word of the static array: no bounded wait ran out
+    assert ccv3d.ccv3d_noalloc_get_status() == ccv3d.CCV3D_OK
 
 
 def test_noalloc_refuses_what_it_cannot_hold():
