@@ -34,6 +34,7 @@ __device__ __forceinline__ void copy_new_cache(const CopyJob& c, long long part,
         const long long lo = begin > f * per_frame ? begin - f * per_frame : 0;
         const long long hi = end < (f + 1) * per_frame ? end - f * per_frame : per_frame;
         const int n = (int)(f / c.keep), j = (int)(f % c.keep);
+        if ((c.paced_mask >> j) & 1u) continue;  // copied tile by tile with the GEMM
         const int t = c.z_len - c.keep + j;
         const uint8_t* src = z_frame(c, n, t);
         uint8_t* dst = c.dst + (long long)ring_frame(n, j, c.dst_slots, c.dst_head) * c.frame_bytes;
@@ -67,6 +68,53 @@ __device__ __forceinline__ void copy_new_cache(const CopyJob& c, long long part,
             unsigned short* d = reinterpret_cast<unsigned short*>(dst);
             for (long long v = lo + tid; v < hi; v += nthreads) d[v] = __ldg(s + v);
         }
+    }
+}
+
+// Copy the share of kept frame j of batch entry n that belongs to the output
+// box (tx, ty): input rows [ty*box_h*s_h, (ty+1)*box_h*s_h) and columns
+// [tx*box_w*s_w, (tx+1)*box_w*s_w), the last box row and column extended to
+// the frame's edge, so the boxes' shares partition the frame.  `nthreads`
+// threads, 16-byte vectors (frames of tensor-core calls have Cin % 16 == 0).
+__device__ __forceinline__ void copy_box_share(const CopyJob& c, int n, int j, int tx, int ty,
+                                               int tiles_x, int tiles_y, int box_w, int box_h,
+                                               int s_w, int s_h, int H, int W, int tid,
+                                               int nthreads) {
+    const int r0 = ty * box_h * s_h, c0 = tx * box_w * s_w;
+    const int r1 = ty + 1 == tiles_y ? H : min(H, (ty + 1) * box_h * s_h);
+    const int c1 = tx + 1 == tiles_x ? W : min(W, (tx + 1) * box_w * s_w);
+    if (r0 >= r1 || c0 >= c1) return;
+    const long long px_bytes = c.frame_bytes / ((long long)H * W);
+    const long long row_vecs = (long long)(c1 - c0) * px_bytes / 16;
+    const int t = c.z_len - c.keep + j;
+    const uint8_t* src = z_frame(c, n, t);
+    uint8_t* dst = c.dst + (long long)ring_frame(n, j, c.dst_slots, c.dst_head) * c.frame_bytes;
+    const long long first = ((long long)r0 * W + c0) * px_bytes;
+    const long long span = ((long long)(r1 - 1) * W + c1) * px_bytes - first;
+    if (!in_bounds(c.status, src + first, span, t < c.cache_len ? c.cache : c.x,
+                   t < c.cache_len ? c.cache_bytes : c.x_bytes) ||
+        !in_bounds(c.status, dst + first, span, c.dst, c.dst_bytes))
+        return;
+    const long long total = (long long)(r1 - r0) * row_vecs;
+    constexpr int kU = 4;
+    long long v = tid;
+    for (; v + (long long)(kU - 1) * nthreads < total; v += (long long)kU * nthreads) {
+        int4 r[kU];
+        long long off[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const long long e = v + (long long)u * nthreads;
+            const long long row = e / row_vecs;
+            off[u] = ((long long)(r0 + row) * W + c0) * px_bytes + (e - row * row_vecs) * 16;
+            r[u] = __ldg(reinterpret_cast<const int4*>(src + off[u]));
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) __stcs(reinterpret_cast<int4*>(dst + off[u]), r[u]);
+    }
+    for (; v < total; v += nthreads) {
+        const long long row = v / row_vecs;
+        const long long off = ((long long)(r0 + row) * W + c0) * px_bytes + (v - row * row_vecs) * 16;
+        __stcs(reinterpret_cast<int4*>(dst + off), __ldg(reinterpret_cast<const int4*>(src + off)));
     }
 }
 

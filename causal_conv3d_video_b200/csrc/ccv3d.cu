@@ -614,6 +614,34 @@ Taps make_taps(const ccv3d_plan_s* p) {
     return t;
 }
 
+// Paced new_cache copy of the persistent kernel: for each frame the call
+// keeps, the output frame and tap that read it (the last such tap) and that
+// tap's first k-block in the frame's tiles.  Frames no tap reads stay with
+// the sliced copy.  CCV3D_PACED=0 turns it off (tests and sweeps).
+void plan_paced_copy(const ccv3d_plan_s* p, TcParams& prm) {
+    prm.copy.paced_mask = 0u;
+    const int keep = prm.copy.keep;
+    if (!p->persist || keep <= 0 || keep > kMaxPaced) return;
+    if (override_env("CCV3D_PACED") != nullptr && env_int("CCV3D_PACED") == 0) return;
+    const ccv3d_desc& d = p->d;
+    const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
+    for (int j = 0; j < keep; ++j) {
+        const int t = p->z_len - keep + j;
+        for (int k = d.kt - 1; k >= 0; --k) {
+            const int rel = t - p->delta[k];
+            if (rel < 0 || rel % d.stride_t != 0) continue;
+            const int o = rel / d.stride_t;
+            if (o < p->o_l[k] || o >= p->o_h[k]) continue;
+            int ti = 0;  // position of tap k among frame o's active taps
+            for (int k2 = 0; k2 < k; ++k2) ti += (o >= p->o_l[k2] && o < p->o_h[k2]) ? 1 : 0;
+            prm.paced.o[j] = o;
+            prm.paced.kb[j] = ti * per_tap;
+            prm.copy.paced_mask |= 1u << j;
+            break;
+        }
+    }
+}
+
 template <int BK>
 cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s) {
     set_smem_attrs<BK>();
@@ -655,6 +683,8 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     prm.cache_slots = io.cache_slots; prm.cache_head = io.cache_head;
     prm.x_frames = d.N * d.T_x;
     prm.c_frames = d.N * io.cache_slots;
+    prm.H = d.H;
+    prm.W = d.W;
     prm.box_h = p->box_h; prm.box_w = p->box_w;
     prm.tiles_x = p->tiles_x; prm.tiles_y = p->tiles_y; prm.tiles_n = p->tiles_n;
     prm.BN = p->BN; prm.n_sub = p->n_sub; prm.n_cb = ceil_div(d.Cin, p->BK);
@@ -681,6 +711,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
         unsigned e = p->epoch.fetch_add(1) + 1;
         if (e == 0) e = p->epoch.fetch_add(1) + 1;  // 0 marks "never published"
         prm.sk.epoch = e;
+        plan_paced_copy(p, prm);
     }
     if (grid > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
     // spread the K-start offsets over one wave of concurrently running tiles

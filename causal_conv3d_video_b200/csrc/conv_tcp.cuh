@@ -268,6 +268,54 @@ __device__ __forceinline__ void tcp_segment_epilogue(const TcParams& p, uint32_t
     fetch_uses = use0 + (uint32_t)units;
 }
 
+// Named barrier over the four new_cache copy warps (barrier 2, 128 threads).
+__device__ __forceinline__ void copy_bar() {
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+// The paced share of the new_cache copy (frames of copy.paced_mask): walking
+// the pair's range like the producer, for every tile of Cout tile 0 whose
+// segment issues the first k-block of a tap that reads kept frame j, wait
+// (bounded) until the producer has issued that k-block, then copy this CTA's
+// box share of frame j.  The input lines the copy reads are then being
+// fetched into L2 for the GEMM's loads at the same time, so the frame
+// crosses from DRAM once instead of twice.  Called by the 128 copy threads.
+__device__ __forceinline__ void tcp_paced_copy(const TcParams& p, int rank, long long range0,
+                                               long long range1,
+                                               volatile long long* progress, int ctid) {
+    const CopyJob& c = p.copy;
+    bool pace = true;  // stop waiting after a wait ran out (the producer stopped)
+    for (long long I = range0; I < range1;) {
+        const Seg sg = sk_locate(p, I, range1);
+        I = sg.tile_start + sg.kb1;
+        if (sg.tile_in_frame % p.tiles_n != 0) continue;  // one Cout tile copies
+        const int o = sg.f % p.T_o, n = sg.f / p.T_o;
+        const int box = (sg.tile_in_frame / p.tiles_n) * 2 + rank;
+        if (box >= p.tiles_x * p.tiles_y) continue;
+        const int tx = box % p.tiles_x, ty = box / p.tiles_x;
+        for (int j = 0; j < c.keep && j < kMaxPaced; ++j) {
+            if (!((c.paced_mask >> j) & 1u) || p.paced.o[j] != o) continue;
+            const int kb = p.paced.kb[j];
+            if (kb < sg.kb0 || kb >= sg.kb1) continue;
+            if (pace && ctid == 0) {
+                const long long want = sg.tile_start + kb + 1;
+                const uint64_t t0 = globaltimer_ns();
+                while (*progress < want) {
+                    if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+                        atomicCAS(p.status, 0, kStatusTimeout);
+                        break;
+                    }
+                    __nanosleep(256);
+                }
+                if (*progress < want) pace = false;
+            }
+            copy_bar();
+            copy_box_share(c, n, j, tx, ty, p.tiles_x, p.tiles_y, p.box_w, p.box_h, p.s_w,
+                           p.s_h, p.H, p.W, ctid, 128);
+        }
+    }
+}
+
 // Two staging buffers of one output block (kCh channels x 128 rows, bf16).
 __host__ __device__ constexpr size_t tcp_staging_bytes(int bn) {
     return (size_t)2 * kTileM * out_block_channels(bn) * 2;
@@ -286,7 +334,8 @@ __host__ __device__ constexpr size_t tcp_smem_bytes(int bn, int stages) {
     // 2 x (acc full, acc empty) barriers, fetch barriers, TMEM address slot,
     // the Cout tile's bias
     return 1024 + tcp_ring_bytes<BK>(bn, stages) + tcp_staging_bytes(bn) +
-           (size_t)(2 * stages + 4 + kTcpFetchBufs) * 8 + 16 + (size_t)bn * 4;
+           (size_t)(2 * stages + 4 + kTcpFetchBufs) * 8 + 8 /* producer progress */ + 16 +
+           (size_t)bn * 4;
 }
 
 constexpr int kTcpThreads = 320;  // + warps 6-9: the new_cache copy
@@ -316,7 +365,10 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
     uint64_t* acc_full = empty_bar + stages;   // [2]
     uint64_t* acc_empty = acc_full + 2;        // [2], used in the even CTA
     uint64_t* fetch_bar = acc_empty + 2;       // [kTcpFetchBufs]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fetch_bar + kTcpFetchBufs);
+    // k-blocks of this pair's range the producer has issued (global index + 1)
+    volatile long long* progress = reinterpret_cast<volatile long long*>(fetch_bar + kTcpFetchBufs);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(
+        const_cast<long long*>(progress) + 1);
     float* bias_s = reinterpret_cast<float*>(tmem_slot + 4);
 
     const int warp = threadIdx.x >> 5;
@@ -336,6 +388,7 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
             mbar_init(smem_u32(&acc_empty[b]), 8);  // 4 epilogue warps x 2 CTAs
         }
         for (int b = 0; b < kTcpFetchBufs; ++b) mbar_init(smem_u32(&fetch_bar[b]), 1);
+        *progress = range0;
         fence_mbar_init();
         tma_prefetch_desc(&p.tmap_x);
         if (p.cache_len > 0) tma_prefetch_desc(&p.tmap_c);
@@ -396,6 +449,7 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
                                          w.cb * BK, wrow, nrow + j * BNs);
                     ring.next(stages);
                     ++issued;
+                    *progress = sg.tile_start + kb + 1;  // paces the new_cache copy
                     if (w.next(p) && kb + 1 < sg.kb1) ts = tap_source(p, act[w.ti], n, o);
                 }
                 I = sg.tile_start + sg.kb1;
@@ -448,8 +502,11 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
         }
         __syncwarp();
     } else if (warp >= 6) {
-        // ----------------- new_cache slice, beside the GEMM of this CTA
-        copy_new_cache(p.copy, blockIdx.x, gridDim.x, threadIdx.x - 192, 128);
+        // ----------------- new_cache, beside the GEMM of this CTA: frames no
+        // tap reads in equal slices, the others tile by tile with the loads
+        const int ctid = threadIdx.x - 192;
+        copy_new_cache(p.copy, blockIdx.x, gridDim.x, ctid, 128);
+        if (p.copy.paced_mask != 0u) tcp_paced_copy(p, (int)rank, range0, range1, progress, ctid);
     } else {
         // ------------------------------------------------- the epilogues
         const int etid = threadIdx.x - 64;

@@ -37,6 +37,19 @@ struct CopyJob {
     int dst_slots, dst_head;
     long long x_bytes, cache_bytes, dst_bytes;  // buffer extents (checked build)
     int* status;                                // status word (checked build)
+    unsigned paced_mask;  // bit j: frame j is copied tile by tile with the GEMM's loads
+};
+
+constexpr int kMaxPaced = 8;  // kept frames the paced copy can handle
+
+// Paced new_cache copy of the persistent kernel: kept frame j (Z's frame
+// z_len - keep + j) is read by output frame o[j] through the tap whose first
+// k-block in that frame's tiles is kb[j]; the CTA that issues that k-block
+// copies its box's share of the frame right after issuing it, while the same
+// input lines are being fetched into L2 for the GEMM.
+struct PacedCopy {
+    int o[kMaxPaced];
+    int kb[kMaxPaced];
 };
 
 // Temporal bookkeeping of one call (paper, Sec. 4): tap k of output frame o
@@ -85,6 +98,8 @@ struct __align__(64) TcParams {
     StreamK sk;
     uint64_t wait_limit_ns;
     int x_frames, c_frames;  // frames of the x and cache tensor maps (checked build)
+    PacedCopy paced;         // persistent kernel: frames of copy.paced_mask
+    int H, W;                // input frame extent (the paced copy's regions)
 };
 
 struct SimtParams {

@@ -328,3 +328,30 @@ def test_forward_refusals_on_device():
                              call.out, call.nc, p.stride, p.pad, p.dilation, check=False)
     assert rc == ccv3d.CCV3D_ERR_ALIGNMENT
     assert p.stats()["errors"] == 2 and p.stats()["calls"] == 0
+
+
+PACED = [
+    # kept frames read by a tap are copied tile by tile with the GEMM's loads
+    Conv("p64_c2", 64, 64, 20, 37, T_x=1, cache_len=2),
+    Conv("p64_c2_t3", 64, 64, 20, 37, T_x=3, cache_len=2),             # kept frames of o > 0
+    Conv("p64_dt2_c4", 64, 64, 18, 32, T_x=1, cache_len=4, dilation=(2, 1, 1)),  # 2 of 4 unread
+    Conv("p64_s2", 64, 64, 36, 64, T_x=1, cache_len=2, stride=(2, 2)),
+    Conv("p64_s2_odd", 32, 32, 17, 23, T_x=2, cache_len=1, stride=(2, 2)),  # edges extend
+    Conv("p64_st2", 64, 96, 12, 20, T_x=4, cache_len=2, stride_t=2),
+    Conv("p3x1x1", 384, 768, 10, 16, T_x=1, cache_len=2, kh=1, kw=1, pad=(0, 0)),  # 2 Cout tiles
+    Conv("p_batch2", 32, 48, 10, 12, T_x=2, cache_len=2, N=2),
+]
+
+
+@pytest.mark.parametrize("pairs", [0, 3])
+@pytest.mark.parametrize("paced", [1, 0], ids=["paced", "sliced"])
+@pytest.mark.parametrize("c", PACED, ids=lambda c: c.name)
+def test_persistent_new_cache_paced_or_sliced(c, paced, pairs):
+    """The persistent kernel's new_cache copy, paced with the producer (box
+    shares of the frames a tap reads) or in equal slices: out against the
+    oracle and new_cache exact either way, with whole or split tiles."""
+    env = {"CCV3D_PERSIST": 1, "CCV3D_PACED": paced}
+    if pairs:
+        env["CCV3D_SK_PAIRS"] = pairs
+    call, _ = _run_small(c, env=env)
+    assert call.plan.kernel == "tc_persistent"
