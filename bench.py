@@ -193,21 +193,34 @@ def run_gpu(args, rank, world, local_rank):
     plan = ccv3d.Plan(ccv3d.desc_for(conv))
     plan_us = (time.perf_counter() - t0) * 1e6
     flops, nbytes = algorithmic(conv, plan.intervals)
+    if args.ring:
+        nbytes = ring_algorithmic_bytes(conv, plan.intervals, nbytes)
+    slots = conv.cache_len + plan.ring_writes()
     dt = torch.bfloat16 if conv.dtype == "bf16" else torch.float32
 
     # independent operand sets, enough to exceed L2 between two uses of one set
     n_sets = max(2, int(np.ceil(2.0 * L2_BYTES / nbytes)) + 1)
     sets = []
+    heads = [0] * n_sets
     for i in range(n_sets):
         inp = synth.conv_inputs(**conv.synth_kwargs(), stream_base=16 * i)
         to = lambda a: None if a is None else torch.from_numpy(a).to(dt).to(dev)
         out, nc = plan.alloc_outputs(dev)
-        sets.append((to(inp["x"]), to(inp["cache"]), to(inp["w"]), to(inp["bias"]), out, nc))
+        cache = to(inp["cache"])
+        if args.ring:  # the cache frames in a ring of |C| + n_w slots
+            ring = torch.zeros((conv.N, slots, conv.H, conv.W, conv.Cin), dtype=dt, device=dev)
+            if cache is not None:
+                ring[:, :conv.cache_len] = cache
+            cache, nc = ring, None
+        sets.append((to(inp["x"]), cache, to(inp["w"]), to(inp["bias"]), out, nc))
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
         x, c, w, b, out, nc = sets[i % n_sets]
-        plan.forward(x, c, w, b, out, nc, stream)
+        if args.ring:
+            heads[i % n_sets] = plan.forward_ring(x, c, slots, heads[i % n_sets], w, b, out, stream)
+        else:
+            plan.forward(x, c, w, b, out, nc, stream)
 
     for i in range(args.warmup):
         step(i)
@@ -246,6 +259,8 @@ def run_gpu(args, rank, world, local_rank):
     # streaming decoder runs them: step i+1's upload and step i-1's download
     # overlap step i's compute (PCIe is full duplex).
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    if args.ring:
+        e2e_steps = 0  # the host-buffer legs run the dense call only
     w0, b0 = sets[0][2], sets[0][3]
     bufs = []
     for i in range(2):
@@ -300,66 +315,70 @@ def run_gpu(args, rank, world, local_rank):
             stream.wait_stream(s_down)
             end_ev.record(stream)
 
-    e2e_run(3)
-    torch.cuda.synchronize()
-    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        tdist.barrier()
-    torch.cuda.synchronize()
-    e2e_run(e2e_steps, ea, eb)
-    torch.cuda.synchronize()
-    e2e_ms = ea.elapsed_time(eb)
-
-    # Streaming decode: the cache stays on the device, each call's new_cache
-    # being the next call's cache (two device buffers, ping-pong); only the
-    # new frames go up and only the output comes back.  Needs a steady-state
-    # signature (new_cache the shape of the cache).
-    stream_ms = None
-    if c0 is not None and nc0 is not None and tuple(nc0.shape) == tuple(c0.shape):
-        caches = [bufs[0][1], bufs[1][1]]
-
-        def stream_run(steps, start_ev=None, end_ev=None):
-            uploaded, computed, freed = [None, None], [None, None], [None, None]
-            if start_ev is not None:
-                start_ev.record(stream)
-                s_up.wait_stream(stream)
-                s_down.wait_stream(stream)
-            for i in range(steps):
-                k = i % 2
-                x, _, out, _ = bufs[k]
-                with torch.cuda.stream(s_up):
-                    if computed[k] is not None:
-                        s_up.wait_event(computed[k])
-                    x.copy_(hx[k], non_blocking=True)
-                    uploaded[k] = ev()
-                    uploaded[k].record(s_up)
-                stream.wait_event(uploaded[k])
-                if freed[k] is not None:
-                    stream.wait_event(freed[k])
-                plan.forward(x, caches[i % 2], w0, b0, out, caches[(i + 1) % 2], stream)
-                computed[k] = ev()
-                computed[k].record(stream)
-                with torch.cuda.stream(s_down):
-                    s_down.wait_event(computed[k])
-                    ho[k].copy_(out, non_blocking=True)
-                    freed[k] = ev()
-                    freed[k].record(s_down)
-            if end_ev is not None:
-                stream.wait_stream(s_up)
-                stream.wait_stream(s_down)
-                end_ev.record(stream)
-
-        stream_run(3)
+    e2e_ms = stream_ms = None
+    if e2e_steps > 0:
+        e2e_run(3)
         torch.cuda.synchronize()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if dist:
             tdist.barrier()
         torch.cuda.synchronize()
-        stream_run(e2e_steps, ea, eb)
+        e2e_run(e2e_steps, ea, eb)
         torch.cuda.synchronize()
-        stream_ms = ea.elapsed_time(eb)
+        e2e_ms = ea.elapsed_time(eb)
+
+        # Streaming decode: the cache stays on the device, each call's new_cache
+        # being the next call's cache (two device buffers, ping-pong); only the
+        # new frames go up and only the output comes back.  Needs a steady-state
+        # signature (new_cache the shape of the cache).
+        stream_ms = None
+        if c0 is not None and nc0 is not None and tuple(nc0.shape) == tuple(c0.shape):
+            caches = [bufs[0][1], bufs[1][1]]
+
+            def stream_run(steps, start_ev=None, end_ev=None):
+                uploaded, computed, freed = [None, None], [None, None], [None, None]
+                if start_ev is not None:
+                    start_ev.record(stream)
+                    s_up.wait_stream(stream)
+                    s_down.wait_stream(stream)
+                for i in range(steps):
+                    k = i % 2
+                    x, _, out, _ = bufs[k]
+                    with torch.cuda.stream(s_up):
+                        if computed[k] is not None:
+                            s_up.wait_event(computed[k])
+                        x.copy_(hx[k], non_blocking=True)
+                        uploaded[k] = ev()
+                        uploaded[k].record(s_up)
+                    stream.wait_event(uploaded[k])
+                    if freed[k] is not None:
+                        stream.wait_event(freed[k])
+                    plan.forward(x, caches[i % 2], w0, b0, out, caches[(i + 1) % 2], stream)
+                    computed[k] = ev()
+                    computed[k].record(stream)
+                    with torch.cuda.stream(s_down):
+                        s_down.wait_event(computed[k])
+                        ho[k].copy_(out, non_blocking=True)
+                        freed[k] = ev()
+                        freed[k].record(s_down)
+                if end_ev is not None:
+                    stream.wait_stream(s_up)
+                    stream.wait_stream(s_down)
+                    end_ev.record(stream)
+
+            stream_run(3)
+            torch.cuda.synchronize()
+            if dist:
+                tdist.barrier()
+            torch.cuda.synchronize()
+            stream_run(e2e_steps, ea, eb)
+            torch.cuda.synchronize()
+            stream_ms = ea.elapsed_time(eb)
 
     if dist:
-        total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
+        total_ms = max_over_ranks([total_ms], dev)[0]
+        if e2e_ms is not None:
+            e2e_ms = max_over_ranks([e2e_ms], dev)[0]
         if stream_ms is not None:
             stream_ms = max_over_ranks([stream_ms], dev)[0]
 
@@ -370,7 +389,7 @@ def run_gpu(args, rank, world, local_rank):
     achieved = flops / avg_launch_s / 1e12
     peak = peaks["bf16_tflops"]
     value = job_throughput(flops, args.steps, total_ms, world)
-    e2e_value = job_throughput(flops, e2e_steps, e2e_ms, world)
+    e2e_value = job_throughput(flops, e2e_steps, e2e_ms, world) if e2e_ms else None
     csum = clocks.summary()
     line = {
         "metric": "cached causal Conv3D effective TFLOP/s (bf16), 1 GPU",
@@ -407,12 +426,12 @@ def run_gpu(args, rank, world, local_rank):
             "peak": peak,
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": traffic_from_profiles(conv.name),
+            "traffic": traffic_from_profiles(conv.name + ("+ring" if args.ring else "")),
             "peak_source": f"{peaks['source']} (bf16 burst)",
             "hbm_frac_of_measured": round(nbytes / avg_launch_s / 1e9 / peaks["hbm_gbs"], 4),
             "t_star_us": round(max(flops / (peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e6, 2),
         },
-        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+        "e2e": None if e2e_value is None else {"value": round(e2e_value, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "steps": e2e_steps,
                 "what": "per step: pinned host x+cache -> device, ccv3d_forward, "
@@ -995,6 +1014,9 @@ def main():
                     help="skip the 164-call synthetic decode sequence leg")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the per-workload legs")
+    ap.add_argument("--ring", action="store_true",
+                    help="time the headline workload with a ring-buffer cache "
+                         "(ccv3d_forward_ring) instead of ping-pong new_cache buffers")
     ap.add_argument("--sequence-passes", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -37,6 +37,26 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
 constexpr int kSimtThreads = 128;
 constexpr int kSimtCoT = 4;
 
+// The 16 bytes of one vector load as fp32 values (8 bf16 or 4 fp32).
+template <typename T>
+__device__ __forceinline__ void unpack16(uint4 v, float (&f)[16 / sizeof(T)]);
+template <>
+__device__ __forceinline__ void unpack16<float>(uint4 v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+}
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(uint4 v, float (&f)[8]) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // a bf16 is the high half of its fp32
+        f[2 * j] = __uint_as_float(u[j] << 16);
+        f[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 conv_simt_kernel(const __grid_constant__ SimtParams p) {
@@ -94,12 +114,32 @@ conv_simt_kernel(const __grid_constant__ SimtParams p) {
                              in_bounds(p.status, wrow + j * w_co_stride,
                                        (long long)p.Cin * sizeof(T), w,
                                        p.w_floats * (long long)sizeof(T));
-                for (int ci = 0; ci < p.Cin; ++ci) {
-                    const float z = to_f32<T>(zrow[ci]);
+                if (p.Cin % (16 / (int)sizeof(T)) == 0) {
+                    // 16-byte loads: 8 bf16 or 4 fp32 channels of the pixel and
+                    // of each weight row (both 16-byte aligned: their element
+                    // offsets are multiples of Cin)
+                    constexpr int V = 16 / sizeof(T);
+                    for (int ci = 0; ci < p.Cin; ci += V) {
+                        float z[V];
+                        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(zrow + ci)), z);
 #pragma unroll
-                    for (int j = 0; j < kSimtCoT; ++j)
-                        if (wok[j])
-                            acc[j] = fmaf(z, to_f32<T>(wrow[j * w_co_stride + ci]), acc[j]);
+                        for (int j = 0; j < kSimtCoT; ++j) {
+                            if (!wok[j]) continue;
+                            float wv[V];
+                            unpack16<T>(__ldg(reinterpret_cast<const uint4*>(
+                                            wrow + j * w_co_stride + ci)), wv);
+#pragma unroll
+                            for (int e = 0; e < V; ++e) acc[j] = fmaf(z[e], wv[e], acc[j]);
+                        }
+                    }
+                } else {
+                    for (int ci = 0; ci < p.Cin; ++ci) {
+                        const float z = to_f32<T>(zrow[ci]);
+#pragma unroll
+                        for (int j = 0; j < kSimtCoT; ++j)
+                            if (wok[j])
+                                acc[j] = fmaf(z, to_f32<T>(wrow[j * w_co_stride + ci]), acc[j]);
+                    }
                 }
             }
         }
