@@ -26,6 +26,7 @@
 #include "conv_tc.cuh"
 #include "conv_tc2.cuh"
 #include "conv_tc2f.cuh"
+#include "conv_tc2fp.cuh"
 #include "conv_tc2h.cuh"
 #include "conv_tcp.cuh"
 #include "params.h"
@@ -45,6 +46,7 @@ struct ccv3d_plan_s {
     int halo;     // 1: pair kernel loading each input row strip once per (tap, channel block)
     int halo_w;   // halo: pixels per strip
     int fused;    // 1: halo pair kernel computing two output frames per tile
+    int fused_persist;  // 1: the persistent form of the two-frame kernel (conv_tc2fp.cuh)
     int simt_kind;  // SIMT plans: 0 thread per unit, 1 warp per unit, 2 shared-memory blocks
     int simt_band_h, simt_rows_in, simt_threads;
     size_t simt_smem;
@@ -205,6 +207,8 @@ void set_smem_attrs() {
                              (int)(227 * 1024));
         cudaFuncSetAttribute(conv_tc2f_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
+        cudaFuncSetAttribute(conv_tc2fp_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
         cudaGetLastError();
     }
     done[dev].store(true, std::memory_order_release);
@@ -223,7 +227,7 @@ ResidentEntry g_resident[kResidentEntries];
 int g_resident_n = 0;
 
 template <int BK>
-int resident_pairs(size_t smem) {
+int resident_pairs(size_t smem, bool fused = false) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -232,7 +236,8 @@ int resident_pairs(size_t smem) {
     {
         std::lock_guard<std::mutex> lock(g_resident_mu);
         for (int i = 0; i < g_resident_n; ++i)
-            if (g_resident[i].dev == dev && g_resident[i].bk == BK && g_resident[i].smem == smem)
+            if (g_resident[i].dev == dev && g_resident[i].bk == (fused ? -BK : BK) &&
+                g_resident[i].smem == smem)
                 return g_resident[i].pairs;
     }
     set_smem_attrs<BK>();
@@ -241,12 +246,14 @@ int resident_pairs(size_t smem) {
     cfg.blockDim = dim3(kTcpThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, conv_tcp_kernel<BK>, &cfg) != cudaSuccess) {
+    const cudaError_t e = fused ? cudaOccupancyMaxActiveClusters(&n, conv_tc2fp_kernel<BK>, &cfg)
+                                : cudaOccupancyMaxActiveClusters(&n, conv_tcp_kernel<BK>, &cfg);
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
     std::lock_guard<std::mutex> lock(g_resident_mu);
-    if (g_resident_n < kResidentEntries) g_resident[g_resident_n++] = {dev, BK, n, smem};
+    if (g_resident_n < kResidentEntries) g_resident[g_resident_n++] = {dev, fused ? -BK : BK, n, smem};
     return n;
 }
 
@@ -303,6 +310,7 @@ bool setup_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->BK = bk;
     p->halo = 0;
     p->fused = 0;
+    p->fused_persist = 0;
     p->persist = 1;
     return true;
 }
@@ -391,6 +399,41 @@ void setup_fused(const ccv3d_desc& d, ccv3d_plan_s* p) {
     }
 }
 
+size_t fused_persist_smem_for(int bk, int bn, int stages, int kh, int kw, int halo_w) {
+    switch (bk) {
+        case 64: return tc2fp_smem_bytes<64>(bn, stages, kh, kw, halo_w);
+        case 32: return tc2fp_smem_bytes<32>(bn, stages, kh, kw, halo_w);
+        default: return tc2fp_smem_bytes<16>(bn, stages, kh, kw, halo_w);
+    }
+}
+
+// The persistent form of the two-frame kernel (conv_tc2fp.cuh): one CTA pair
+// per SM pair walks the tiles with a continuous ring and double-buffered TMEM
+// accumulators.  Sized for one CTA per SM: the widest channel block that
+// keeps at least four stages.  Opt-in (CCV3D_FUSED_PERSIST=1) until measured.
+void setup_fused_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    p->fused_persist = 0;
+    if (!p->fused || p->persist) return;
+    if (!(override_env("CCV3D_FUSED_PERSIST") != nullptr && env_int("CCV3D_FUSED_PERSIST") > 0))
+        return;
+    const int want_s = env_int("CCV3D_STAGES");
+    for (int min_s : {4, 2})
+        for (int bk : {64, 32, 16}) {
+            if (d.Cin % bk != 0) continue;
+            int s = want_s >= 2 ? want_s : 12;
+            while (s >= 2 && fused_persist_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w) > kSmemBudget)
+                --s;
+            if (s < min_s) continue;
+            p->fused_persist = 1;
+            p->BK = bk;
+            p->stages = s;
+            p->smem_bytes = fused_persist_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w);
+            p->tmem_cols = 32;
+            while (p->tmem_cols < 4 * p->BN) p->tmem_cols *= 2;  // two buffers of two frames
+            return;
+        }
+}
+
 // Whether the persistent stream-K kernel should replace one launch of pair
 // tiles (the plan as sized for that launch).  Measured over the decoder
 // signatures on B200, stream-K is 5-30% faster where
@@ -456,12 +499,30 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     const char* ps = override_env("CCV3D_PERSIST");
     const bool persist = ps != nullptr ? std::atoi(ps) > 0 : prefer_persistent(d, *p);
     if (persist && setup_persistent(d, p)) size_tc(d, p);
+    setup_fused_persistent(d, p);
     p->path_tc = 1;
 }
 
 // Persistent grid size: one CTA pair per resident pair slot, but at least 32
 // k-blocks per pair.  CCV3D_SK_PAIRS forces a size (tests of split tiles).
 void size_persistent(ccv3d_plan_s* p, bool have_device) {
+    if (p->fused_persist) {
+        // one CTA pair per resident pair slot, at most one per tile; no scratch
+        int pairs = 74;
+        if (have_device) {
+            int n = 0;
+            switch (p->BK) {
+                case 64: n = resident_pairs<64>(p->smem_bytes, true); break;
+                case 32: n = resident_pairs<32>(p->smem_bytes, true); break;
+                default: n = resident_pairs<16>(p->smem_bytes, true); break;
+            }
+            if (n > 0) pairs = n;
+        }
+        const long long tiles =
+            (long long)p->d.N * ((p->T_o + 1) / 2) * ((p->tiles_x * p->tiles_y + 1) / 2);
+        p->G = (int)std::max<long long>(1, std::min<long long>(pairs, tiles));
+        return;
+    }
     if (!p->persist) return;
     int pairs = 74;
     if (have_device) {
@@ -642,10 +703,34 @@ void plan_paced_copy(const ccv3d_plan_s* p, TcParams& prm) {
     }
 }
 
+// Paced new_cache copy of the persistent two-frame kernel: kept frame j is
+// copied box by box when the producer starts the tile of the output-frame
+// pair that reads it (all of a tile's stages run within one tile's time).
+void plan_paced_copy_fused(const ccv3d_plan_s* p, TcParams& prm) {
+    prm.copy.paced_mask = 0u;
+    const int keep = prm.copy.keep;
+    if (keep <= 0 || keep > kMaxPaced) return;
+    if (override_env("CCV3D_PACED") != nullptr && env_int("CCV3D_PACED") == 0) return;
+    const ccv3d_desc& d = p->d;
+    for (int j = 0; j < keep; ++j) {
+        const int t = p->z_len - keep + j;
+        for (int k = d.kt - 1; k >= 0; --k) {
+            const int o = t - p->delta[k];  // unit temporal stride and dilation here
+            if (o < p->o_l[k] || o >= p->o_h[k]) continue;
+            prm.paced.o[j] = o / 2;  // the output-frame pair holding o
+            prm.paced.kb[j] = 0;
+            prm.copy.paced_mask |= 1u << j;
+            break;
+        }
+    }
+}
+
 template <int BK>
 cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s) {
     set_smem_attrs<BK>();
-    if (kind == 4)
+    if (kind == 5)
+        conv_tc2fp_kernel<BK><<<grid, kTcpThreads, smem, s>>>(prm);
+    else if (kind == 4)
         conv_tc2f_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
     else if (kind == 3)
         conv_tc2h_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
@@ -696,6 +781,10 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
         p->pair ? 2LL * d.N * p->T_o * prm.pairs_per_frame * p->tiles_n
                 : (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
     if (p->fused) grid = 2LL * d.N * ((p->T_o + 1) / 2) * prm.pairs_per_frame;  // frame pairs
+    if (p->fused_persist) {
+        grid = 2LL * p->G;
+        plan_paced_copy_fused(p, prm);
+    }
     if (p->persist) {
         if (p->scratch == nullptr) return CCV3D_ERR_CUDA;
         grid = 2LL * p->G;
@@ -718,7 +807,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     const long long units = p->pair ? grid / 2 : grid;
     const long long wave = p->pair ? kSmCount / 2 : kSmCount;
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
-    const int kind = p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair));
+    const int kind = p->fused_persist ? 5 : (p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair)));
     prm.halo_w = p->halo_w;
     cudaError_t e;
     switch (p->BK) {
@@ -1022,6 +1111,7 @@ int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
 const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
     if (p == nullptr) return "";
     if (!p->path_tc) return p->simt_kind == 2 ? "simt_smem" : (p->simt_kind == 1 ? "simt_warp" : "simt");
+    if (p->fused_persist) return "tc_pair_fused_persistent";
     if (p->fused) return "tc_pair_fused";
     if (p->halo) return "tc_pair_halo";
     if (p->persist) return "tc_persistent";

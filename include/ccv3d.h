@@ -132,7 +132,8 @@ typedef struct ccv3d_plan_s* ccv3d_plan_t;
  * The kernel and tiling are the planner's own choice.  Environment variables
  * CCV3D_PERSIST, CCV3D_HALO, CCV3D_FUSE, CCV3D_PAIR, CCV3D_TILE_N,
  * CCV3D_STAGES, CCV3D_BOX_W, CCV3D_HALO_BK, CCV3D_SK_PAIRS, CCV3D_NO_ROT,
- * CCV3D_SIMT_SMEM and CCV3D_FORCE_PATH=simt override it for tests and tuning
+ * CCV3D_SIMT_SMEM, CCV3D_PACED, CCV3D_FUSED_PERSIST and CCV3D_FORCE_PATH=simt
+ * override it for tests and tuning
  * sweeps, and are read only when CCV3D_TEST_OVERRIDES=1 is also set.
  *
  * The persistent stream-K kernel ("tc_persistent") launches one CTA pair per
@@ -163,6 +164,8 @@ CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
  *   "tc_pair"        CTA-pair implicit GEMM (cta_group::2)
  *   "tc_pair_halo"   CTA pair, one input row strip per (tap, channel block)
  *   "tc_pair_fused"  CTA pair with row strips, two output frames per tile
+ *   "tc_pair_fused_persistent"  the same stages, one resident CTA pair per SM
+ *                    pair walking the tiles, double-buffered accumulators
  *   "tc_persistent"  persistent stream-K over all SM pairs
  *   "tc_single"      one CTA per tile
  *   "simt"           FFMA, one thread per pixel and 4 output channels

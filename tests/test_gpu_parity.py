@@ -355,3 +355,35 @@ def test_persistent_new_cache_paced_or_sliced(c, paced, pairs):
         env["CCV3D_SK_PAIRS"] = pairs
     call, _ = _run_small(c, env=env)
     assert call.plan.kernel == "tc_persistent"
+
+
+@pytest.mark.parametrize("paced", [1, 0], ids=["paced", "sliced"])
+@pytest.mark.parametrize("c", FUSED, ids=lambda c: c.name)
+def test_small_fused_persistent(c, paced):
+    """The persistent form of the two-frame kernel: the same stages, one CTA
+    pair per SM pair walking the tiles with double-buffered accumulators; with
+    a few pairs every pair runs many tiles, so both accumulator buffers and
+    both staging buffers cycle."""
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_FUSED_PERSIST": 1,
+                                 "CCV3D_PACED": paced})
+    assert call.plan.kernel == "tc_pair_fused_persistent", call.plan.kernel
+    first = call.out.clone()
+    call.run()
+    torch.cuda.synchronize()
+    assert torch.equal(first, call.out)
+    assert call.plan.status() == ccv3d.CCV3D_OK
+
+
+def test_full_size_fused_persistent_sampled():
+    """The 96-channel 720x1280 four-frame call on the persistent two-frame kernel."""
+    c = workloads.C3
+    inp = inputs_for(c)
+    call = GpuCall(c, inp, env={"CCV3D_FUSED_PERSIST": 1}).run()
+    torch.cuda.synchronize()
+    assert call.plan.kernel == "tc_pair_fused_persistent"
+    idx = sample_indices(tuple(call.out.shape), call.plan, n_random=2000)
+    ref = oracle.points(oracle_params(c), inp["x"], inp["cache"], inp["w"], inp["bias"], idx)
+    got = call.out[tuple(torch.from_numpy(idx.T).cuda())].double().cpu().numpy()
+    assert_close(got, ref, c.dtype, c.name)
+    assert np.array_equal(call.nc_f64(), expected_new_cache(c, inp))
+    assert call.guards_intact() and call.plan.status() == ccv3d.CCV3D_OK

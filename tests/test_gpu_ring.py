@@ -124,6 +124,8 @@ RING_SIGS = [
      {"CCV3D_HALO": 1, "CCV3D_PERSIST": 0, "CCV3D_FUSE": 0}),
     (Conv("r96_fused_t3", 96, 96, 3, 256, T_x=3, cache_len=0, sigma_b=0.1),
      {"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1}),
+    (Conv("r96_fused_persist_t3", 96, 96, 3, 256, T_x=3, cache_len=0, sigma_b=0.1),
+     {"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_FUSED_PERSIST": 1}),
     (Conv("r64_dt2", 64, 64, 18, 32, T_x=1, cache_len=0, dilation=(2, 1, 1)), {}),
     (Conv("r32_batch2_t2", 32, 48, 10, 12, T_x=2, cache_len=0, N=2), {}),
     (Conv("r16_fp32", 16, 16, 16, 16, T_x=3, cache_len=0, dtype="fp32", sigma_b=0.1), {}),
@@ -151,7 +153,10 @@ def test_ring_chunks_every_kernel(sig, env, extra):
         seen += c.T_x
     # the override that forces a kernel form (key, value) -> the form
     forced = {("CCV3D_PAIR", 0): "tc_single", ("CCV3D_HALO", 1): "tc_pair_halo",
-              ("CCV3D_FUSE", 1): "tc_pair_fused", ("CCV3D_PERSIST", 1): "tc_persistent"}
+              ("CCV3D_PERSIST", 1): "tc_persistent"}
+    if env.get("CCV3D_FUSE") == 1:
+        forced[("CCV3D_FUSE", 1)] = ("tc_pair_fused_persistent" if env.get("CCV3D_FUSED_PERSIST")
+                                     else "tc_pair_fused")
     for (k, v), name in forced.items():
         if env.get(k) == v:
             assert kernels == {name}, (sig.name, kernels)

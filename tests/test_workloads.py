@@ -102,3 +102,25 @@ def test_bench_algorithmic_flops_and_bytes(name):
     gf, mb = _TABLE[name]
     assert abs(flops / 1e9 - gf) <= 0.051 * max(1.0, gf / 100), (flops / 1e9, gf)
     assert abs(nbytes / 1e6 - mb) <= 0.6 + 0.001 * mb, (nbytes / 1e6, mb)
+
+
+def test_bench_ring_bytes_and_legs():
+    """A ring-buffer call writes only the arriving frames of the new cache:
+    on the stride-2 call (|C| = 2, T_x = 1, K' = 2) one 88.5 MB frame less
+    than the dense call.  The bench reports a leg for every configuration."""
+    import bench
+    c = workloads.C4_STRIDE
+    iv = {"T_o": 1, "H_o": 180, "W_o": 320, "o_l": [0, 0, 0], "o_h": [1, 1, 1]}
+    _, dense = bench.algorithmic(c, iv)
+    ring = bench.ring_algorithmic_bytes(c, iv, dense)
+    assert dense - ring == 2 * 360 * 640 * 192
+    c3 = workloads.C3  # T_x = 4 >= K' = 2: both kept frames arrive with the call
+    iv3 = {"T_o": 4, "H_o": 720, "W_o": 1280, "o_l": [0] * 3, "o_h": [4] * 3}
+    _, d3 = bench.algorithmic(c3, iv3)
+    assert bench.ring_algorithmic_bytes(c3, iv3, d3) == d3
+    names = {n for n, _, _ in bench.bench_legs()}
+    for w in (workloads.C1, workloads.C2, workloads.C2_EMPTY, workloads.C3, workloads.C3B,
+              workloads.C4_TIME, workloads.C4_DIL, workloads.C4_STRIDE, workloads.C4_C1,
+              workloads.C4_ODD, workloads.C6_ST2, workloads.C6_ST2_TIME, workloads.C_RGB):
+        assert w.name in names
+    assert workloads.C4_STRIDE.name + "+ring" in names
