@@ -95,26 +95,21 @@ __device__ __forceinline__ void copy_box_share(const CopyJob& c, int n, int j, i
                    t < c.cache_len ? c.cache_bytes : c.x_bytes) ||
         !in_bounds(c.status, dst + first, span, c.dst, c.dst_bytes))
         return;
-    const long long total = (long long)(r1 - r0) * row_vecs;
+    // warps take rows, lanes take 16-byte vectors of a row (no division)
+    const int warp = tid >> 5, lane = tid & 31, nwarps = nthreads >> 5;
     constexpr int kU = 4;
-    long long v = tid;
-    for (; v + (long long)(kU - 1) * nthreads < total; v += (long long)kU * nthreads) {
-        int4 r[kU];
-        long long off[kU];
+    for (int row = r0 + warp; row < r1; row += nwarps) {
+        const int4* s = reinterpret_cast<const int4*>(src + ((long long)row * W + c0) * px_bytes);
+        int4* d = reinterpret_cast<int4*>(dst + ((long long)row * W + c0) * px_bytes);
+        long long v = lane;
+        for (; v + (kU - 1) * 32 < row_vecs; v += kU * 32) {
+            int4 r[kU];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const long long e = v + (long long)u * nthreads;
-            const long long row = e / row_vecs;
-            off[u] = ((long long)(r0 + row) * W + c0) * px_bytes + (e - row * row_vecs) * 16;
-            r[u] = __ldg(reinterpret_cast<const int4*>(src + off[u]));
+            for (int u = 0; u < kU; ++u) r[u] = __ldg(s + v + u * 32);
+#pragma unroll
+            for (int u = 0; u < kU; ++u) __stcs(d + v + u * 32, r[u]);
         }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) __stcs(reinterpret_cast<int4*>(dst + off[u]), r[u]);
-    }
-    for (; v < total; v += nthreads) {
-        const long long row = v / row_vecs;
-        const long long off = ((long long)(r0 + row) * W + c0) * px_bytes + (v - row * row_vecs) * 16;
-        __stcs(reinterpret_cast<int4*>(dst + off), __ldg(reinterpret_cast<const int4*>(src + off)));
+        for (; v < row_vecs; v += 32) __stcs(d + v, __ldg(s + v));
     }
 }
 

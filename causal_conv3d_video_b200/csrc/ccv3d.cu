@@ -678,12 +678,18 @@ Taps make_taps(const ccv3d_plan_s* p) {
 // Paced new_cache copy of the persistent kernel: for each frame the call
 // keeps, the output frame and tap that read it (the last such tap) and that
 // tap's first k-block in the frame's tiles.  Frames no tap reads stay with
-// the sliced copy.  CCV3D_PACED=0 turns it off (tests and sweeps).
+// the sliced copy.  Opt-in (CCV3D_PACED=1): measured on the decoder calls it
+// was no faster than the sliced copy, which starts at once and overlaps the
+// whole GEMM, while the paced copy of the last tiles lengthens the kernel's
+// tail.
+bool paced_copy_on() {
+    return override_env("CCV3D_PACED") != nullptr && env_int("CCV3D_PACED") > 0;
+}
+
 void plan_paced_copy(const ccv3d_plan_s* p, TcParams& prm) {
     prm.copy.paced_mask = 0u;
     const int keep = prm.copy.keep;
-    if (!p->persist || keep <= 0 || keep > kMaxPaced) return;
-    if (override_env("CCV3D_PACED") != nullptr && env_int("CCV3D_PACED") == 0) return;
+    if (!p->persist || keep <= 0 || keep > kMaxPaced || !paced_copy_on()) return;
     const ccv3d_desc& d = p->d;
     const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
     for (int j = 0; j < keep; ++j) {
@@ -709,8 +715,7 @@ void plan_paced_copy(const ccv3d_plan_s* p, TcParams& prm) {
 void plan_paced_copy_fused(const ccv3d_plan_s* p, TcParams& prm) {
     prm.copy.paced_mask = 0u;
     const int keep = prm.copy.keep;
-    if (keep <= 0 || keep > kMaxPaced) return;
-    if (override_env("CCV3D_PACED") != nullptr && env_int("CCV3D_PACED") == 0) return;
+    if (keep <= 0 || keep > kMaxPaced || !paced_copy_on()) return;
     const ccv3d_desc& d = p->d;
     for (int j = 0; j < keep; ++j) {
         const int t = p->z_len - keep + j;

@@ -271,43 +271,36 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
 // shared memory, four input channels per float4 read.  Global memory is read
 // once per block and never in the reduction loop, which removes the load
 // latency chains that bound these calls.
+// Stage n values of T as fp32 into shared memory; with `vec` (n a multiple of
+// 16 / sizeof(T), both ends 16-byte aligned) by 16-byte loads, four in flight
+// per thread before their stores.
 template <typename T>
 __device__ __forceinline__ void stage_f32(float* dst, const T* src, long long n, bool vec,
-                                          int tid, int nthreads);
-
-template <>
-__device__ __forceinline__ void stage_f32<float>(float* dst, const float* src, long long n,
-                                                 bool vec, int tid, int nthreads) {
-    if (vec) {  // n % 4 == 0, both 16-byte aligned
-        const float4* s4 = reinterpret_cast<const float4*>(src);
-        float4* d4 = reinterpret_cast<float4*>(dst);
-        for (long long i = tid; i < n / 4; i += nthreads) d4[i] = __ldg(s4 + i);
-    } else {
-        for (long long i = tid; i < n; i += nthreads) dst[i] = __ldg(src + i);
-    }
-}
-
-template <>
-__device__ __forceinline__ void stage_f32<__nv_bfloat16>(float* dst, const __nv_bfloat16* src,
-                                                         long long n, bool vec, int tid,
-                                                         int nthreads) {
-    if (vec) {  // n % 8 == 0, src 16-byte and dst 16-byte aligned
-        const uint4* s8 = reinterpret_cast<const uint4*>(src);
-        float4* d4 = reinterpret_cast<float4*>(dst);
-        for (long long i = tid; i < n / 8; i += nthreads) {
-            const uint4 v = __ldg(s8 + i);
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-            float f[8];
+                                          int tid, int nthreads) {
+    constexpr int V = 16 / sizeof(T);
+    if (vec) {
+        const uint4* s = reinterpret_cast<const uint4*>(src);
+        const int nv = (int)(n / V);
+        constexpr int kU = 4;
+        for (int i0 = tid; i0 < nv; i0 += kU * nthreads) {
+            uint4 r[kU];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {  // a bf16 is the high half of its fp32
-                f[2 * j] = __uint_as_float(u[j] << 16);
-                f[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+            for (int u = 0; u < kU; ++u)
+                if (i0 + u * nthreads < nv) r[u] = __ldg(s + i0 + u * nthreads);
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int i = i0 + u * nthreads;
+                if (i >= nv) break;
+                float f[V];
+                unpack16<T>(r[u], f);
+#pragma unroll
+                for (int q = 0; q < V / 4; ++q)
+                    reinterpret_cast<float4*>(dst + (long long)i * V)[q] =
+                        make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
             }
-            d4[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
-            d4[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
         }
     } else {
-        for (long long i = tid; i < n; i += nthreads) dst[i] = __bfloat162float(src[i]);
+        for (long long i = tid; i < n; i += nthreads) dst[i] = to_f32<T>(src[i]);
     }
 }
 
@@ -345,31 +338,69 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
         stage_f32<T>(wsm, static_cast<const T*>(p.w), p.w_floats, p.w_floats % V == 0, tid, nth);
     const T* x = static_cast<const T*>(p.x);
     const T* cache = static_cast<const T*>(p.cache);
-    const long long row_elems = (long long)p.W * p.Cin;
+    const int row_elems = p.W * p.Cin;  // < 2^31: the rows fit in shared memory
+    const int Wp_elems = p.Wp * p.Cin;
+    int act[kMaxTaps], n_act = 0;
+    for (int k = 0; k < p.taps.kt; ++k)
+        if (o >= p.taps.o_l[k] && o < p.taps.o_h[k]) act[n_act++] = k;
+    // zeros: padding columns, and rows outside the frame
+    for (int e = tid; e < n_act * p.rows_in * Wp_elems; e += nth) {
+        const int ai = e / Wp_elems, c = e - ai * Wp_elems;
+        const int a = ai / p.rows_in, i = ai - a * p.rows_in;
+        const int yi = y0 * p.s_h - p.p_h + i;
+        if (yi < 0 || yi >= p.H || c < p.p_w * p.Cin || c >= (p.p_w + p.W) * p.Cin)
+            band[((long long)act[a] * p.rows_in + i) * Wp_elems + c] = 0.f;
+    }
+    // rows inside the frame: one pass over (active tap, row, 16-byte vector),
+    // four loads in flight per thread before their stores
     const bool row_vec = (row_elems % V == 0) && (p.Cin % 4 == 0);
-    for (int k = 0; k < p.taps.kt; ++k) {
-        if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
-        const int t = o * p.taps.s_t + p.taps.delta[k];
-        const T* fr = t < p.cache_len
-                          ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) *
-                                        p.H * row_elems
-                          : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * row_elems;
-        for (int i = 0; i < p.rows_in; ++i) {
-            float* drow = band + ((long long)k * p.rows_in + i) * p.Wp * p.Cin;
+    const int rv = row_vec ? row_elems / V : row_elems;  // units per row
+    const int total = n_act * p.rows_in * rv;
+    constexpr int kU = 4;
+    for (int e0 = tid; e0 < total; e0 += kU * nth) {
+        uint4 r[kU];
+        float* dst[kU];
+        bool live[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int e = e0 + u * nth;
+            live[u] = false;
+            if (e >= total) continue;
+            const int ai = e / rv, v = e - ai * rv;
+            const int a = ai / p.rows_in, i = ai - a * p.rows_in;
             const int yi = y0 * p.s_h - p.p_h + i;
-            if (yi < 0 || yi >= p.H) {
-                for (long long e = tid; e < (long long)p.Wp * p.Cin; e += nth) drow[e] = 0.f;
+            if (yi < 0 || yi >= p.H) continue;
+            const int t = o * p.taps.s_t + p.taps.delta[act[a]];
+            const T* fr = t < p.cache_len
+                              ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) *
+                                            p.H * row_elems
+                              : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * row_elems;
+            const T* sp = fr + (long long)yi * row_elems + (long long)v * (row_vec ? V : 1);
+            if (!in_bounds(p.status, sp, (row_vec ? 16 : (int)sizeof(T)),
+                           t < p.cache_len ? (const void*)cache : (const void*)x,
+                           t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
                 continue;
+            dst[u] = band + ((long long)act[a] * p.rows_in + i) * Wp_elems +
+                     (long long)p.p_w * p.Cin + (long long)v * (row_vec ? V : 1);
+            live[u] = true;
+            if (row_vec)
+                r[u] = __ldg(reinterpret_cast<const uint4*>(sp));
+            else
+                r[u].x = __float_as_uint(to_f32<T>(*sp));
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (!live[u]) continue;
+            if (row_vec) {
+                float f[V];
+                unpack16<T>(r[u], f);
+#pragma unroll
+                for (int q = 0; q < V / 4; ++q)
+                    reinterpret_cast<float4*>(dst[u])[q] =
+                        make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+            } else {
+                *dst[u] = __uint_as_float(r[u].x);
             }
-            for (long long e = tid; e < (long long)p.p_w * p.Cin; e += nth) {
-                drow[e] = 0.f;                                   // left padding
-                drow[(long long)(p.p_w + p.W) * p.Cin + e] = 0.f;  // right padding
-            }
-            const T* srow = fr + (long long)yi * row_elems;
-            if (in_bounds(p.status, srow, row_elems * (long long)sizeof(T),
-                          t < p.cache_len ? (const void*)cache : (const void*)x,
-                          t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
-                stage_f32<T>(drow + (long long)p.p_w * p.Cin, srow, row_elems, row_vec, tid, nth);
         }
     }
     __syncthreads();
