@@ -839,6 +839,19 @@ constexpr size_t kSimtSmemMax = 96 * 1024;
 void choose_simt(ccv3d_plan_s* p) {
     const ccv3d_desc& d = p->d;
     p->simt_kind = simt_uses_warps(*p) ? 1 : 0;
+    // large calls with <= 4 output channels: the tiled kernel (two blocks per SM)
+    const bool tile_off = override_env("CCV3D_SIMT_TILE") != nullptr && env_int("CCV3D_SIMT_TILE") == 0;
+    if (p->simt_kind == 0 && !tile_off && d.Cout <= 4 && d.Cin % kTileCc == 0 &&
+        d.stride_h == 1 && d.stride_w == 1 && d.dil_w == 1 && (d.kw == 1 || d.kw == 3)) {
+        const size_t bytes =
+            4 * (size_t)simt_tile_smem_floats(d.kt, d.kh, d.kw, d.Cin, d.dil_h, d.dil_w);
+        if (bytes <= 113 * 1024) {
+            p->simt_kind = 3;
+            p->simt_smem = bytes;
+            p->simt_threads = 256;
+            return;
+        }
+    }
     const bool smem_off = override_env("CCV3D_SIMT_SMEM") != nullptr && env_int("CCV3D_SIMT_SMEM") == 0;
     if (p->simt_kind != 1 || smem_off) return;
     const long long w_floats = (long long)d.Cout * d.kt * d.kh * d.kw * d.Cin;
@@ -871,8 +884,21 @@ void set_simt_smem_attr() {
     if (dev < 0 || dev >= kMaxDevices || done[dev].load(std::memory_order_acquire)) return;
     cudaFuncSetAttribute(conv_simt_smem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kSimtSmemMax);
+    cudaFuncSetAttribute(conv_simt_tile_kernel<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         113 * 1024);
+    cudaFuncSetAttribute(conv_simt_tile_kernel<T, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         113 * 1024);
     cudaGetLastError();
     done[dev].store(true, std::memory_order_release);
+}
+
+template <typename T>
+void launch_simt_tile(const SimtParams& prm, int kw, int grid, size_t smem, cudaStream_t s) {
+    set_simt_smem_attr<T>();
+    if (kw == 3)
+        conv_simt_tile_kernel<T, 3><<<grid, 256, smem, s>>>(prm);
+    else
+        conv_simt_tile_kernel<T, 1><<<grid, 256, smem, s>>>(prm);
 }
 
 ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const CacheIO& io, const void* w,
@@ -896,6 +922,21 @@ ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const CacheIO& io, const v
     prm.cache_len = d.cache_len; prm.T_x = d.T_x;
     prm.co_groups = ceil_div(d.Cout, kSimtCoT);
     prm.conv_threads = (long long)d.N * p->T_o * p->H_o * p->W_o * prm.co_groups;
+    if (p->simt_kind == 3) {
+        const long long cb = (long long)d.N * p->T_o * ceil_div(p->H_o, kTileRows) *
+                             ceil_div(p->W_o, kTileCols);
+        const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
+        const long long kb =
+            copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 65535) / 65536) : 0;
+        if (cb + kb > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
+        prm.conv_blocks = (int)cb;
+        prm.copy_blocks = (int)kb;
+        if (d.dtype == CCV3D_FP32)
+            launch_simt_tile<float>(prm, d.kw, (int)(cb + kb), p->simt_smem, stream);
+        else
+            launch_simt_tile<__nv_bfloat16>(prm, d.kw, (int)(cb + kb), p->simt_smem, stream);
+        return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+    }
     if (p->simt_kind == 2) {
         prm.band_h = p->simt_band_h;
         prm.bands = ceil_div(p->H_o, p->simt_band_h);
@@ -1115,7 +1156,10 @@ int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
 
 const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
     if (p == nullptr) return "";
-    if (!p->path_tc) return p->simt_kind == 2 ? "simt_smem" : (p->simt_kind == 1 ? "simt_warp" : "simt");
+    if (!p->path_tc)
+        return p->simt_kind == 3 ? "simt_tile"
+                                 : (p->simt_kind == 2 ? "simt_smem"
+                                                      : (p->simt_kind == 1 ? "simt_warp" : "simt"));
     if (p->fused_persist) return "tc_pair_fused_persistent";
     if (p->fused) return "tc_pair_fused";
     if (p->halo) return "tc_pair_halo";

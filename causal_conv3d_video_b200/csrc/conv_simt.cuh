@@ -464,4 +464,175 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
     }
 }
 
+// Large calls with at most 4 output channels (the decoder's RGB output conv,
+// 96 -> 3 channels at full resolution), unit spatial stride: every input
+// value feeds only Cout FMAs, so the kernel is bound by how often an input
+// value is read, not by the arithmetic.  A block of 256 threads owns 8 output
+// rows x 128 output columns of one frame; a thread owns 4 adjacent pixels of
+// one row and all (<= 4) output channels.
+//   * The weights are staged once per block as fp32, [k][r][s][ci][4 channels],
+//     so one broadcast float4 read gives all output channels of a tap.
+//   * Per (active tap, block of 8 input channels) the block stages the input
+//     patch the tile reads, (8 - 1 + (kh - 1) d_h + 1) rows x (128 + (kw - 1)
+//     d_w) columns, as fp32 in [channel quad][row][column][4] order (a thread
+//     loads 16 bytes of one pixel: 8 bf16 or 4 fp32 channels), zeros outside
+//     the frame; lanes then read consecutive 16-byte words.
+//   * A thread reads the 4 + KW - 1 patch columns of a kernel row once into
+//     registers and uses each for all KW column taps (KW = kw in {1, 3}, unit
+//     column dilation: compile-time window indices).
+constexpr int kTileRows = 8, kTileCols = 128, kTilePx = 4, kTileCc = 8;
+
+__host__ __device__ inline int simt_tile_rows_in(int kh, int d_h) {
+    return kTileRows - 1 + (kh - 1) * d_h + 1;
+}
+__host__ __device__ inline int simt_tile_cols_in(int kw, int d_w) {
+    return kTileCols + (kw - 1) * d_w;
+}
+// shared memory in floats: weights [kt*kh*kw*Cin][4] + one patch [2 quads][rows][cols][4]
+__host__ __device__ inline long long simt_tile_smem_floats(int kt, int kh, int kw, int Cin,
+                                                           int d_h, int d_w) {
+    return (long long)kt * kh * kw * Cin * 4 +
+           (long long)(kTileCc / 4) * simt_tile_rows_in(kh, d_h) * simt_tile_cols_in(kw, d_w) * 4;
+}
+
+template <typename T, int KW>
+__global__ void __launch_bounds__(256, 2)
+conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
+    if ((int)blockIdx.x >= p.conv_blocks) {
+        copy_new_cache(p.copy, blockIdx.x - p.conv_blocks, p.copy_blocks, threadIdx.x,
+                       blockDim.x);
+        return;
+    }
+    extern __shared__ __align__(16) float sm[];
+    const int taps2d = p.kh * p.kw;
+    float* wsm = sm;                                         // [kt*kh*kw*Cin][4]
+    float* patch = sm + (long long)p.taps.kt * taps2d * p.Cin * 4;
+    const int rows_in = simt_tile_rows_in(p.kh, p.d_h);
+    const int cols_in = simt_tile_cols_in(p.kw, p.d_w);
+    const int quad_stride = rows_in * cols_in * 4;           // floats per channel quad
+
+    const int tid = threadIdx.x;
+    const int tiles_x = (p.W_o + kTileCols - 1) / kTileCols;
+    const int tiles_y = (p.H_o + kTileRows - 1) / kTileRows;
+    const int tile = blockIdx.x % (tiles_x * tiles_y);
+    const int frame = blockIdx.x / (tiles_x * tiles_y);
+    const int o = frame % p.T_o, n = frame / p.T_o;
+    const int oy0 = (tile / tiles_x) * kTileRows, ox0 = (tile % tiles_x) * kTileCols;
+    const int iy0 = oy0 - p.p_h, ix0 = ox0 - p.p_w;          // patch origin in the frame (s = 1)
+
+    // ---- weights, once: [co][k][r][s][ci] -> [(k, r, s, ci)][co]
+    const T* w = static_cast<const T*>(p.w);
+    const int wk = p.taps.kt * taps2d * p.Cin;
+    for (int e = tid; e < wk * 4; e += blockDim.x) {
+        const int co = e / wk, rest = e - co * wk;
+        float v = 0.f;
+        if (co < p.Cout && in_bounds(p.status, w + (long long)co * wk + rest, sizeof(T), w,
+                                     p.w_floats * (long long)sizeof(T)))
+            v = to_f32<T>(w[(long long)co * wk + rest]);
+        wsm[rest * 4 + co] = v;
+    }
+
+    const int ty = tid >> 5, lane = tid & 31;                // output row ty, pixels 4 lane ..
+    float acc[kTilePx][4];
+#pragma unroll
+    for (int i = 0; i < kTilePx; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
+
+    const T* x = static_cast<const T*>(p.x);
+    const T* cache = static_cast<const T*>(p.cache);
+    const int V = 16 / (int)sizeof(T);                       // channels per 16-byte load
+    for (int k = 0; k < p.taps.kt; ++k) {
+        if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
+        const int t = o * p.taps.s_t + p.taps.delta[k];
+        const T* fr = t < p.cache_len
+                          ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) *
+                                        p.H * p.W * p.Cin
+                          : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * p.W * p.Cin;
+        const void* fbase = t < p.cache_len ? (const void*)cache : (const void*)x;
+        const long long fbytes = t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes;
+        for (int c0 = 0; c0 < p.Cin; c0 += kTileCc) {
+            __syncthreads();  // the previous patch is no longer read
+            // ---- stage the patch: one 16-byte load per (pixel, V channels)
+            const int loads_px = kTileCc / V;                // 1 (bf16) or 2 (fp32)
+            for (int e = tid; e < rows_in * cols_in * loads_px; e += blockDim.x) {
+                const int h = e % loads_px, pix = e / loads_px;
+                const int ry = pix / cols_in, rx = pix - ry * cols_in;
+                const int yi = iy0 + ry, xi = ix0 + rx;
+                float f[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) f[q] = 0.f;
+                if (yi >= 0 && yi < p.H && xi >= 0 && xi < p.W) {
+                    const T* sp = fr + ((long long)yi * p.W + xi) * p.Cin + c0 + h * V;
+                    if (in_bounds(p.status, sp, 16, fbase, fbytes)) {
+                        float g[16 / sizeof(T)];
+                        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(sp)), g);
+#pragma unroll
+                        for (int q = 0; q < (int)(16 / sizeof(T)); ++q) f[q] = g[q];
+                    }
+                }
+                // channel quads h*V/4 .. of this load
+#pragma unroll
+                for (int q = 0; q < 8 / 4; ++q) {
+                    const int quad = h * (V / 4) + q;
+                    if (q < V / 4)
+                        *reinterpret_cast<float4*>(patch + quad * quad_stride +
+                                                   (ry * cols_in + rx) * 4) =
+                            make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+                }
+            }
+            __syncthreads();
+            // ---- accumulate: kernel rows, channel quads, the register window
+            for (int r = 0; r < p.kh; ++r) {
+                const int prow = ty + r * p.d_h;
+#pragma unroll
+                for (int q = 0; q < kTileCc / 4; ++q) {
+                    float4 z[kTilePx + KW - 1];
+                    const float* zrow = patch + q * quad_stride + (prow * cols_in + lane * kTilePx) * 4;
+#pragma unroll
+                    for (int j = 0; j < kTilePx + KW - 1; ++j)
+                        z[j] = *reinterpret_cast<const float4*>(zrow + j * 4);
+#pragma unroll
+                    for (int sx = 0; sx < KW; ++sx) {
+                        const float* wq =
+                            wsm + ((((k * p.kh + r) * KW + sx) * p.Cin) + c0 + q * 4) * 4;
+                        const float4 w0 = *reinterpret_cast<const float4*>(wq);
+                        const float4 w1 = *reinterpret_cast<const float4*>(wq + 4);
+                        const float4 w2 = *reinterpret_cast<const float4*>(wq + 8);
+                        const float4 w3 = *reinterpret_cast<const float4*>(wq + 12);
+#pragma unroll
+                        for (int i = 0; i < kTilePx; ++i) {
+                            const float4 zz = z[i + sx];
+                            acc[i][0] = fmaf(zz.x, w0.x, fmaf(zz.y, w1.x, fmaf(zz.z, w2.x, fmaf(zz.w, w3.x, acc[i][0]))));
+                            acc[i][1] = fmaf(zz.x, w0.y, fmaf(zz.y, w1.y, fmaf(zz.z, w2.y, fmaf(zz.w, w3.y, acc[i][1]))));
+                            acc[i][2] = fmaf(zz.x, w0.z, fmaf(zz.y, w1.z, fmaf(zz.z, w2.z, fmaf(zz.w, w3.z, acc[i][2]))));
+                            acc[i][3] = fmaf(zz.x, w0.w, fmaf(zz.y, w1.w, fmaf(zz.z, w2.w, fmaf(zz.w, w3.w, acc[i][3]))));
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- bias once, round, store
+    const T* bias = static_cast<const T*>(p.bias);
+    const int yo = oy0 + ty;
+    if (yo >= p.H_o) return;
+#pragma unroll
+    for (int i = 0; i < kTilePx; ++i) {
+        const int xo = ox0 + lane * kTilePx + i;
+        if (xo >= p.W_o) break;
+        const long long out_i = (((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo;
+        T* out = static_cast<T*>(p.out) + out_i * p.Cout;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (c >= p.Cout) break;
+            if (!index_ok(p.status, out_i * p.Cout + c, p.out_elems)) break;
+            float v = acc[i][c];
+            if (bias != nullptr) v += to_f32<T>(bias[c]);
+            out[c] = from_f32<T>(v);
+        }
+    }
+}
+
 }  // namespace ccv3d

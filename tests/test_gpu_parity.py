@@ -387,3 +387,26 @@ def test_full_size_fused_persistent_sampled():
     assert_close(got, ref, c.dtype, c.name)
     assert np.array_equal(call.nc_f64(), expected_new_cache(c, inp))
     assert call.guards_intact() and call.plan.status() == ccv3d.CCV3D_OK
+
+
+SIMT_TILE = [
+    # large calls with <= 4 output channels: 8 x 128 output tiles, patches per
+    # 8 input channels (>= 148 x 128 (pixel, 4-channel) units each)
+    Conv("t16to3_45x150_t3", 16, 3, 45, 150, T_x=3, cache_len=2, sigma_b=0.1),     # ragged rows, cols
+    Conv("t32to4_40x160_c0", 32, 4, 40, 160, T_x=3, cache_len=0),
+    Conv("t8to1_48x130_c1", 8, 1, 48, 130, T_x=4, cache_len=1),
+    Conv("t16to2_3x1x1", 16, 2, 40, 200, T_x=3, cache_len=2, kh=1, kw=1, pad=(0, 0)),
+    Conv("t16to3_dilh2", 16, 3, 48, 140, T_x=3, cache_len=2, pad=(2, 1), dilation=(1, 2, 1)),
+    Conv("t16to3_st2", 16, 3, 40, 160, T_x=6, cache_len=2, stride_t=2),
+    Conv("t16to3_fp32", 16, 3, 49, 139, T_x=3, cache_len=2, dtype="fp32", sigma_b=0.1),
+    Conv("t8to4_fp32_3x1x1", 8, 4, 48, 150, T_x=3, cache_len=1, kh=1, kw=1, pad=(0, 0),
+         dtype="fp32"),
+]
+
+
+@pytest.mark.parametrize("tile", [1, 0], ids=["tile", "thread"])
+@pytest.mark.parametrize("c", SIMT_TILE, ids=lambda c: c.name)
+def test_simt_tile_thin_cout(c, tile):
+    call, _ = _run_small(c, env={"CCV3D_SIMT_TILE": tile})
+    assert call.plan.path["tc"] is False
+    assert call.plan.kernel == ("simt_tile" if tile else "simt"), call.plan.kernel
