@@ -814,6 +814,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
     const int kind = p->fused_persist ? 5 : (p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair)));
     prm.halo_w = p->halo_w;
+    prm.mma_interleave = env_int("CCV3D_MMA_INTERLEAVE") > 0 ? 1 : 0;
     cudaError_t e;
     switch (p->BK) {
         case 64: e = launch_tc<64>(prm, kind, (int)grid, p->smem_bytes, stream); break;
