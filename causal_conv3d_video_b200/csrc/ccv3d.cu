@@ -814,7 +814,6 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
     const int kind = p->fused_persist ? 5 : (p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair)));
     prm.halo_w = p->halo_w;
-    prm.mma_interleave = env_int("CCV3D_MMA_INTERLEAVE") > 0 ? 1 : 0;
     cudaError_t e;
     switch (p->BK) {
         case 64: e = launch_tc<64>(prm, kind, (int)grid, p->smem_bytes, stream); break;
@@ -855,13 +854,13 @@ void choose_simt(ccv3d_plan_s* p) {
     }
     const bool smem_off = override_env("CCV3D_SIMT_SMEM") != nullptr && env_int("CCV3D_SIMT_SMEM") == 0;
     if (p->simt_kind != 1 || smem_off) return;
-    const long long w_floats = (long long)d.Cout * d.kt * d.kh * d.kw * d.Cin;
     const int Wp = d.W + 2 * d.pad_w;
     const long long row_units = (long long)p->W_o * ceil_div(d.Cout, kSimtCoT);
     int bh = (int)std::max<long long>(1, std::min<long long>(p->H_o, 256 / std::max(1LL, row_units)));
     for (; bh >= 1; --bh) {
         const int rows_in = (bh - 1) * d.stride_h + (d.kh - 1) * d.dil_h + 1;
-        const size_t bytes = 4 * (size_t)simt_smem_floats(w_floats, d.kt, rows_in, Wp, d.Cin);
+        const size_t bytes =
+            4 * (size_t)simt_smem_floats(d.kt, d.kh, d.kw, d.Cin, d.Cout, rows_in, Wp);
         if (bytes <= kSimtSmemMax) {
             p->simt_kind = 2;
             p->simt_band_h = bh;

@@ -304,14 +304,17 @@ __device__ __forceinline__ void stage_f32(float* dst, const T* src, long long n,
     }
 }
 
-// Offset of the staged input rows after the weights (16-byte aligned), and
-// the kernel's dynamic shared memory, in floats.
-__host__ __device__ inline long long simt_band_offset(long long w_floats) {
-    return (w_floats + 3) / 4 * 4;
+// Shared-memory layout of the small-call kernel, in floats: the weights as
+// [(k, r, s, ci)][Cout rounded up to 4] (one float4 holds the 4 output
+// channels of a thread's unit), then the input rows as [tap][row][Wp][Cin + 4]
+// (the 4 pad floats per pixel put the pixels a warp reads in different banks).
+__host__ __device__ inline int simt_cout_pad(int Cout) { return (Cout + 3) / 4 * 4; }
+__host__ __device__ inline long long simt_band_offset(int kt, int kh, int kw, int Cin, int Cout) {
+    return (long long)kt * kh * kw * Cin * simt_cout_pad(Cout);
 }
-__host__ __device__ inline long long simt_smem_floats(long long w_floats, int kt, int rows_in,
-                                                      int Wp, int Cin) {
-    return simt_band_offset(w_floats) + (long long)kt * rows_in * Wp * Cin;
+__host__ __device__ inline long long simt_smem_floats(int kt, int kh, int kw, int Cin, int Cout,
+                                                      int rows_in, int Wp) {
+    return simt_band_offset(kt, kh, kw, Cin, Cout) + (long long)kt * rows_in * Wp * (Cin + 4);
 }
 
 template <typename T>
@@ -323,8 +326,11 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
         return;
     }
     extern __shared__ __align__(16) float sm[];
-    float* wsm = sm;                      // [Cout][kt][kh][kw][Cin]
-    float* band = sm + simt_band_offset(p.w_floats);  // [kt][rows_in][Wp = W + 2 p_w][Cin]
+    const int K = p.taps.kt * p.kh * p.kw * p.Cin;  // reduction length per output channel
+    const int CoP = simt_cout_pad(p.Cout), CinP = p.Cin + 4;
+    float* wsm = sm;                                 // [(k, r, s, ci)][CoP]
+    float* band = sm + simt_band_offset(p.taps.kt, p.kh, p.kw, p.Cin, p.Cout);
+                                                     // [kt][rows_in][Wp = W + 2 p_w][CinP]
     const int tid = threadIdx.x, nth = blockDim.x;
     const int frame = blockIdx.x / p.bands;
     const int bnd = blockIdx.x - frame * p.bands;
@@ -332,14 +338,36 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
     const int y0 = bnd * p.band_h;
     const int V = sizeof(T) == 4 ? 4 : 8;  // elements per 16-byte load
 
-    // ---- stage the weights and, per active tap, the band's input rows
-    if (in_bounds(p.status, p.w, p.w_floats * (long long)sizeof(T), p.w,
-                  p.w_floats * (long long)sizeof(T)))
-        stage_f32<T>(wsm, static_cast<const T*>(p.w), p.w_floats, p.w_floats % V == 0, tid, nth);
+    // ---- stage the weights, transposed to [(k, r, s, ci)][co] (four loads in
+    // flight per thread), zeros for the padded output channels
+    {
+        const T* w = static_cast<const T*>(p.w);
+        constexpr int kU = 4;
+        for (int e0 = tid; e0 < K * CoP; e0 += kU * nth) {
+            float r[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int e = e0 + u * nth;
+                r[u] = 0.f;
+                if (e >= K * CoP) continue;
+                const int co = e / K;  // e = co * K + (k, r, s, ci): w[e] when co < Cout
+                if (co < p.Cout && in_bounds(p.status, w + e, sizeof(T), w,
+                                             p.w_floats * (long long)sizeof(T)))
+                    r[u] = to_f32<T>(w[e]);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int e = e0 + u * nth;
+                if (e >= K * CoP) break;
+                const int co = e / K, ki = e - co * K;
+                wsm[ki * CoP + co] = r[u];
+            }
+        }
+    }
     const T* x = static_cast<const T*>(p.x);
     const T* cache = static_cast<const T*>(p.cache);
     const int row_elems = p.W * p.Cin;  // < 2^31: the rows fit in shared memory
-    const int Wp_elems = p.Wp * p.Cin;
+    const int Wp_elems = p.Wp * CinP;
     int act[kMaxTaps], n_act = 0;
     for (int k = 0; k < p.taps.kt; ++k)
         if (o >= p.taps.o_l[k] && o < p.taps.o_h[k]) act[n_act++] = k;
@@ -348,12 +376,13 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
         const int ai = e / Wp_elems, c = e - ai * Wp_elems;
         const int a = ai / p.rows_in, i = ai - a * p.rows_in;
         const int yi = y0 * p.s_h - p.p_h + i;
-        if (yi < 0 || yi >= p.H || c < p.p_w * p.Cin || c >= (p.p_w + p.W) * p.Cin)
+        if (yi < 0 || yi >= p.H || c < p.p_w * CinP || c >= (p.p_w + p.W) * CinP)
             band[((long long)act[a] * p.rows_in + i) * Wp_elems + c] = 0.f;
     }
     // rows inside the frame: one pass over (active tap, row, 16-byte vector),
-    // four loads in flight per thread before their stores
-    const bool row_vec = (row_elems % V == 0) && (p.Cin % 4 == 0);
+    // four loads in flight per thread before their stores (a vector never
+    // straddles two pixels: Cin is a multiple of its V channels)
+    const bool row_vec = p.Cin % V == 0;
     const int rv = row_vec ? row_elems / V : row_elems;  // units per row
     const int total = n_act * p.rows_in * rv;
     constexpr int kU = 4;
@@ -380,8 +409,10 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
                            t < p.cache_len ? (const void*)cache : (const void*)x,
                            t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
                 continue;
+            const int el = v * (row_vec ? V : 1);    // element of the row
+            const int px = el / p.Cin, c = el - px * p.Cin;
             dst[u] = band + ((long long)act[a] * p.rows_in + i) * Wp_elems +
-                     (long long)p.p_w * p.Cin + (long long)v * (row_vec ? V : 1);
+                     (long long)(p.p_w + px) * CinP + c;
             live[u] = true;
             if (row_vec)
                 r[u] = __ldg(reinterpret_cast<const uint4*>(sp));
@@ -407,7 +438,6 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
 
     // ---- one (pixel, 4-channel group) unit per thread step
     const int units = p.band_h * p.W_o * p.co_groups;
-    const long long w_co = (long long)p.taps.kt * p.kh * p.kw * p.Cin;
     for (int u = tid; u < units; u += nth) {
         const int cog = u % p.co_groups;
         const int px = u / p.co_groups;
@@ -415,37 +445,39 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
         const int yo = y0 + yl;
         if (yo >= p.H_o) continue;
         const int co0 = cog * kSimtCoT;
-        const float* wj[kSimtCoT];
-#pragma unroll
-        for (int j = 0; j < kSimtCoT; ++j)
-            wj[j] = wsm + (long long)min(co0 + j, p.Cout - 1) * w_co;  // rows past Cout unused
         float acc[kSimtCoT] = {0.f, 0.f, 0.f, 0.f};
         for (int k = 0; k < p.taps.kt; ++k) {
             if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
             for (int r = 0; r < p.kh; ++r) {
                 const float* zrow = band + ((long long)k * p.rows_in + yl * p.s_h + r * p.d_h) *
-                                               p.Wp * p.Cin;
+                                               Wp_elems;
                 for (int s = 0; s < p.kw; ++s) {
-                    const float* z = zrow + (long long)(xo * p.s_w + s * p.d_w) * p.Cin;
-                    const long long woff = (((long long)k * p.kh + r) * p.kw + s) * p.Cin;
+                    const float* z = zrow + (long long)(xo * p.s_w + s * p.d_w) * CinP;
+                    // this tap's weights: float4 of output channels co0..co0+3 per ci
+                    const float* wk = wsm + (long long)(((k * p.kh + r) * p.kw + s) * p.Cin) * CoP + co0;
                     if (p.Cin % 4 == 0) {
                         for (int ci = 0; ci < p.Cin; ci += 4) {
                             const float4 z4 = *reinterpret_cast<const float4*>(z + ci);
+                            const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
-                            for (int j = 0; j < kSimtCoT; ++j) {
+                            for (int e = 0; e < 4; ++e) {
                                 const float4 w4 =
-                                    *reinterpret_cast<const float4*>(wj[j] + woff + ci);
-                                acc[j] = fmaf(z4.x, w4.x, acc[j]);
-                                acc[j] = fmaf(z4.y, w4.y, acc[j]);
-                                acc[j] = fmaf(z4.z, w4.z, acc[j]);
-                                acc[j] = fmaf(z4.w, w4.w, acc[j]);
+                                    *reinterpret_cast<const float4*>(wk + (long long)(ci + e) * CoP);
+                                acc[0] = fmaf(zz[e], w4.x, acc[0]);
+                                acc[1] = fmaf(zz[e], w4.y, acc[1]);
+                                acc[2] = fmaf(zz[e], w4.z, acc[2]);
+                                acc[3] = fmaf(zz[e], w4.w, acc[3]);
                             }
                         }
                     } else {
-                        for (int ci = 0; ci < p.Cin; ++ci)
-#pragma unroll
-                            for (int j = 0; j < kSimtCoT; ++j)
-                                acc[j] = fmaf(z[ci], wj[j][woff + ci], acc[j]);
+                        for (int ci = 0; ci < p.Cin; ++ci) {
+                            const float4 w4 =
+                                *reinterpret_cast<const float4*>(wk + (long long)ci * CoP);
+                            acc[0] = fmaf(z[ci], w4.x, acc[0]);
+                            acc[1] = fmaf(z[ci], w4.y, acc[1]);
+                            acc[2] = fmaf(z[ci], w4.z, acc[2]);
+                            acc[3] = fmaf(z[ci], w4.w, acc[3]);
+                        }
                     }
                 }
             }

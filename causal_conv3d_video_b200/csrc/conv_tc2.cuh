@@ -167,23 +167,12 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
                 tc_fence_after();
                 const uint64_t a_desc = a0 + (uint64_t)((ring.st * kA) >> 4);
                 const uint64_t b_desc = b0 + (uint64_t)((ring.st * kBc) >> 4);
-                if (p.mma_interleave) {
-                    // the n_sub accumulators' MMAs alternate: independent
-                    // accumulation chains overlap in the tensor pipe
+                for (int j = 0; j < p.n_sub; ++j) {
+                    const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        for (int j = 0; j < p.n_sub; ++j)
-                            umma_bf16_pair(tmem_base + (uint32_t)(j * BNs), a_desc + 2u * kk,
-                                           b_desc + (uint64_t)((j * kBh) >> 4) + 2u * kk, idesc,
-                                           (it | kk) != 0 ? 1u : 0u);
-                } else {
-                    for (int j = 0; j < p.n_sub; ++j) {
-                        const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            umma_bf16_pair(tmem_base + (uint32_t)(j * BNs), a_desc + 2u * kk,
-                                           bj + 2u * kk, idesc, (it | kk) != 0 ? 1u : 0u);
-                    }
+                        umma_bf16_pair(tmem_base + (uint32_t)(j * BNs), a_desc + 2u * kk,
+                                       bj + 2u * kk, idesc, (it | kk) != 0 ? 1u : 0u);
                 }
                 umma_commit_pair(smem_u32(&empty_bar[ring.st]), (uint16_t)0x3);
                 ring.next(stages);

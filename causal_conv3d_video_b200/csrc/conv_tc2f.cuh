@@ -157,7 +157,13 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
         ty = box / p.tiles_x;
     }
     const FusedSrc src = fused_sources(p, o0);
-    const int iters = src.n * p.n_cb * p.kh;  // stages: (source frame, channel block, row r)
+    const int per_slot = p.n_cb * p.kh;       // stages of one source frame
+    const int iters = src.n * per_slot;       // stages: (source frame, channel block, row r)
+    // Each pair starts every source frame's (channel block, row) walk at its
+    // own offset, so pairs running at the same time read different weight
+    // tiles (the first stage of a slot is always the offset one, and it is
+    // the one that starts the slot's accumulator region when zero[] says so).
+    const int rot = (int)(((long long)pair * per_slot) / p.rot_div % per_slot);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -194,7 +200,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
             const int xs = tx * p.box_w - p.p_w;  // first pixel of the strip (s_w = 1)
             const int y_out = ty * p.box_h;
             Ring ring;
-            int si = 0, cb = 0, r = 0;
+            int si = 0, j = 0, cb = rot / p.kh, r = rot % p.kh;
             for (int it = 0; it < iters; ++it) {
                 if (it >= stages && !mbar_wait(smem_u32(&empty_bar[ring.st]), ring.ph ^ 1u,
                                                p.status, p.wait_limit_ns))
@@ -234,10 +240,13 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 ring.next(stages);
                 if (++r == p.kh) {
                     r = 0;
-                    if (++cb == p.n_cb) {
-                        cb = 0;
-                        ++si;
-                    }
+                    if (++cb == p.n_cb) cb = 0;
+                }
+                if (++j == per_slot) {  // next source frame, from the offset again
+                    j = 0;
+                    ++si;
+                    cb = rot / p.kh;
+                    r = rot % p.kh;
                 }
             }
         }
@@ -248,7 +257,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
             const uint32_t idesc_two = idesc_bf16_m256((uint32_t)(2 * BN));
             const uint64_t d0 = smem_desc_kmajor(smem_u32(smem), kRow);
             Ring ring;
-            int si = 0, cb = 0, r = 0;
+            int si = 0, j = 0;
             for (int it = 0; it < iters; ++it) {
                 if (!mbar_wait(smem_u32(&full_bar[ring.st]), ring.ph, p.status, p.wait_limit_ns))
                     break;
@@ -256,7 +265,7 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 const bool both = src.k0[si] >= 0 && src.k1[si] >= 0;
                 const uint32_t idesc = both ? idesc_two : idesc_one;
                 const uint32_t d_tmem = tmem_base + (src.k0[si] >= 0 ? 0u : (uint32_t)BN);
-                const bool zero = src.zero[si] && cb == 0 && r == 0;
+                const bool zero = src.zero[si] && j == 0;
                 const uint32_t st_off = (uint32_t)ring.st * (uint32_t)kStage;
                 for (int sx = 0; sx < p.kw; ++sx) {
                     // A: the strip shifted by sx*d_w pixels (rows)
@@ -270,12 +279,9 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 }
                 umma_commit_pair(smem_u32(&empty_bar[ring.st]), (uint16_t)0x3);
                 ring.next(stages);
-                if (++r == p.kh) {
-                    r = 0;
-                    if (++cb == p.n_cb) {
-                        cb = 0;
-                        ++si;
-                    }
+                if (++j == per_slot) {
+                    j = 0;
+                    ++si;
                 }
             }
             umma_commit_pair(smem_u32(acc_bar), (uint16_t)0x3);

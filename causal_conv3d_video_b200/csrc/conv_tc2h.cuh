@@ -178,15 +178,7 @@ conv_tc2h_kernel(const __grid_constant__ TcParams p) {
                         const uint64_t b_desc =
                             d0 + (uint64_t)((st_off + kAst + (r * p.kw + s) * kBc) >> 4);
                         const bool first = it == 0 && r == 0 && s == 0;
-                        if (p.mma_interleave) {
-#pragma unroll
-                            for (int kk = 0; kk < BK / 16; ++kk)
-                                for (int j = 0; j < p.n_sub; ++j)
-                                    umma_bf16_pair(tmem_base + (uint32_t)(j * BNs),
-                                                   a_desc + 2u * kk,
-                                                   b_desc + (uint64_t)((j * kBh) >> 4) + 2u * kk,
-                                                   idesc, (first && kk == 0) ? 0u : 1u);
-                        } else for (int j = 0; j < p.n_sub; ++j) {
+                        for (int j = 0; j < p.n_sub; ++j) {
                             const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < BK / 16; ++kk)

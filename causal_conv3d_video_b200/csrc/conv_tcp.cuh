@@ -486,21 +486,12 @@ conv_tcp_kernel(const __grid_constant__ TcParams p) {
                     const uint64_t a_desc = a0 + (uint64_t)((ring.st * kA) >> 4);
                     const uint64_t b_desc = b0 + (uint64_t)((ring.st * kBc) >> 4);
                     const uint32_t first = kb == sg.kb0 ? 1u : 0u;
-                    if (p.mma_interleave) {
+                    for (int j = 0; j < p.n_sub; ++j) {
+                        const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            for (int j = 0; j < p.n_sub; ++j)
-                                umma_bf16_pair(d_tmem + (uint32_t)(j * BNs), a_desc + 2u * kk,
-                                               b_desc + (uint64_t)((j * kBh) >> 4) + 2u * kk,
-                                               idesc, (first && kk == 0) ? 0u : 1u);
-                    } else {
-                        for (int j = 0; j < p.n_sub; ++j) {
-                            const uint64_t bj = b_desc + (uint64_t)((j * kBh) >> 4);
-#pragma unroll
-                            for (int kk = 0; kk < BK / 16; ++kk)
-                                umma_bf16_pair(d_tmem + (uint32_t)(j * BNs), a_desc + 2u * kk,
-                                               bj + 2u * kk, idesc, (first && kk == 0) ? 0u : 1u);
-                        }
+                            umma_bf16_pair(d_tmem + (uint32_t)(j * BNs), a_desc + 2u * kk,
+                                           bj + 2u * kk, idesc, (first && kk == 0) ? 0u : 1u);
                     }
                     umma_commit_pair(smem_u32(&empty_bar[ring.st]), (uint16_t)0x3);
                     ring.next(stages);

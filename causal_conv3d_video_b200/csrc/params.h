@@ -100,7 +100,6 @@ struct __align__(64) TcParams {
     int x_frames, c_frames;  // frames of the x and cache tensor maps (checked build)
     PacedCopy paced;         // persistent kernel: frames of copy.paced_mask
     int H, W;                // input frame extent (the paced copy's regions)
-    int mma_interleave;      // 1: issue the n_sub accumulators' MMAs alternately per K step
 };
 
 struct SimtParams {

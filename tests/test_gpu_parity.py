@@ -81,10 +81,7 @@ def test_config1_fp32_exact_workload(smem, kernel):
 
 
 KERNELS = {"persistent": {"CCV3D_PERSIST": 1}, "pair": {"CCV3D_PERSIST": 0},
-           "single": {"CCV3D_PAIR": 0, "CCV3D_PERSIST": 0},
-           # the n_sub accumulators' MMAs issued alternately per K step
-           "persistent_interleaved": {"CCV3D_PERSIST": 1, "CCV3D_MMA_INTERLEAVE": 1},
-           "pair_interleaved": {"CCV3D_PERSIST": 0, "CCV3D_MMA_INTERLEAVE": 1}}
+           "single": {"CCV3D_PAIR": 0, "CCV3D_PERSIST": 0}}
 
 
 @pytest.mark.parametrize("kernel", sorted(KERNELS))
@@ -131,12 +128,10 @@ HALO = [
 ]
 
 
-@pytest.mark.parametrize("inter", [0, 1], ids=["chained", "interleaved"])
 @pytest.mark.parametrize("halo", [1, 0], ids=["halo", "no_halo"])
 @pytest.mark.parametrize("c", HALO, ids=lambda c: c.name)
-def test_small_halo_strips(c, halo, inter):
-    call, _ = _run_small(c, env={"CCV3D_HALO": halo, "CCV3D_PERSIST": 0, "CCV3D_FUSE": 0,
-                                 "CCV3D_MMA_INTERLEAVE": inter})
+def test_small_halo_strips(c, halo):
+    call, _ = _run_small(c, env={"CCV3D_HALO": halo, "CCV3D_PERSIST": 0, "CCV3D_FUSE": 0})
     assert (call.plan.kernel == "tc_pair_halo") == bool(halo), call.plan.kernel
 
 
