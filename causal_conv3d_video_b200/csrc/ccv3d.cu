@@ -842,7 +842,8 @@ void choose_simt(ccv3d_plan_s* p) {
     // large calls with <= 4 output channels: the tiled kernel (two blocks per SM)
     const bool tile_off = override_env("CCV3D_SIMT_TILE") != nullptr && env_int("CCV3D_SIMT_TILE") == 0;
     if (p->simt_kind == 0 && !tile_off && d.Cout <= 4 && d.Cin % kTileCc == 0 &&
-        d.stride_h == 1 && d.stride_w == 1 && d.dil_w == 1 && (d.kw == 1 || d.kw == 3)) {
+        d.stride_h == 1 && d.stride_w == 1 && d.dil_w == 1 && (d.kw == 1 || d.kw == 3) &&
+        simt_tile_patch_loads(d.kh, d.kw, d.dil_h, d.dil_w, (int)elt(d)) <= kTilePf * 256) {
         const size_t bytes =
             4 * (size_t)simt_tile_smem_floats(d.kt, d.kh, d.kw, d.Cin, d.dil_h, d.dil_w);
         if (bytes <= 113 * 1024) {
@@ -857,6 +858,7 @@ void choose_simt(ccv3d_plan_s* p) {
     const int Wp = d.W + 2 * d.pad_w;
     const long long row_units = (long long)p->W_o * ceil_div(d.Cout, kSimtCoT);
     int bh = (int)std::max<long long>(1, std::min<long long>(p->H_o, 256 / std::max(1LL, row_units)));
+    if (env_int("CCV3D_SIMT_BAND") > 0) bh = std::min(p->H_o, env_int("CCV3D_SIMT_BAND"));
     for (; bh >= 1; --bh) {
         const int rows_in = (bh - 1) * d.stride_h + (d.kh - 1) * d.dil_h + 1;
         const size_t bytes =

@@ -456,6 +456,7 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
                     // this tap's weights: float4 of output channels co0..co0+3 per ci
                     const float* wk = wsm + (long long)(((k * p.kh + r) * p.kw + s) * p.Cin) * CoP + co0;
                     if (p.Cin % 4 == 0) {
+#pragma unroll 4
                         for (int ci = 0; ci < p.Cin; ci += 4) {
                             const float4 z4 = *reinterpret_cast<const float4*>(z + ci);
                             const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
@@ -513,12 +514,17 @@ conv_simt_smem_kernel(const __grid_constant__ SimtParams p) {
 //     registers and uses each for all KW column taps (KW = kw in {1, 3}, unit
 //     column dilation: compile-time window indices).
 constexpr int kTileRows = 8, kTileCols = 128, kTilePx = 4, kTileCc = 8;
+constexpr int kTilePf = 8;  // 16-byte loads of the next patch a thread holds (x 256 threads)
 
 __host__ __device__ inline int simt_tile_rows_in(int kh, int d_h) {
     return kTileRows - 1 + (kh - 1) * d_h + 1;
 }
 __host__ __device__ inline int simt_tile_cols_in(int kw, int d_w) {
     return kTileCols + (kw - 1) * d_w;
+}
+// 16-byte loads of one patch (element size `esize`): must not exceed kTilePf x 256
+__host__ __device__ inline int simt_tile_patch_loads(int kh, int kw, int d_h, int d_w, int esize) {
+    return simt_tile_rows_in(kh, d_h) * simt_tile_cols_in(kw, d_w) * (kTileCc * esize / 16);
 }
 // shared memory in floats: weights [kt*kh*kw*Cin][4] + one patch [2 quads][rows][cols][4]
 __host__ __device__ inline long long simt_tile_smem_floats(int kt, int kh, int kw, int Cin,
@@ -552,16 +558,29 @@ conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
     const int oy0 = (tile / tiles_x) * kTileRows, ox0 = (tile % tiles_x) * kTileCols;
     const int iy0 = oy0 - p.p_h, ix0 = ox0 - p.p_w;          // patch origin in the frame (s = 1)
 
-    // ---- weights, once: [co][k][r][s][ci] -> [(k, r, s, ci)][co]
+    // ---- weights, once: [co][k][r][s][ci] -> [(k, r, s, ci)][co], four
+    // loads in flight per thread
     const T* w = static_cast<const T*>(p.w);
     const int wk = p.taps.kt * taps2d * p.Cin;
-    for (int e = tid; e < wk * 4; e += blockDim.x) {
-        const int co = e / wk, rest = e - co * wk;
-        float v = 0.f;
-        if (co < p.Cout && in_bounds(p.status, w + (long long)co * wk + rest, sizeof(T), w,
-                                     p.w_floats * (long long)sizeof(T)))
-            v = to_f32<T>(w[(long long)co * wk + rest]);
-        wsm[rest * 4 + co] = v;
+    for (int e0 = tid; e0 < wk * 4; e0 += 4 * (int)blockDim.x) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u * (int)blockDim.x;
+            v[u] = 0.f;
+            if (e >= wk * 4) continue;
+            const int co = e / wk, rest = e - co * wk;
+            if (co < p.Cout && in_bounds(p.status, w + (long long)co * wk + rest, sizeof(T), w,
+                                         p.w_floats * (long long)sizeof(T)))
+                v[u] = to_f32<T>(w[(long long)co * wk + rest]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u * (int)blockDim.x;
+            if (e >= wk * 4) break;
+            const int co = e / wk, rest = e - co * wk;
+            wsm[rest * 4 + co] = v[u];
+        }
     }
 
     const int ty = tid >> 5, lane = tid & 31;                // output row ty, pixels 4 lane ..
@@ -571,11 +590,22 @@ conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
 
+    // ---- steps (active tap, block of 8 channels); each thread holds its
+    // share of the next step's patch (<= kTilePf 16-byte loads, checked by the
+    // planner) in registers while the current step's FMAs run
     const T* x = static_cast<const T*>(p.x);
     const T* cache = static_cast<const T*>(p.cache);
-    const int V = 16 / (int)sizeof(T);                       // channels per 16-byte load
-    for (int k = 0; k < p.taps.kt; ++k) {
-        if (!(o >= p.taps.o_l[k] && o < p.taps.o_h[k])) continue;
+    constexpr int V = 16 / (int)sizeof(T);                   // channels per 16-byte load
+    constexpr int loads_px = kTileCc / V;                    // 1 (bf16) or 2 (fp32)
+    const int nload = rows_in * cols_in * loads_px;
+    int act[kMaxTaps], n_act = 0;
+    for (int k = 0; k < p.taps.kt; ++k)
+        if (o >= p.taps.o_l[k] && o < p.taps.o_h[k]) act[n_act++] = k;
+    const int chunks = p.Cin / kTileCc;
+    const int steps = n_act * chunks;
+    uint4 pf[kTilePf];
+    auto fetch = [&](int step) {
+        const int k = act[step / chunks], c0 = (step % chunks) * kTileCc;
         const int t = o * p.taps.s_t + p.taps.delta[k];
         const T* fr = t < p.cache_len
                           ? cache + (long long)ring_frame(n, t, p.cache_slots, p.cache_head) *
@@ -583,63 +613,64 @@ conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
                           : x + ((long long)n * p.T_x + (t - p.cache_len)) * p.H * p.W * p.Cin;
         const void* fbase = t < p.cache_len ? (const void*)cache : (const void*)x;
         const long long fbytes = t < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes;
-        for (int c0 = 0; c0 < p.Cin; c0 += kTileCc) {
-            __syncthreads();  // the previous patch is no longer read
-            // ---- stage the patch: one 16-byte load per (pixel, V channels)
-            const int loads_px = kTileCc / V;                // 1 (bf16) or 2 (fp32)
-            for (int e = tid; e < rows_in * cols_in * loads_px; e += blockDim.x) {
-                const int h = e % loads_px, pix = e / loads_px;
-                const int ry = pix / cols_in, rx = pix - ry * cols_in;
-                const int yi = iy0 + ry, xi = ix0 + rx;
-                float f[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) f[q] = 0.f;
-                if (yi >= 0 && yi < p.H && xi >= 0 && xi < p.W) {
-                    const T* sp = fr + ((long long)yi * p.W + xi) * p.Cin + c0 + h * V;
-                    if (in_bounds(p.status, sp, 16, fbase, fbytes)) {
-                        float g[16 / sizeof(T)];
-                        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(sp)), g);
+        for (int i = 0; i < kTilePf; ++i) {
+            pf[i] = make_uint4(0u, 0u, 0u, 0u);  // zeros outside the frame
+            const int e = tid + i * (int)blockDim.x;
+            if (e >= nload) continue;
+            const int h = e % loads_px, pix = e / loads_px;
+            const int ry = pix / cols_in, rx = pix - ry * cols_in;
+            const int yi = iy0 + ry, xi = ix0 + rx;
+            if (yi < 0 || yi >= p.H || xi < 0 || xi >= p.W) continue;
+            const T* sp = fr + ((long long)yi * p.W + xi) * p.Cin + c0 + h * V;
+            if (in_bounds(p.status, sp, 16, fbase, fbytes))
+                pf[i] = __ldg(reinterpret_cast<const uint4*>(sp));
+        }
+    };
+    fetch(0);
+    for (int step = 0; step < steps; ++step) {
+        const int k = act[step / chunks], c0 = (step % chunks) * kTileCc;
+        __syncthreads();  // the previous step's patch is no longer read
+        // ---- the held loads into the patch, [channel quad][row][column][4]
 #pragma unroll
-                        for (int q = 0; q < (int)(16 / sizeof(T)); ++q) f[q] = g[q];
-                    }
-                }
-                // channel quads h*V/4 .. of this load
+        for (int i = 0; i < kTilePf; ++i) {
+            const int e = tid + i * (int)blockDim.x;
+            if (e >= nload) break;
+            const int h = e % loads_px, pix = e / loads_px;
+            float g[V];
+            unpack16<T>(pf[i], g);
 #pragma unroll
-                for (int q = 0; q < 8 / 4; ++q) {
-                    const int quad = h * (V / 4) + q;
-                    if (q < V / 4)
-                        *reinterpret_cast<float4*>(patch + quad * quad_stride +
-                                                   (ry * cols_in + rx) * 4) =
-                            make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
-                }
-            }
-            __syncthreads();
-            // ---- accumulate: kernel rows, channel quads, the register window
-            for (int r = 0; r < p.kh; ++r) {
-                const int prow = ty + r * p.d_h;
+            for (int q = 0; q < V / 4; ++q)
+                *reinterpret_cast<float4*>(patch + (h * (V / 4) + q) * quad_stride + pix * 4) =
+                    make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
+        }
+        __syncthreads();
+        if (step + 1 < steps) fetch(step + 1);  // in flight during the FMAs below
+        // ---- accumulate: kernel rows, channel quads, the register window
+        for (int r = 0; r < p.kh; ++r) {
+            const int prow = ty + r * p.d_h;
 #pragma unroll
-                for (int q = 0; q < kTileCc / 4; ++q) {
-                    float4 z[kTilePx + KW - 1];
-                    const float* zrow = patch + q * quad_stride + (prow * cols_in + lane * kTilePx) * 4;
+            for (int q = 0; q < kTileCc / 4; ++q) {
+                float4 z[kTilePx + KW - 1];
+                const float* zrow = patch + q * quad_stride + (prow * cols_in + lane * kTilePx) * 4;
 #pragma unroll
-                    for (int j = 0; j < kTilePx + KW - 1; ++j)
-                        z[j] = *reinterpret_cast<const float4*>(zrow + j * 4);
+                for (int j = 0; j < kTilePx + KW - 1; ++j)
+                    z[j] = *reinterpret_cast<const float4*>(zrow + j * 4);
 #pragma unroll
-                    for (int sx = 0; sx < KW; ++sx) {
-                        const float* wq =
-                            wsm + ((((k * p.kh + r) * KW + sx) * p.Cin) + c0 + q * 4) * 4;
-                        const float4 w0 = *reinterpret_cast<const float4*>(wq);
-                        const float4 w1 = *reinterpret_cast<const float4*>(wq + 4);
-                        const float4 w2 = *reinterpret_cast<const float4*>(wq + 8);
-                        const float4 w3 = *reinterpret_cast<const float4*>(wq + 12);
+                for (int sx = 0; sx < KW; ++sx) {
+                    const float* wq =
+                        wsm + ((((k * p.kh + r) * KW + sx) * p.Cin) + c0 + q * 4) * 4;
+                    const float4 w0 = *reinterpret_cast<const float4*>(wq);
+                    const float4 w1 = *reinterpret_cast<const float4*>(wq + 4);
+                    const float4 w2 = *reinterpret_cast<const float4*>(wq + 8);
+                    const float4 w3 = *reinterpret_cast<const float4*>(wq + 12);
 #pragma unroll
-                        for (int i = 0; i < kTilePx; ++i) {
-                            const float4 zz = z[i + sx];
-                            acc[i][0] = fmaf(zz.x, w0.x, fmaf(zz.y, w1.x, fmaf(zz.z, w2.x, fmaf(zz.w, w3.x, acc[i][0]))));
-                            acc[i][1] = fmaf(zz.x, w0.y, fmaf(zz.y, w1.y, fmaf(zz.z, w2.y, fmaf(zz.w, w3.y, acc[i][1]))));
-                            acc[i][2] = fmaf(zz.x, w0.z, fmaf(zz.y, w1.z, fmaf(zz.z, w2.z, fmaf(zz.w, w3.z, acc[i][2]))));
-                            acc[i][3] = fmaf(zz.x, w0.w, fmaf(zz.y, w1.w, fmaf(zz.z, w2.w, fmaf(zz.w, w3.w, acc[i][3]))));
-                        }
+                    for (int i = 0; i < kTilePx; ++i) {
+                        const float4 zz = z[i + sx];
+                        acc[i][0] = fmaf(zz.x, w0.x, fmaf(zz.y, w1.x, fmaf(zz.z, w2.x, fmaf(zz.w, w3.x, acc[i][0]))));
+                        acc[i][1] = fmaf(zz.x, w0.y, fmaf(zz.y, w1.y, fmaf(zz.z, w2.y, fmaf(zz.w, w3.y, acc[i][1]))));
+                        acc[i][2] = fmaf(zz.x, w0.z, fmaf(zz.y, w1.z, fmaf(zz.z, w2.z, fmaf(zz.w, w3.z, acc[i][2]))));
+                        acc[i][3] = fmaf(zz.x, w0.w, fmaf(zz.y, w1.w, fmaf(zz.z, w2.w, fmaf(zz.w, w3.w, acc[i][3]))));
                     }
                 }
             }

@@ -409,4 +409,7 @@ SIMT_TILE = [
 def test_simt_tile_thin_cout(c, tile):
     call, _ = _run_small(c, env={"CCV3D_SIMT_TILE": tile})
     assert call.plan.path["tc"] is False
-    assert call.plan.kernel == ("simt_tile" if tile else "simt"), call.plan.kernel
+    # an fp32 3x3 patch takes more 16-byte loads than a thread holds ahead
+    # (10 x 130 pixels x 2): those calls keep the thread kernel
+    fits = c.dtype == "bf16" or c.kh * c.kw == 1
+    assert call.plan.kernel == ("simt_tile" if tile and fits else "simt"), call.plan.kernel
