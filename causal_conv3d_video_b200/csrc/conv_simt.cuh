@@ -526,11 +526,18 @@ __host__ __device__ inline int simt_tile_cols_in(int kw, int d_w) {
 __host__ __device__ inline int simt_tile_patch_loads(int kh, int kw, int d_h, int d_w, int esize) {
     return simt_tile_rows_in(kh, d_h) * simt_tile_cols_in(kw, d_w) * (kTileCc * esize / 16);
 }
-// shared memory in floats: weights [kt*kh*kw*Cin][4] + one patch [2 quads][rows][cols][4]
+// Patch columns are stored permuted, column c at (c % 4) * C4 + c / 4 with
+// C4 = ceil(cols / 4): a warp whose lane l reads column 4 l + j then touches
+// 32 consecutive 16-byte words (no bank conflicts), and the permuted index of
+// 4 l + j is (j % 4) * C4 + l + j / 4.
+__host__ __device__ inline int simt_tile_c4(int kw, int d_w) {
+    return (simt_tile_cols_in(kw, d_w) + 3) / 4;
+}
+// shared memory in floats: weights [kt*kh*kw*Cin][4] + one patch [2 quads][rows][4*C4][4]
 __host__ __device__ inline long long simt_tile_smem_floats(int kt, int kh, int kw, int Cin,
                                                            int d_h, int d_w) {
     return (long long)kt * kh * kw * Cin * 4 +
-           (long long)(kTileCc / 4) * simt_tile_rows_in(kh, d_h) * simt_tile_cols_in(kw, d_w) * 4;
+           (long long)(kTileCc / 4) * simt_tile_rows_in(kh, d_h) * 4 * simt_tile_c4(kw, d_w) * 4;
 }
 
 template <typename T, int KW>
@@ -547,7 +554,9 @@ conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
     float* patch = sm + (long long)p.taps.kt * taps2d * p.Cin * 4;
     const int rows_in = simt_tile_rows_in(p.kh, p.d_h);
     const int cols_in = simt_tile_cols_in(p.kw, p.d_w);
-    const int quad_stride = rows_in * cols_in * 4;           // floats per channel quad
+    const int C4 = simt_tile_c4(p.kw, p.d_w);
+    const int row_pos = 4 * C4;                              // permuted positions per row
+    const int quad_stride = rows_in * row_pos * 4;           // floats per channel quad
 
     const int tid = threadIdx.x;
     const int tiles_x = (p.W_o + kTileCols - 1) / kTileCols;
@@ -637,11 +646,13 @@ conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
             const int e = tid + i * (int)blockDim.x;
             if (e >= nload) break;
             const int h = e % loads_px, pix = e / loads_px;
+            const int ry = pix / cols_in, rx = pix - ry * cols_in;
+            const int pos = ry * row_pos + (rx & 3) * C4 + (rx >> 2);
             float g[V];
             unpack16<T>(pf[i], g);
 #pragma unroll
             for (int q = 0; q < V / 4; ++q)
-                *reinterpret_cast<float4*>(patch + (h * (V / 4) + q) * quad_stride + pix * 4) =
+                *reinterpret_cast<float4*>(patch + (h * (V / 4) + q) * quad_stride + pos * 4) =
                     make_float4(g[4 * q], g[4 * q + 1], g[4 * q + 2], g[4 * q + 3]);
         }
         __syncthreads();
@@ -652,10 +663,10 @@ conv_simt_tile_kernel(const __grid_constant__ SimtParams p) {
 #pragma unroll
             for (int q = 0; q < kTileCc / 4; ++q) {
                 float4 z[kTilePx + KW - 1];
-                const float* zrow = patch + q * quad_stride + (prow * cols_in + lane * kTilePx) * 4;
+                const float* zrow = patch + q * quad_stride + (prow * row_pos + lane) * 4;
 #pragma unroll
-                for (int j = 0; j < kTilePx + KW - 1; ++j)
-                    z[j] = *reinterpret_cast<const float4*>(zrow + j * 4);
+                for (int j = 0; j < kTilePx + KW - 1; ++j)  // column 4 lane + j
+                    z[j] = *reinterpret_cast<const float4*>(zrow + ((j & 3) * C4 + (j >> 2)) * 4);
 #pragma unroll
                 for (int sx = 0; sx < KW; ++sx) {
                     const float* wq =

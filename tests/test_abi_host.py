@@ -222,10 +222,10 @@ def test_quantize_validation_without_gpu():
 def test_simt_variant_choice():
     """Calls too small for one thread per (pixel, 4 channels) to fill the SMs
     run one warp per unit (the lanes split the reduction)."""
-    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_smem"
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
     from parity_util import plan_env
-    with plan_env({"CCV3D_SIMT_SMEM": 0}):
-        assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
+    with plan_env({"CCV3D_SIMT_SMEM": 1}):  # the shared-memory kernel is opt-in
+        assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_smem"
     # weights of 384 -> 384 x 27 fp32 (15.9 MB) do not fit in shared memory
     wide = workloads.Conv("f32_wide", 384, 384, 4, 4, T_x=1, cache_len=2, dtype="fp32")
     assert ccv3d.Plan(ccv3d.desc_for(wide)).kernel == "simt_warp"

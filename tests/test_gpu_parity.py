@@ -242,7 +242,7 @@ def test_small_simt_bf16(c, smem):
 def test_small_simt_other(c):
     call, _ = _run_small(c)
     assert call.plan.path["tc"] is False
-    call, _ = _run_small(c, env={"CCV3D_SIMT_SMEM": 0})
+    call, _ = _run_small(c, env={"CCV3D_SIMT_SMEM": 1})
     assert call.plan.path["tc"] is False
 
 
