@@ -220,6 +220,7 @@ void set_smem_attrs() {
 struct ResidentEntry {
     int dev, bk, pairs;
     size_t smem;
+    int threads;
 };
 constexpr int kResidentEntries = 64;
 std::mutex g_resident_mu;
@@ -227,7 +228,7 @@ ResidentEntry g_resident[kResidentEntries];
 int g_resident_n = 0;
 
 template <int BK>
-int resident_pairs(size_t smem, bool fused = false) {
+int resident_pairs(size_t smem, bool fused = false, int threads = kTcpThreads) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -237,13 +238,13 @@ int resident_pairs(size_t smem, bool fused = false) {
         std::lock_guard<std::mutex> lock(g_resident_mu);
         for (int i = 0; i < g_resident_n; ++i)
             if (g_resident[i].dev == dev && g_resident[i].bk == (fused ? -BK : BK) &&
-                g_resident[i].smem == smem)
+                g_resident[i].smem == smem && g_resident[i].threads == threads)
                 return g_resident[i].pairs;
     }
     set_smem_attrs<BK>();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kTcpThreads, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     int n = 0;
     const cudaError_t e = fused ? cudaOccupancyMaxActiveClusters(&n, conv_tc2fp_kernel<BK>, &cfg)
@@ -253,7 +254,8 @@ int resident_pairs(size_t smem, bool fused = false) {
         return 0;
     }
     std::lock_guard<std::mutex> lock(g_resident_mu);
-    if (g_resident_n < kResidentEntries) g_resident[g_resident_n++] = {dev, fused ? -BK : BK, n, smem};
+    if (g_resident_n < kResidentEntries)
+        g_resident[g_resident_n++] = {dev, fused ? -BK : BK, n, smem, threads};
     return n;
 }
 
@@ -413,23 +415,24 @@ size_t fused_persist_smem_for(int bk, int bn, int stages, int kh, int kw, int ha
 // keeps at least four stages.  Opt-in (CCV3D_FUSED_PERSIST=1) until measured.
 void setup_fused_persistent(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->fused_persist = 0;
-    if (!p->fused || p->persist) return;
-    if (!(override_env("CCV3D_FUSED_PERSIST") != nullptr && env_int("CCV3D_FUSED_PERSIST") > 0))
-        return;
+    const int mode = env_int("CCV3D_FUSED_PERSIST");  // 1: one CTA per SM, 2: two
+    if (!p->fused || p->persist || mode <= 0) return;
     const int want_s = env_int("CCV3D_STAGES");
-    for (int min_s : {4, 2})
+    const size_t budget = mode == 2 ? kSmemBudget / 2 : kSmemBudget;
+    for (int min_s : {4, 3, 2})
         for (int bk : {64, 32, 16}) {
             if (d.Cin % bk != 0) continue;
             int s = want_s >= 2 ? want_s : 12;
-            while (s >= 2 && fused_persist_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w) > kSmemBudget)
+            while (s >= 2 && fused_persist_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w) > budget)
                 --s;
             if (s < min_s) continue;
             p->fused_persist = 1;
             p->BK = bk;
             p->stages = s;
             p->smem_bytes = fused_persist_smem_for(bk, p->BN, s, d.kh, d.kw, p->halo_w);
+            p->n_acc = mode == 2 ? 1 : 2;
             p->tmem_cols = 32;
-            while (p->tmem_cols < 4 * p->BN) p->tmem_cols *= 2;  // two buffers of two frames
+            while (p->tmem_cols < 2 * p->n_acc * p->BN) p->tmem_cols *= 2;  // buffers of two frames
             return;
         }
 }
@@ -480,8 +483,13 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     // Cout tile: up to 256 columns per MMA, up to 2 MMAs (512 TMEM columns).
     // One CTA covers up to 384 output channels so that each A box is loaded
     // once for all of them (measured best on the 384-channel decoder calls).
+    // Wider outputs that split into 256-column tiles (768 = 3 x 256) take
+    // those instead, on the persistent kernel (below): one N = 256 MMA per
+    // k-step and double-buffered accumulators, 136 against 148 us on the
+    // 3x1x1 384 -> 768 call at 180x320.
     const int want_n = env_int("CCV3D_TILE_N");
-    const int max_n = (want_n >= 16 && want_n <= 512) ? want_n : 384;
+    const bool wide256 = want_n == 0 && d.Cout > 384 && d.Cout % 256 == 0;
+    const int max_n = (want_n >= 16 && want_n <= 512) ? want_n : (wide256 ? 256 : 384);
     p->tiles_n = ceil_div(d.Cout, max_n);
     p->BN = ((ceil_div(d.Cout, p->tiles_n) + 15) / 16) * 16;
     p->n_sub = p->BN > 256 ? 2 : 1;
@@ -497,7 +505,7 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     setup_halo(d, p);
     setup_fused(d, p);
     const char* ps = override_env("CCV3D_PERSIST");
-    const bool persist = ps != nullptr ? std::atoi(ps) > 0 : prefer_persistent(d, *p);
+    const bool persist = ps != nullptr ? std::atoi(ps) > 0 : (wide256 || prefer_persistent(d, *p));
     if (persist && setup_persistent(d, p)) size_tc(d, p);
     setup_fused_persistent(d, p);
     p->path_tc = 1;
@@ -505,16 +513,22 @@ void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
 
 // Persistent grid size: one CTA pair per resident pair slot, but at least 32
 // k-blocks per pair.  CCV3D_SK_PAIRS forces a size (tests of split tiles).
+// Threads of the persistent two-frame kernel: with two CTAs per SM (one
+// accumulator buffer each) it runs without the copy warps, so that two CTAs'
+// registers fit on an SM.
+int fused_persist_threads(const ccv3d_plan_s* p) { return p->n_acc == 1 ? 192 : kTcpThreads; }
+
 void size_persistent(ccv3d_plan_s* p, bool have_device) {
     if (p->fused_persist) {
         // one CTA pair per resident pair slot, at most one per tile; no scratch
         int pairs = 74;
         if (have_device) {
             int n = 0;
+            const int th = fused_persist_threads(p);
             switch (p->BK) {
-                case 64: n = resident_pairs<64>(p->smem_bytes, true); break;
-                case 32: n = resident_pairs<32>(p->smem_bytes, true); break;
-                default: n = resident_pairs<16>(p->smem_bytes, true); break;
+                case 64: n = resident_pairs<64>(p->smem_bytes, true, th); break;
+                case 32: n = resident_pairs<32>(p->smem_bytes, true, th); break;
+                default: n = resident_pairs<16>(p->smem_bytes, true, th); break;
             }
             if (n > 0) pairs = n;
         }
@@ -715,7 +729,8 @@ void plan_paced_copy(const ccv3d_plan_s* p, TcParams& prm) {
 void plan_paced_copy_fused(const ccv3d_plan_s* p, TcParams& prm) {
     prm.copy.paced_mask = 0u;
     const int keep = prm.copy.keep;
-    if (keep <= 0 || keep > kMaxPaced || !paced_copy_on()) return;
+    // (the two-CTA-per-SM form has no copy warps: it takes the sliced copy)
+    if (keep <= 0 || keep > kMaxPaced || !paced_copy_on() || p->n_acc == 1) return;
     const ccv3d_desc& d = p->d;
     for (int j = 0; j < keep; ++j) {
         const int t = p->z_len - keep + j;
@@ -731,10 +746,11 @@ void plan_paced_copy_fused(const ccv3d_plan_s* p, TcParams& prm) {
 }
 
 template <int BK>
-cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s,
+                      int threads) {
     set_smem_attrs<BK>();
     if (kind == 5)
-        conv_tc2fp_kernel<BK><<<grid, kTcpThreads, smem, s>>>(prm);
+        conv_tc2fp_kernel<BK><<<grid, threads, smem, s>>>(prm);
     else if (kind == 4)
         conv_tc2f_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
     else if (kind == 3)
@@ -788,6 +804,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     if (p->fused) grid = 2LL * d.N * ((p->T_o + 1) / 2) * prm.pairs_per_frame;  // frame pairs
     if (p->fused_persist) {
         grid = 2LL * p->G;
+        prm.sk.n_acc = p->n_acc;
         plan_paced_copy_fused(p, prm);
     }
     if (p->persist) {
@@ -815,10 +832,11 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     const int kind = p->fused_persist ? 5 : (p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair)));
     prm.halo_w = p->halo_w;
     cudaError_t e;
+    const int threads = p->fused_persist ? fused_persist_threads(p) : kTcpThreads;
     switch (p->BK) {
-        case 64: e = launch_tc<64>(prm, kind, (int)grid, p->smem_bytes, stream); break;
-        case 32: e = launch_tc<32>(prm, kind, (int)grid, p->smem_bytes, stream); break;
-        default: e = launch_tc<16>(prm, kind, (int)grid, p->smem_bytes, stream); break;
+        case 64: e = launch_tc<64>(prm, kind, (int)grid, p->smem_bytes, stream, threads); break;
+        case 32: e = launch_tc<32>(prm, kind, (int)grid, p->smem_bytes, stream, threads); break;
+        default: e = launch_tc<16>(prm, kind, (int)grid, p->smem_bytes, stream, threads); break;
     }
     return e == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
 }

@@ -10,9 +10,11 @@
 // and walks the tiles g, g + G, g + 2G, ... (G pairs), so
 //   * the operand ring runs continuously across tiles (no per-tile prologue,
 //     pipeline fill or drain);
-//   * the accumulators are double-buffered in TMEM (2 x 2 Cout columns): the
-//     epilogue warps drain tile u's frames while the MMA issuer fills tile
-//     u + 1's buffer;
+//   * the accumulators are double-buffered in TMEM (2 x 2 Cout columns) when
+//     the kernel runs one CTA per SM: the epilogue warps drain tile u's
+//     frames while the MMA issuer fills tile u + 1's buffer; sized for two
+//     CTAs per SM (n_acc = 1) each CTA holds one buffer and the other CTA's
+//     MMAs run while it drains;
 //   * the epilogue stages output blocks in two dedicated buffers (the ring is
 //     never idle) and stores them with TMA tensor stores;
 //   * warps 6-9 copy new_cache: frames no tap reads in equal slices at the
@@ -121,6 +123,7 @@ conv_tc2fp_kernel(const __grid_constant__ TcParams p) {
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
+    const int n_acc = p.sk.n_acc;  // TMEM accumulator buffers (1 or 2)
     const int G = (int)(gridDim.x >> 1);
     const int g = (int)(blockIdx.x >> 1);
     const int fpairs = (p.T_o + 1) / 2;
@@ -245,7 +248,7 @@ conv_tc2fp_kernel(const __grid_constant__ TcParams p) {
                 const int o0 = (fp % fpairs) * 2;
                 const FusedSrc src = fused_sources(p, o0);
                 const int iters = src.n * p.n_cb * p.kh;
-                const int b = u & 1, round = u >> 1;
+                const int b = n_acc == 2 ? (u & 1) : 0, round = n_acc == 2 ? (u >> 1) : u;
                 if (round > 0 &&
                     !mbar_wait(smem_u32(&acc_empty[b]), (uint32_t)((round & 1) ^ 1), p.status,
                                p.wait_limit_ns)) {
@@ -330,6 +333,9 @@ conv_tc2fp_kernel(const __grid_constant__ TcParams p) {
         // ------------------------------------------------- the epilogues
         const int etid = threadIdx.x - 64;
         const int q = warp & 3;
+        // launched without copy warps (192 threads, two CTAs per SM): the
+        // epilogue warps take the sliced new_cache copy before the first tile
+        if (blockDim.x <= 192) copy_new_cache(p.copy, blockIdx.x, gridDim.x, etid, 128);
         const uint32_t empty_leader = mapa_cluster(smem_u32(&acc_empty[0]), 0);
         int slot = 0;
         bool ok = true;
@@ -344,7 +350,7 @@ conv_tc2fp_kernel(const __grid_constant__ TcParams p) {
                 ty = box / p.tiles_x;
             }
             const FusedSrc src = fused_sources(p, o0);
-            const int b = u & 1, round = u >> 1;
+            const int b = n_acc == 2 ? (u & 1) : 0, round = n_acc == 2 ? (u >> 1) : u;
             if (ok && !mbar_wait(smem_u32(&acc_full[b]), (uint32_t)(round & 1), p.status,
                                  p.wait_limit_ns))
                 ok = false;

@@ -163,7 +163,7 @@ def test_tile_choice_on_bottleneck():
     plan = ccv3d.Plan(ccv3d.desc_for(workloads.C2))
     assert plan.path == {"tc": True, "tile_m": 256, "tile_n": 384}
     assert ccv3d.Plan(ccv3d.desc_for(workloads.C3)).path["tile_n"] == 96
-    assert ccv3d.Plan(ccv3d.desc_for(workloads.C4_TIME)).path["tile_n"] == 384
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C4_TIME)).path["tile_n"] == 256  # 768 = 3 x 256
     thin = ccv3d.Plan(ccv3d.make_desc(N=1, Cin=3, Cout=16, H=8, W=8, T_x=1, cache_len=0))
     assert thin.path["tc"] is False
 

@@ -357,14 +357,15 @@ def test_persistent_new_cache_paced_or_sliced(c, paced, pairs):
     assert call.plan.kernel == "tc_persistent"
 
 
-@pytest.mark.parametrize("paced", [1, 0], ids=["paced", "sliced"])
+@pytest.mark.parametrize("mode,paced", [(1, 1), (1, 0), (2, 0)],
+                         ids=["one_cta_paced", "one_cta_sliced", "two_ctas"])
 @pytest.mark.parametrize("c", FUSED, ids=lambda c: c.name)
-def test_small_fused_persistent(c, paced):
-    """The persistent form of the two-frame kernel: the same stages, one CTA
-    pair per SM pair walking the tiles with double-buffered accumulators; with
-    a few pairs every pair runs many tiles, so both accumulator buffers and
-    both staging buffers cycle."""
-    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_FUSED_PERSIST": 1,
+def test_small_fused_persistent(c, mode, paced):
+    """The persistent form of the two-frame kernel: the same stages, CTA pairs
+    walking the tiles, with double-buffered accumulators at one CTA per SM or
+    one buffer each at two CTAs per SM (no copy warps); every pair runs many
+    tiles, so the accumulator and staging buffers cycle."""
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_FUSED_PERSIST": mode,
                                  "CCV3D_PACED": paced})
     assert call.plan.kernel == "tc_pair_fused_persistent", call.plan.kernel
     first = call.out.clone()

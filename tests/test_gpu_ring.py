@@ -126,6 +126,8 @@ RING_SIGS = [
      {"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1}),
     (Conv("r96_fused_persist_t3", 96, 96, 3, 256, T_x=3, cache_len=0, sigma_b=0.1),
      {"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_FUSED_PERSIST": 1}),
+    (Conv("r96_fused_persist2_t3", 96, 96, 3, 256, T_x=3, cache_len=0, sigma_b=0.1),
+     {"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_FUSED_PERSIST": 2}),
     (Conv("r64_dt2", 64, 64, 18, 32, T_x=1, cache_len=0, dilation=(2, 1, 1)), {}),
     (Conv("r32_batch2_t2", 32, 48, 10, 12, T_x=2, cache_len=0, N=2), {}),
     (Conv("r16_fp32", 16, 16, 16, 16, T_x=3, cache_len=0, dtype="fp32", sigma_b=0.1), {}),
