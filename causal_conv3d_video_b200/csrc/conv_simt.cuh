@@ -196,6 +196,65 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
     float acc[kSimtCoT];
 #pragma unroll
     for (int j = 0; j < kSimtCoT; ++j) acc[j] = 0.f;
+    if (32 % p.Cin == 0) {
+        // Cin divides 32 (the 16-channel contract call): lane = (tap offset,
+        // channel); a lane walks the taps tpi = 32 / Cin apart with its
+        // (k, r, s) position advanced step by step -- no division in the loop
+        const int tpi = 32 / p.Cin, ci = lane % p.Cin;
+        const int ntaps = p.taps.kt * taps2d;
+        int t = lane / p.Cin;
+        int k = t / taps2d, r = (t % taps2d) / p.kw, sx = t % p.kw;
+        constexpr int kU = 4;
+        while (t < ntaps) {
+            float z[kU], wv[kU][kSimtCoT];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                z[u] = 0.f;
+#pragma unroll
+                for (int j = 0; j < kSimtCoT; ++j) wv[u][j] = 0.f;
+                if (t < ntaps) {
+                    const int yi = yo * p.s_h + r * p.d_h - p.p_h;
+                    const int xi = xo * p.s_w + sx * p.d_w - p.p_w;
+                    if (o >= p.taps.o_l[k] && o < p.taps.o_h[k] && yi >= 0 && yi < p.H &&
+                        xi >= 0 && xi < p.W) {
+                        const int tf = o * p.taps.s_t + p.taps.delta[k];
+                        const T* frame =
+                            tf < p.cache_len
+                                ? cache + (long long)ring_frame(n, tf, p.cache_slots,
+                                                                p.cache_head) * p.H * p.W * p.Cin
+                                : x + ((long long)n * p.T_x + (tf - p.cache_len)) * p.H * p.W *
+                                          p.Cin;
+                        const T* zp = frame + ((long long)yi * p.W + xi) * p.Cin + ci;
+                        if (in_bounds(p.status, zp, sizeof(T),
+                                      tf < p.cache_len ? (const void*)cache : (const void*)x,
+                                      tf < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
+                            z[u] = to_f32<T>(*zp);
+                        const T* wcol = w + (long long)co0 * w_co_stride + (long long)t * p.Cin + ci;
+#pragma unroll
+                        for (int j = 0; j < kSimtCoT; ++j)
+                            if (co0 + j < p.Cout &&
+                                in_bounds(p.status, wcol + j * w_co_stride, sizeof(T), w,
+                                          p.w_floats * (long long)sizeof(T)))
+                                wv[u][j] = to_f32<T>(wcol[j * w_co_stride]);
+                    }
+                    // next tap of this lane: tpi single steps of (k, r, s)
+                    t += tpi;
+                    for (int q = 0; q < tpi; ++q)
+                        if (++sx == p.kw) {
+                            sx = 0;
+                            if (++r == p.kh) {
+                                r = 0;
+                                ++k;
+                            }
+                        }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+#pragma unroll
+                for (int j = 0; j < kSimtCoT; ++j) acc[j] = fmaf(z[u], wv[u][j], acc[j]);
+        }
+    } else {
     // kU reduction steps per lane at a time: their (predicated) loads are
     // independent, so they are all in flight before the FMAs need them
     constexpr int kU = 4;
@@ -241,6 +300,7 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
         for (int u = 0; u < kU; ++u)
 #pragma unroll
             for (int j = 0; j < kSimtCoT; ++j) acc[j] = fmaf(z[u], wv[u][j], acc[j]);
+    }
     }
 #pragma unroll
     for (int j = 0; j < kSimtCoT; ++j)
