@@ -577,6 +577,9 @@ def time_leg(conv, ring, dev, peaks, sampler, seconds=0.6, min_calls=20, max_cal
     t_flop = flops / (peak * 1e12) * 1e6
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_star = max(t_flop, t_hbm)
+    # the leg runs ~0.6 s of back-to-back calls: a kernel timed inside a long
+    # run, for which the sustained (power-capped) tensor peak is the measure
+    sustained = peaks.get("bf16_tflops_sustained")
     line = {
         "kernel": plan.kernel, "calls": n, "us_per_call_median": round(us, 2),
         "us_per_call_min": round(min(per), 2),
@@ -589,6 +592,8 @@ def time_leg(conv, ring, dev, peaks, sampler, seconds=0.6, min_calls=20, max_cal
             "traffic": traffic_from_profiles(conv.name + ("+ring" if ring else "")),
         },
         "tensor_frac": round(t_flop / us, 4) if conv.dtype == "bf16" else None,
+        "frac_of_sustained": (round(max(flops / (sustained * 1e12) * 1e6, t_hbm) / us, 4)
+                              if conv.dtype == "bf16" and sustained else None),
         "hbm_frac": round(t_hbm / us, 4),
         "l2": ("256 MB buffer written between calls" if flush
                else f"rotating {n_sets} operand sets ({n_sets * nbytes / 1e6:.0f} MB)"),
