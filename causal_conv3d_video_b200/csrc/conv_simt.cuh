@@ -173,17 +173,18 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
                        blockDim.x);
         return;
     }
-    const long long unit = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    // small calls only (fewer than 148 x 128 units): 32-bit unit decode
+    const int unit = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     const int lane = threadIdx.x & 31;
     if (unit >= p.conv_threads) return;  // whole warps leave together
-    const int cog = (int)(unit % p.co_groups);
-    long long pix = unit / p.co_groups;
-    const int xo = (int)(pix % p.W_o);
+    const int cog = unit % p.co_groups;
+    int pix = unit / p.co_groups;
+    const int xo = pix % p.W_o;
     pix /= p.W_o;
-    const int yo = (int)(pix % p.H_o);
+    const int yo = pix % p.H_o;
     pix /= p.H_o;
-    const int o = (int)(pix % p.T_o);
-    const int n = (int)(pix / p.T_o);
+    const int o = pix % p.T_o;
+    const int n = pix / p.T_o;
     const int co0 = cog * kSimtCoT;
 
     const T* x = static_cast<const T*>(p.x);
@@ -199,60 +200,59 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
     if (32 % p.Cin == 0) {
         // Cin divides 32 (the 16-channel contract call): lane = (tap offset,
         // channel); a lane walks the taps tpi = 32 / Cin apart with its
-        // (k, r, s) position advanced step by step -- no division in the loop
+        // (k, r, s) position advanced step by step.  The temporal taps' frame
+        // pointers and the weight base are fixed per warp, and offsets inside
+        // a frame are 32-bit (a frame holds < 2^31 elements), so a reduction
+        // step is a handful of integer ops, two loads and four FMAs.
         const int tpi = 32 / p.Cin, ci = lane % p.Cin;
         const int ntaps = p.taps.kt * taps2d;
+        const T* fb[kMaxTaps];
+        bool act[kMaxTaps];
+#pragma unroll
+        for (int k = 0; k < kMaxTaps; ++k) {
+            act[k] = k < p.taps.kt && o >= p.taps.o_l[k] && o < p.taps.o_h[k];
+            const int tf = o * p.taps.s_t + p.taps.delta[k];
+            fb[k] = !act[k] ? x
+                            : (tf < p.cache_len
+                                   ? cache + (long long)ring_frame(n, tf, p.cache_slots,
+                                                                   p.cache_head) *
+                                                 p.H * p.W * p.Cin
+                                   : x + ((long long)n * p.T_x + (tf - p.cache_len)) * p.H *
+                                             p.W * p.Cin);
+        }
+        const int ybase = yo * p.s_h - p.p_h, xbase = xo * p.s_w - p.p_w;
+        const T* wb = w + (long long)co0 * w_co_stride + ci;  // + j w_co_stride + t Cin
+        const int jmax = min(kSimtCoT, p.Cout - co0);
         int t = lane / p.Cin;
-        int k = t / taps2d, r = (t % taps2d) / p.kw, sx = t % p.kw;
-        constexpr int kU = 4;
-        while (t < ntaps) {
-            float z[kU], wv[kU][kSimtCoT];
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                z[u] = 0.f;
-#pragma unroll
-                for (int j = 0; j < kSimtCoT; ++j) wv[u][j] = 0.f;
-                if (t < ntaps) {
-                    const int yi = yo * p.s_h + r * p.d_h - p.p_h;
-                    const int xi = xo * p.s_w + sx * p.d_w - p.p_w;
-                    if (o >= p.taps.o_l[k] && o < p.taps.o_h[k] && yi >= 0 && yi < p.H &&
-                        xi >= 0 && xi < p.W) {
-                        const int tf = o * p.taps.s_t + p.taps.delta[k];
-                        const T* frame =
-                            tf < p.cache_len
-                                ? cache + (long long)ring_frame(n, tf, p.cache_slots,
-                                                                p.cache_head) * p.H * p.W * p.Cin
-                                : x + ((long long)n * p.T_x + (tf - p.cache_len)) * p.H * p.W *
-                                          p.Cin;
-                        const T* zp = frame + ((long long)yi * p.W + xi) * p.Cin + ci;
-                        if (in_bounds(p.status, zp, sizeof(T),
-                                      tf < p.cache_len ? (const void*)cache : (const void*)x,
-                                      tf < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
-                            z[u] = to_f32<T>(*zp);
-                        const T* wcol = w + (long long)co0 * w_co_stride + (long long)t * p.Cin + ci;
-#pragma unroll
-                        for (int j = 0; j < kSimtCoT; ++j)
-                            if (co0 + j < p.Cout &&
-                                in_bounds(p.status, wcol + j * w_co_stride, sizeof(T), w,
-                                          p.w_floats * (long long)sizeof(T)))
-                                wv[u][j] = to_f32<T>(wcol[j * w_co_stride]);
-                    }
-                    // next tap of this lane: tpi single steps of (k, r, s)
-                    t += tpi;
-                    for (int q = 0; q < tpi; ++q)
-                        if (++sx == p.kw) {
-                            sx = 0;
-                            if (++r == p.kh) {
-                                r = 0;
-                                ++k;
-                            }
-                        }
-                }
+        int k = t / taps2d, r = (t - k * taps2d) / p.kw, sx = t - k * taps2d - r * p.kw;
+#pragma unroll 4
+        for (; t < ntaps; t += tpi) {
+            const int yi = ybase + r * p.d_h, xi = xbase + sx * p.d_w;
+            const T* f = k == 0 ? fb[0] : (k == 1 ? fb[1] : fb[2]);
+            const bool a = k == 0 ? act[0] : (k == 1 ? act[1] : act[2]);
+            float z = 0.f;
+            if (a && (unsigned)yi < (unsigned)p.H && (unsigned)xi < (unsigned)p.W) {
+                const T* zp = f + (yi * p.W + xi) * p.Cin + ci;
+                const int tf = o * p.taps.s_t + p.taps.delta[k];
+                if (in_bounds(p.status, zp, sizeof(T),
+                              tf < p.cache_len ? (const void*)cache : (const void*)x,
+                              tf < p.cache_len ? p.copy.cache_bytes : p.copy.x_bytes))
+                    z = to_f32<T>(__ldg(zp));
             }
+            const T* wt = wb + t * p.Cin;
 #pragma unroll
-            for (int u = 0; u < kU; ++u)
-#pragma unroll
-                for (int j = 0; j < kSimtCoT; ++j) acc[j] = fmaf(z[u], wv[u][j], acc[j]);
+            for (int j = 0; j < kSimtCoT; ++j)
+                if (j < jmax && in_bounds(p.status, wt + j * w_co_stride, sizeof(T), w,
+                                          p.w_floats * (long long)sizeof(T)))
+                    acc[j] = fmaf(z, to_f32<T>(__ldg(wt + j * w_co_stride)), acc[j]);
+            for (int q = 0; q < tpi; ++q)  // next tap of this lane
+                if (++sx == p.kw) {
+                    sx = 0;
+                    if (++r == p.kh) {
+                        r = 0;
+                        ++k;
+                    }
+                }
         }
     } else {
     // kU reduction steps per lane at a time: their (predicated) loads are
