@@ -29,6 +29,7 @@
 #include "conv_tc2fp.cuh"
 #include "conv_tc2h.cuh"
 #include "conv_tcp.cuh"
+#include "conv_tcn.cuh"
 #include "params.h"
 #include "quantize.cuh"
 
@@ -47,6 +48,8 @@ struct ccv3d_plan_s {
     int halo_w;   // halo: pixels per strip
     int fused;    // 1: halo pair kernel computing two output frames per tile
     int fused_persist;  // 1: the persistent form of the two-frame kernel (conv_tc2fp.cuh)
+    int thin;     // 1: thin-output kernel, taps stacked along N (conv_tcn.cuh)
+    int tn_G, tn_groups, tn_cbk;  // thin: frames per tile, frame groups, TMEM columns per frame
     int simt_kind;  // SIMT plans: 0 thread per unit, 1 warp per unit, 2 shared-memory blocks
     int simt_band_h, simt_rows_in, simt_threads;
     size_t simt_smem;
@@ -208,6 +211,8 @@ void set_smem_attrs() {
         cudaFuncSetAttribute(conv_tc2f_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaFuncSetAttribute(conv_tc2fp_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(227 * 1024));
+        cudaFuncSetAttribute(conv_tcn_kernel<BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(227 * 1024));
         cudaGetLastError();
     }
@@ -456,12 +461,84 @@ bool prefer_persistent(const ccv3d_desc& d, const ccv3d_plan_s& p) {
     return waves >= 2.0 && waves / std::ceil(waves) < 0.9;
 }
 
+size_t thin_smem_for(int bk, int n, int stages, int kw, int cout) {
+    switch (bk) {
+        case 64: return tcn_smem_bytes<64>(n, stages, kw, cout);
+        case 32: return tcn_smem_bytes<32>(n, stages, kw, cout);
+        default: return tcn_smem_bytes<16>(n, stages, kw, cout);
+    }
+}
+
+// Thin outputs (conv_tcn.cuh): Cout too narrow for an MMA's N (not a multiple
+// of 16, e.g. the RGB output conv 96 -> 3).  The kernel stacks the temporal
+// and column taps along N (kt blocks of kw*Cout rounded up to 16 columns) and
+// needs unit temporal stride and dilation and unit W stride.  A tile covers
+// one output row, 128 - (kw-1)*d_w output pixels and a group of G output
+// frames whose accumulators take (G + kt - 2) blocks + N TMEM columns; G is
+// as large as 256 columns allow (two CTAs per SM), in equal groups.  Stages
+// aim at three CTAs per SM so that one CTA's epilogue overlaps the others'
+// MMAs.  CCV3D_THIN=0 disables the kernel; CCV3D_THIN=1 also takes it for
+// Cout that are multiples of 16 (tests).
+bool setup_thin(const ccv3d_desc& d, ccv3d_plan_s* p) {
+    p->thin = 0;
+    const char* te = override_env("CCV3D_THIN");
+    if (te != nullptr && std::atoi(te) == 0) return false;
+    if (d.dtype != CCV3D_BF16 || d.Cin % 16 != 0 || force_simt()) return false;
+    if (d.stride_t != 1 || d.dil_t != 1 || d.stride_w != 1) return false;
+    const int cbk = ((d.kw * d.Cout + 15) / 16) * 16;
+    const int nb = d.kt * cbk;
+    if (nb > 256) return false;
+    const int mo = kTileM - (d.kw - 1) * d.dil_w;
+    if (mo < 64) return false;
+    const int gmax = (256 - nb) / cbk - d.kt + 2;
+    if (gmax < 1) return false;
+    const int groups = ceil_div(p->T_o, gmax);
+    const int G = ceil_div(p->T_o, groups);
+    const int bk = widest_bk(d.Cin);
+    const int want_s = env_int("CCV3D_STAGES");
+    int s = want_s >= 2 ? want_s : 8;
+    const size_t cap = want_s >= 2 ? kSmemBudget : kSmemBudget / 3;
+    while (s >= 2 && thin_smem_for(bk, nb, s, d.kw, d.Cout) > cap) --s;
+    if (s < 2) return false;
+    p->thin = 1;
+    p->path_tc = 1;
+    p->pair = p->persist = p->halo = p->fused = p->fused_persist = 0;
+    p->BK = bk;
+    p->BN = nb;
+    p->n_sub = 1;
+    p->stages = s;
+    p->smem_bytes = thin_smem_for(bk, nb, s, d.kw, d.Cout);
+    p->box_w = mo;
+    p->box_h = 1;
+    p->halo_w = kTileM;
+    p->tiles_x = ceil_div(p->W_o, mo);
+    p->tiles_y = p->H_o;
+    p->tiles_n = 1;
+    p->tn_G = G;
+    p->tn_groups = groups;
+    p->tn_cbk = cbk;
+    const int cols = cbk * (G + d.kt - 2) + nb;
+    p->tmem_cols = 32;
+    while (p->tmem_cols < cols) p->tmem_cols *= 2;
+    // no more CTAs per SM than their TMEM columns fit (a further CTA's
+    // allocation would wait for one of them to finish): request enough
+    // shared memory to keep the (512 / tmem_cols + 1)-th CTA off the SM
+    const size_t per_sm = 228 * 1024;
+    const size_t floor_bytes = per_sm / (size_t)(512 / p->tmem_cols + 1) + 1024;
+    if (p->smem_bytes < floor_bytes) p->smem_bytes = floor_bytes;
+    return true;
+}
+
 // Kernel choice and tiling.
 void choose_path(const ccv3d_desc& d, ccv3d_plan_s* p) {
     p->path_tc = 0;
+    p->thin = 0;
     const bool tc_ok = d.dtype == CCV3D_BF16 && d.Cin % 16 == 0 && d.Cout % 16 == 0 &&
                        d.stride_h <= 2 && d.stride_w <= 2 && !force_simt();
-    if (!tc_ok) return;
+    if (!tc_ok || env_int("CCV3D_THIN") > 0) {
+        setup_thin(d, p);
+        return;
+    }
     // spatial box of 128 output pixels: fewest tiles, then widest rows
     int best_w = 0, best_tiles = 0;
     const int want_w = env_int("CCV3D_BOX_W");
@@ -572,13 +649,14 @@ ccv3d_status encode_act(CUtensorMap* m, const void* base, int frames, const ccv3
                                 (cuuint64_t)frames};
     const cuuint64_t strides[3] = {(cuuint64_t)d.Cin * 2, (cuuint64_t)d.W * d.Cin * 2,
                                    (cuuint64_t)d.H * d.W * d.Cin * 2};
-    // halo kernel: one input row strip of halo_w pixels; otherwise the
+    // halo and thin kernels: one input row strip of halo_w pixels; otherwise the
     // shifted, strided box of box_h x box_w output pixels
+    const bool strip = p->halo || p->thin;
     const cuuint32_t box[4] = {(cuuint32_t)p->BK,
-                               (cuuint32_t)(p->halo ? p->halo_w : p->box_w * d.stride_w),
-                               (cuuint32_t)(p->halo ? 1 : p->box_h * d.stride_h), 1};
-    const cuuint32_t estr[4] = {1, p->halo ? 1u : (cuuint32_t)d.stride_w,
-                                p->halo ? 1u : (cuuint32_t)d.stride_h, 1};
+                               (cuuint32_t)(strip ? p->halo_w : p->box_w * d.stride_w),
+                               (cuuint32_t)(strip ? 1 : p->box_h * d.stride_h), 1};
+    const cuuint32_t estr[4] = {1, strip ? 1u : (cuuint32_t)d.stride_w,
+                                strip ? 1u : (cuuint32_t)d.stride_h, 1};
     const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -602,6 +680,50 @@ ccv3d_status encode_w(CUtensorMap* m, const void* base, const ccv3d_desc& d,
                                   : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
     CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+// Weights as [taps, Cout, Cin] (a view of the [Cout, taps, Cin] tensor with
+// the two outer strides swapped), box [BK, rows, kw]: one load brings a kernel
+// row's kw column taps of `rows` output channels, as kw K-major tiles.
+ccv3d_status encode_w_kw(CUtensorMap* m, const void* base, const ccv3d_desc& d,
+                         const ccv3d_plan_s* p, int rows) {
+    const int taps = d.kt * d.kh * d.kw;
+    const cuuint64_t dims[3] = {(cuuint64_t)d.Cin, (cuuint64_t)d.Cout, (cuuint64_t)taps};
+    const cuuint64_t strides[2] = {(cuuint64_t)taps * d.Cin * 2, (cuuint64_t)d.Cin * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)p->BK, (cuuint32_t)rows, (cuuint32_t)d.kw};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? CCV3D_OK : CCV3D_ERR_CUDA;
+}
+
+// Thin-output kernel: weights as the 5-D tensor [kt, kh, kw, Cout, Cin]
+// (dims Cin, Cout, kw, kh, kt; a view of [Cout, kt, kh, kw, Cin]), box
+// [BK, Cout, kw, 1, 1]: one load brings temporal tap k's kw x Cout rows of
+// kernel row r, row s*Cout + co, as one K-major tile.
+ccv3d_status encode_w_thin(CUtensorMap* m, const void* base, const ccv3d_desc& d,
+                           const ccv3d_plan_s* p) {
+    const cuuint64_t e = 2;
+    const cuuint64_t dims[5] = {(cuuint64_t)d.Cin, (cuuint64_t)d.Cout, (cuuint64_t)d.kw,
+                                (cuuint64_t)d.kh, (cuuint64_t)d.kt};
+    const cuuint64_t strides[4] = {(cuuint64_t)d.kt * d.kh * d.kw * d.Cin * e,
+                                   (cuuint64_t)d.Cin * e, (cuuint64_t)d.kw * d.Cin * e,
+                                   (cuuint64_t)d.kh * d.kw * d.Cin * e};
+    const cuuint32_t box[5] = {(cuuint32_t)p->BK, (cuuint32_t)d.Cout, (cuuint32_t)d.kw, 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = p->BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : p->BK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base),
                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -749,7 +871,9 @@ template <int BK>
 cudaError_t launch_tc(const TcParams& prm, int kind, int grid, size_t smem, cudaStream_t s,
                       int threads) {
     set_smem_attrs<BK>();
-    if (kind == 5)
+    if (kind == 6)
+        conv_tcn_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
+    else if (kind == 5)
         conv_tc2fp_kernel<BK><<<grid, threads, smem, s>>>(prm);
     else if (kind == 4)
         conv_tc2f_kernel<BK><<<grid, kTcThreads, smem, s>>>(prm);
@@ -773,8 +897,18 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     ccv3d_status st = encode_act(&prm.tmap_x, x, d.N * d.T_x, d, p);
     if (st == CCV3D_OK && d.cache_len > 0)
         st = encode_act(&prm.tmap_c, io.cache, d.N * io.cache_slots, d, p);
-    if (st == CCV3D_OK) st = encode_w(&prm.tmap_w, w, d, p);
-    if (st == CCV3D_OK) st = encode_out(&prm.tmap_out, out, d, p);
+    if (st == CCV3D_OK) st = p->thin ? encode_w_thin(&prm.tmap_w, w, d, p) : encode_w(&prm.tmap_w, w, d, p);
+    // two-frame kernel: all kw column taps of a stage in one load (test-gated
+    // A/B switch CCV3D_W_KW=0 keeps one load per column tap)
+    if (st == CCV3D_OK && p->fused && !p->fused_persist && d.kw <= 8 &&
+        !(override_env("CCV3D_W_KW") != nullptr && env_int("CCV3D_W_KW") == 0)) {
+        st = encode_w_kw(&prm.tmap_wkw_full, w, d, p, p->BN);
+        if (st == CCV3D_OK) st = encode_w_kw(&prm.tmap_wkw_half, w, d, p, p->BN / 2);
+        if (st == CCV3D_OK) prm.w_kw_boxes = 1;
+    }
+    // (the thin kernel stores with plain stores: a row of Cout < 8 channels
+    // is no tensor-map stride)
+    if (st == CCV3D_OK && !p->thin) st = encode_out(&prm.tmap_out, out, d, p);
     if (st != CCV3D_OK) return st;
     prm.bias = d.has_bias ? static_cast<const uint16_t*>(bias) : nullptr;
     prm.out = static_cast<uint16_t*>(out);
@@ -802,6 +936,13 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
         p->pair ? 2LL * d.N * p->T_o * prm.pairs_per_frame * p->tiles_n
                 : (long long)d.N * p->T_o * p->tiles_y * p->tiles_x * p->tiles_n;
     if (p->fused) grid = 2LL * d.N * ((p->T_o + 1) / 2) * prm.pairs_per_frame;  // frame pairs
+    if (p->thin) {
+        grid = (long long)d.N * p->tn_groups * p->H_o * p->tiles_x;
+        prm.tn_G = p->tn_G;
+        prm.tn_groups = p->tn_groups;
+        prm.tn_cbk = p->tn_cbk;
+        prm.tn_rows = d.kw * d.Cout;
+    }
     if (p->fused_persist) {
         grid = 2LL * p->G;
         prm.sk.n_acc = p->n_acc;
@@ -829,7 +970,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     const long long units = p->pair ? grid / 2 : grid;
     const long long wave = p->pair ? kSmCount / 2 : kSmCount;
     prm.rot_div = env_int("CCV3D_NO_ROT") ? 0x7fffffff : (int)std::max(1LL, std::min(units, wave));
-    const int kind = p->fused_persist ? 5 : (p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair)));
+    const int kind = p->thin ? 6 : p->fused_persist ? 5 : (p->fused ? 4 : (p->halo ? 3 : (p->persist ? 2 : p->pair)));
     prm.halo_w = p->halo_w;
     cudaError_t e;
     const int threads = p->fused_persist ? fused_persist_threads(p) : kTcpThreads;
@@ -1183,6 +1324,7 @@ const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
         return p->simt_kind == 3 ? "simt_tile"
                                  : (p->simt_kind == 2 ? "simt_smem"
                                                       : (p->simt_kind == 1 ? "simt_warp" : "simt"));
+    if (p->thin) return "tc_thin";
     if (p->fused_persist) return "tc_pair_fused_persistent";
     if (p->fused) return "tc_pair_fused";
     if (p->halo) return "tc_pair_halo";

@@ -226,6 +226,14 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                                  y_out * p.s_h + r * p.d_h - p.p_h, frame);
                 uint8_t* b_base = st_base + kAst;
                 const int wrow = my_tap * p.kh * p.kw + r * p.kw;
+                if (p.w_kw_boxes) {
+                    // one load: kw column taps x (BN or BN/2) rows, [sx][rows][BK]
+                    if (both)
+                        tma_load_3d_pair(smem_u32(b_base), &p.tmap_wkw_full, fb, cb * BK, 0, wrow);
+                    else
+                        tma_load_3d_pair(smem_u32(b_base), &p.tmap_wkw_half, fb, cb * BK,
+                                         (int)rank * hB, wrow);
+                } else
                 for (int sx = 0; sx < p.kw; ++sx) {
                     if (both) {
                         tma_load_3d_pair(smem_u32(b_base + sx * kWt), &p.tmap_w, fb, cb * BK,
@@ -267,10 +275,13 @@ conv_tc2f_kernel(const __grid_constant__ TcParams p) {
                 const uint32_t d_tmem = tmem_base + (src.k0[si] >= 0 ? 0u : (uint32_t)BN);
                 const bool zero = src.zero[si] && j == 0;
                 const uint32_t st_off = (uint32_t)ring.st * (uint32_t)kStage;
+                // weight tile of column tap sx: kWt apart, or, loaded as one
+                // [kw][rows][BK] box, (rows x kRow) apart
+                const int wstride = (p.w_kw_boxes && !both) ? hB * kRow : kWt;
                 for (int sx = 0; sx < p.kw; ++sx) {
                     // A: the strip shifted by sx*d_w pixels (rows)
                     const uint64_t a_desc = d0 + (uint64_t)((st_off + sx * p.d_w * kRow) >> 4);
-                    const uint64_t b_desc = d0 + (uint64_t)((st_off + kAst + sx * kWt) >> 4);
+                    const uint64_t b_desc = d0 + (uint64_t)((st_off + kAst + sx * wstride) >> 4);
                     const bool first = zero && sx == 0;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)

@@ -80,6 +80,12 @@ struct __align__(64) TcParams {
     CUtensorMap tmap_x;      // x      as [N*T_x, H, W, Cin], box [BK, bw*s_w, bh*s_h, 1]
     CUtensorMap tmap_c;      // cache  as [N*|C|, H, W, Cin] (unused when |C| = 0)
     CUtensorMap tmap_w;      // weight as [Cout, kt*kh*kw, Cin], box [BK, 1, BN]
+    // two-frame kernel, one load per stage for all kw column taps: weight as
+    // [taps, Cout, Cin] (dims Cin, Cout, taps), box [BK, rows, kw] -> smem
+    // [kw][rows][BK], the per-tap K-major tiles the MMAs read; rows = BN
+    // (both frames' stages) or BN/2 (one frame's)
+    CUtensorMap tmap_wkw_full, tmap_wkw_half;
+    int w_kw_boxes;          // 1: the two-frame kernel loads weights with the maps above
     CUtensorMap tmap_out;    // out as [N*T_o, H_o, W_o, Cout], box [kCh, box_w, box_h, 1]
     const uint16_t* bias;    // bf16 [Cout] or null
     uint16_t* out;           // bf16 [N, T_o, H_o, W_o, Cout]
@@ -100,6 +106,9 @@ struct __align__(64) TcParams {
     int x_frames, c_frames;  // frames of the x and cache tensor maps (checked build)
     PacedCopy paced;         // persistent kernel: frames of copy.paced_mask
     int H, W;                // input frame extent (the paced copy's regions)
+    // thin-output kernel (conv_tcn.cuh): G output frames per tile in tn_groups
+    // groups, tn_cbk TMEM columns per frame, tn_rows = kw*Cout weight rows per tap
+    int tn_G, tn_groups, tn_cbk, tn_rows;
 };
 
 struct SimtParams {

@@ -80,9 +80,11 @@ def test_planner_shapes_match_oracle_on_workloads(name):
     assert (iv["T_o"], iv["H_o"], iv["W_o"]) == (T_o, H_o, W_o)
     assert (iv["delta"], iv["o_l"], iv["o_h"]) == (delta, o_l, o_h)
     assert plan.sizes["new_cache_frames"] == keep
-    # bf16 workloads with 16-multiple channels take the tensor-core path; fp32
-    # and the 3-channel RGB output conv the SIMT path
-    assert plan.path["tc"] == (c.dtype == "bf16" and c.Cin % 16 == 0 and c.Cout % 16 == 0)
+    # bf16 workloads with 16-multiple input channels take the tensor cores (the
+    # 3-channel RGB output conv the thin-output kernel); fp32 the SIMT path
+    assert plan.path["tc"] == (c.dtype == "bf16" and c.Cin % 16 == 0)
+    if plan.path["tc"] and c.Cout % 16 != 0:
+        assert plan.kernel == "tc_thin"
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -231,6 +233,37 @@ def test_simt_variant_choice():
     assert ccv3d.Plan(ccv3d.desc_for(wide)).kernel == "simt_warp"
     big = workloads.Conv("f32_big", 32, 32, 64, 64, T_x=4, cache_len=2, dtype="fp32")
     assert ccv3d.Plan(ccv3d.desc_for(big)).kernel == "simt"
+
+
+def test_thin_output_kernel_choice():
+    """Outputs too narrow for an MMA's N take the kernel that stacks the
+    temporal and column taps along N, where its conditions hold (unit temporal
+    stride and dilation, unit W stride, kt * (kw * Cout rounded up to 16) <= 256
+    columns); otherwise the SIMT kernels."""
+    from parity_util import plan_env
+    rgb = workloads.C_RGB
+    plan = ccv3d.Plan(ccv3d.desc_for(rgb))
+    assert plan.kernel == "tc_thin"
+    assert plan.path["tile_m"] == 128 and plan.path["tile_n"] == 48  # 3 taps x 16 columns
+    assert plan.tiling["k_block"] == 32  # widest channel block dividing 96
+    with plan_env({"CCV3D_THIN": 0}):
+        assert ccv3d.Plan(ccv3d.desc_for(rgb)).kernel == "simt_tile"
+    with plan_env({"CCV3D_THIN": 1}):  # also for Cout = 16 (tests)
+        c = workloads.Conv("bf16_thin16", 32, 16, 24, 40, T_x=3, cache_len=2)
+        assert ccv3d.Plan(ccv3d.desc_for(c)).kernel == "tc_thin"
+    base = dict(T_x=4, cache_len=2, sigma_b=0.1)
+    # temporal stride 2: output frames do not share the taps' column layout
+    s2 = workloads.Conv("s2", 96, 3, 32, 64, stride_t=2, **base)
+    assert ccv3d.Plan(ccv3d.desc_for(s2)).kernel.startswith("simt")
+    # 3 x (3 x 40 -> 128) columns > 256
+    wide = workloads.Conv("wide", 96, 40, 32, 64, **base)
+    assert ccv3d.Plan(ccv3d.desc_for(wide)).kernel.startswith("simt")
+    # stride 2 along W: the strip is not the output row
+    sw = workloads.Conv("sw2", 96, 3, 32, 64, stride=(1, 2), **base)
+    assert ccv3d.Plan(ccv3d.desc_for(sw)).kernel.startswith("simt")
+    # fp32 and Cin not a multiple of 16 stay on FFMA
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.Conv("f", 96, 3, 32, 64, dtype="fp32", **base))).kernel.startswith("simt")
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.Conv("c8", 8, 3, 32, 64, **base))).kernel.startswith("simt")
 
 
 @pytest.mark.parametrize("kw", [

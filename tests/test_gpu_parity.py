@@ -150,9 +150,12 @@ FUSED = [
 ]
 
 
+@pytest.mark.parametrize("wkw", [1, 0], ids=["w_one_load", "w_load_per_tap"])
 @pytest.mark.parametrize("c", FUSED, ids=lambda c: c.name)
-def test_small_fused_frame_pairs(c):
-    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1})
+def test_small_fused_frame_pairs(c, wkw):
+    """The two-frame kernel, its weights loaded as one [kw][rows][BK] box per
+    stage (default) or one box per column tap."""
+    call, _ = _run_small(c, env={"CCV3D_PERSIST": 0, "CCV3D_FUSE": 1, "CCV3D_W_KW": wkw})
     assert call.plan.kernel == "tc_pair_fused", call.plan.kernel
 
 
@@ -261,7 +264,9 @@ def test_full_size(name):
     inp = inputs_for(c)
     call = GpuCall(c, inp).run()
     torch.cuda.synchronize()
-    assert call.plan.path["tc"] is (c.Cin % 16 == 0 and c.Cout % 16 == 0)
+    assert call.plan.path["tc"] is (c.Cin % 16 == 0)
+    if c.Cout % 16 != 0:
+        assert call.plan.kernel == "tc_thin"
     out = call.out
     if name in SAMPLED_ONLY:
         assert bool(torch.isfinite(out.float()).all())
@@ -408,9 +413,49 @@ SIMT_TILE = [
 @pytest.mark.parametrize("tile", [1, 0], ids=["tile", "thread"])
 @pytest.mark.parametrize("c", SIMT_TILE, ids=lambda c: c.name)
 def test_simt_tile_thin_cout(c, tile):
-    call, _ = _run_small(c, env={"CCV3D_SIMT_TILE": tile})
+    call, _ = _run_small(c, env={"CCV3D_SIMT_TILE": tile, "CCV3D_THIN": 0})
     assert call.plan.path["tc"] is False
     # an fp32 3x3 patch takes more 16-byte loads than a thread holds ahead
     # (10 x 130 pixels x 2): those calls keep the thread kernel
     fits = c.dtype == "bf16" or c.kh * c.kw == 1
     assert call.plan.kernel == ("simt_tile" if tile and fits else "simt"), call.plan.kernel
+
+
+THIN = [
+    # RGB-like 96 -> 3 (channel block 32), ragged last x tile (300 = 2 x 126 + 48)
+    Conv("n96to3_c2_t4", 96, 3, 24, 300, T_x=4, cache_len=2, sigma_b=0.1),
+    # first chunk (no cache), channel block 64
+    Conv("n64to3_c0_t3", 64, 3, 17, 130, T_x=3, cache_len=0),
+    # one output channel, channel block 16
+    Conv("n16to1_c1", 16, 1, 20, 140, T_x=2, cache_len=1),
+    # |C| = 4 > p_l^base: the oldest cached frame is dropped
+    Conv("n32to5_c4_crop", 32, 5, 12, 200, T_x=1, cache_len=4),
+    # 32 TMEM columns per frame: 4 frames per tile, 9 output frames in 3 groups
+    Conv("n48to8_groups", 48, 8, 10, 150, T_x=9, cache_len=2),
+    # spatial dilation 2 (124 outputs per strip) and stride 2 along H
+    Conv("n32to3_dil2", 32, 3, 19, 160, T_x=2, cache_len=2, pad=(2, 2), dilation=(1, 2, 2)),
+    Conv("n32to3_sh2", 32, 3, 21, 150, T_x=2, cache_len=2, stride=(2, 1)),
+    # 3x1x1 and 3x1x3 kernels
+    Conv("n32to3_3x1x1", 32, 3, 16, 140, T_x=3, cache_len=2, kh=1, kw=1, pad=(0, 0)),
+    Conv("n32to6_k3x1x3", 32, 6, 14, 150, T_x=2, cache_len=2, kh=1, kw=3, pad=(0, 1)),
+    # batch 2 without bias; leading bias-only frames; rows with no input row at all
+    Conv("n32to3_batch2_nobias", 32, 3, 10, 140, T_x=2, cache_len=2, N=2, has_bias=False),
+    Conv("n32to3_biasonly", 32, 3, 10, 140, T_x=2, cache_len=0, pad_t_base=4, cache_keep=2),
+    Conv("n32to3_pad3", 32, 3, 9, 140, T_x=2, cache_len=2, pad=(3, 3)),
+]
+
+
+@pytest.mark.parametrize("c", THIN, ids=lambda c: c.name)
+def test_small_thin_output(c):
+    """The thin-output kernel (temporal and column taps stacked along N)
+    against the oracle over the whole output."""
+    call, _ = _run_small(c)
+    assert call.plan.kernel == "tc_thin", call.plan.kernel
+
+
+def test_small_thin_output_forced_cout16():
+    """Cout = 16 on the thin-output kernel (48 TMEM columns per frame, one
+    frame per tile) when forced."""
+    c = Conv("n32to16_thin", 32, 16, 12, 140, T_x=3, cache_len=2)
+    call, _ = _run_small(c, env={"CCV3D_THIN": 1})
+    assert call.plan.kernel == "tc_thin", call.plan.kernel

@@ -9,7 +9,8 @@ Checked through the C ABI on the GPU, call by call, against
   * the FP64 oracle on the same inputs.
 Cases: the 164-call synthetic decode at 16x32; ring sizes from the minimum
 |C| + n_w upwards with the head wrapping; every kernel form (pair, persistent
-with split tiles, halo, frame-pair, single CTA, SIMT fp32 and bf16); the
+with split tiles, halo, frame-pair, single CTA, thin output, SIMT fp32 and
+bf16); the
 full-size stride-2 call.
 """
 import collections
@@ -133,6 +134,7 @@ RING_SIGS = [
     (Conv("r16_fp32", 16, 16, 16, 16, T_x=3, cache_len=0, dtype="fp32", sigma_b=0.1), {}),
     (Conv("r8_fp32_t1", 8, 12, 13, 17, T_x=1, cache_len=0, dtype="fp32"), {}),
     (Conv("r_thin_bf16", 3, 16, 12, 12, T_x=2, cache_len=0), {}),
+    (Conv("r_thin_out_t2", 32, 3, 10, 140, T_x=2, cache_len=0, sigma_b=0.1), {"CCV3D_THIN": 1}),
 ]
 
 
@@ -155,7 +157,7 @@ def test_ring_chunks_every_kernel(sig, env, extra):
         seen += c.T_x
     # the override that forces a kernel form (key, value) -> the form
     forced = {("CCV3D_PAIR", 0): "tc_single", ("CCV3D_HALO", 1): "tc_pair_halo",
-              ("CCV3D_PERSIST", 1): "tc_persistent"}
+              ("CCV3D_PERSIST", 1): "tc_persistent", ("CCV3D_THIN", 1): "tc_thin"}
     if env.get("CCV3D_FUSE") == 1:
         forced[("CCV3D_FUSE", 1)] = ("tc_pair_fused_persistent" if env.get("CCV3D_FUSED_PERSIST")
                                      else "tc_pair_fused")
