@@ -50,7 +50,8 @@ struct ccv3d_plan_s {
     int fused_persist;  // 1: the persistent form of the two-frame kernel (conv_tc2fp.cuh)
     int thin;     // 1: thin-output kernel, taps stacked along N (conv_tcn.cuh)
     int tn_G, tn_groups, tn_cbk;  // thin: frames per tile, frame groups, TMEM columns per frame
-    int simt_kind;  // SIMT plans: 0 thread per unit, 1 warp per unit, 2 shared-memory blocks
+    int simt_kind;  // SIMT plans: 0 thread per unit, 1 warp per unit, 2 shared-memory blocks,
+                    // 3 tiles of thin outputs, 4 warp per pixel for all (<= 16) channels
     int simt_band_h, simt_rows_in, simt_threads;
     size_t simt_smem;
     int G, n_acc;  // persistent: CTA pairs launched, TMEM accumulator buffers
@@ -1016,6 +1017,18 @@ void choose_simt(ccv3d_plan_s* p) {
     // 16-channel fp32 contract call it measured 28.7 us against 18.5 us for
     // one warp per unit (12 blocks cannot hide their staging latency)
     const bool smem_on = env_int("CCV3D_SIMT_SMEM") > 0;
+    // one warp per pixel for all (<= 16) output channels when Cin divides 32
+    // and the weights fit in shared memory (CCV3D_SIMT_W16=0 disables)
+    const bool w16_off = override_env("CCV3D_SIMT_W16") != nullptr && env_int("CCV3D_SIMT_W16") == 0;
+    if (p->simt_kind == 1 && !smem_on && !w16_off && 32 % d.Cin == 0 && d.Cout <= 16) {
+        const size_t bytes = simt_warp16_smem_bytes(d.kt * d.kh * d.kw, d.Cin);
+        if (bytes <= kSimtSmemMax) {
+            p->simt_kind = 4;
+            p->simt_smem = bytes;
+            p->simt_threads = kW16Threads;
+            return;
+        }
+    }
     if (p->simt_kind != 1 || !smem_on) return;
     const int Wp = d.W + 2 * d.pad_w;
     const long long row_units = (long long)p->W_o * ceil_div(d.Cout, kSimtCoT);
@@ -1047,6 +1060,8 @@ void set_simt_smem_attr() {
     }
     if (dev < 0 || dev >= kMaxDevices || done[dev].load(std::memory_order_acquire)) return;
     cudaFuncSetAttribute(conv_simt_smem_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kSimtSmemMax);
+    cudaFuncSetAttribute(conv_simt_warp16_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kSimtSmemMax);
     cudaFuncSetAttribute(conv_simt_tile_kernel<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          113 * 1024);
@@ -1099,6 +1114,27 @@ ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const CacheIO& io, const v
             launch_simt_tile<float>(prm, d.kw, (int)(cb + kb), p->simt_smem, stream);
         else
             launch_simt_tile<__nv_bfloat16>(prm, d.kw, (int)(cb + kb), p->simt_smem, stream);
+        return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
+    }
+    if (p->simt_kind == 4) {
+        prm.co_groups = 1;
+        prm.conv_threads = (long long)d.N * p->T_o * p->H_o * p->W_o;  // pixels
+        const long long cb = (prm.conv_threads * 32 + kW16Threads - 1) / kW16Threads;
+        const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
+        // 8 KB per copy block: two 16-byte vectors per thread, one round of loads
+        const long long kb =
+            copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 8191) / 8192) : 0;
+        if (cb + kb > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
+        prm.conv_blocks = (int)cb;
+        prm.copy_blocks = (int)kb;
+        const int grid = (int)(cb + kb);
+        if (d.dtype == CCV3D_FP32) {
+            set_simt_smem_attr<float>();
+            conv_simt_warp16_kernel<float><<<grid, kW16Threads, p->simt_smem, stream>>>(prm);
+        } else {
+            set_simt_smem_attr<__nv_bfloat16>();
+            conv_simt_warp16_kernel<__nv_bfloat16><<<grid, kW16Threads, p->simt_smem, stream>>>(prm);
+        }
         return cudaGetLastError() == cudaSuccess ? CCV3D_OK : CCV3D_ERR_CUDA;
     }
     if (p->simt_kind == 2) {
@@ -1321,7 +1357,8 @@ int ccv3d_plan_path(ccv3d_plan_t p, int* tile_m, int* tile_n) {
 const char* ccv3d_plan_kernel(ccv3d_plan_t p) {
     if (p == nullptr) return "";
     if (!p->path_tc)
-        return p->simt_kind == 3 ? "simt_tile"
+        return p->simt_kind == 4 ? "simt_warp16"
+               : p->simt_kind == 3 ? "simt_tile"
                                  : (p->simt_kind == 2 ? "simt_smem"
                                                       : (p->simt_kind == 1 ? "simt_warp" : "simt"));
     if (p->thin) return "tc_thin";

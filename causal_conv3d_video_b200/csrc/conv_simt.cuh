@@ -321,6 +321,188 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
     }
 }
 
+// Small calls whose Cin divides 32 and whose Cout <= 16 (the 16-channel fp32
+// contract call): one warp per output pixel computes every output channel.
+// A lane owns (tap offset, input channel) as in conv_simt_warp_kernel and
+// walks the taps 32 / Cin apart.  The block first stages the weights in
+// shared memory as fp32 rows [(tap, ci)][co] of kW16Stride floats (16
+// channels, zero past Cout, and 4 floats of padding so that the 16-byte reads
+// of the 8 lanes of a phase fall in distinct banks); a reduction step is then
+// one input load, four 16-byte shared loads and 16 FMAs.  The lanes' 16
+// partial sums are combined by recursive halving (each shuffle step hands the
+// partner the half of the channels it keeps): 16 shuffles leave every even
+// lane with one channel's total.  conv_threads counts pixels here.
+constexpr int kW16Stride = 20;
+constexpr int kW16Threads = 256;
+
+__host__ __device__ constexpr size_t simt_warp16_smem_bytes(int taps, int cin) {
+    return (size_t)taps * cin * kW16Stride * sizeof(float);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kW16Threads)
+conv_simt_warp16_kernel(const __grid_constant__ SimtParams p) {
+    if ((int)blockIdx.x >= p.conv_blocks) {
+        copy_new_cache(p.copy, blockIdx.x - p.conv_blocks, p.copy_blocks, threadIdx.x,
+                       blockDim.x);
+        return;
+    }
+    extern __shared__ float4 w16_smem[];
+    float* ws = reinterpret_cast<float*>(w16_smem);
+    const T* w = static_cast<const T*>(p.w);
+    const int taps2d = p.kh * p.kw;
+    const int ntaps = p.taps.kt * taps2d;
+    const int K = ntaps * p.Cin;  // weight rows (tap, ci)
+    // this warp's pixel (warps past the last pixel still help stage the weights)
+    const int unit = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    const bool live = unit < p.conv_threads;
+    int pix = live ? unit : 0;
+    const int xo = pix % p.W_o;
+    pix /= p.W_o;
+    const int yo = pix % p.H_o;
+    pix /= p.H_o;
+    const int o = pix % p.T_o;
+    const int n = pix / p.T_o;
+
+    const T* x = static_cast<const T*>(p.x);
+    const T* cache = static_cast<const T*>(p.cache);
+    const T* fb[kMaxTaps];
+    bool act[kMaxTaps], fc[kMaxTaps];  // tap active; its frame is in the cache
+#pragma unroll
+    for (int k = 0; k < kMaxTaps; ++k) {
+        act[k] = k < p.taps.kt && o >= p.taps.o_l[k] && o < p.taps.o_h[k];
+        const int tf = o * p.taps.s_t + p.taps.delta[k];
+        fc[k] = act[k] && tf < p.cache_len;
+        fb[k] = !act[k] ? x
+                        : (fc[k] ? cache + (long long)ring_frame(n, tf, p.cache_slots,
+                                                                 p.cache_head) *
+                                               p.H * p.W * p.Cin
+                                 : x + ((long long)n * p.T_x + (tf - p.cache_len)) * p.H * p.W *
+                                           p.Cin);
+    }
+    const long long cache_bytes = p.copy.cache_bytes, x_bytes = p.copy.x_bytes;
+    const int tpi = 32 / p.Cin, ci = lane % p.Cin;
+    const int ybase = yo * p.s_h - p.p_h, xbase = xo * p.s_w - p.p_w;
+    int t = live ? lane / p.Cin : ntaps;
+    int k = t / taps2d, r = (t - k * taps2d) / p.kw, sx = t - k * taps2d - r * p.kw;
+    // kZ reduction steps at a time: their input loads are issued together
+    // (the first batch before the weight staging, so that both wait out one
+    // round of load latency together), then their FMAs run
+    constexpr int kZ = 16;
+    float z[kZ];
+    int tt[kZ];
+    auto load_batch = [&]() {
+#pragma unroll
+        for (int u = 0; u < kZ; ++u) {
+            z[u] = 0.f;
+            tt[u] = -1;
+            if (t < ntaps) {
+                tt[u] = t;
+                const int yi = ybase + r * p.d_h, xi = xbase + sx * p.d_w;
+                const T* f = k == 0 ? fb[0] : (k == 1 ? fb[1] : fb[2]);
+                const bool a = k == 0 ? act[0] : (k == 1 ? act[1] : act[2]);
+                if (a && (unsigned)yi < (unsigned)p.H && (unsigned)xi < (unsigned)p.W) {
+                    const T* zp = f + (yi * p.W + xi) * p.Cin + ci;
+                    const bool c = k == 0 ? fc[0] : (k == 1 ? fc[1] : fc[2]);
+                    if (in_bounds(p.status, zp, sizeof(T),
+                                  c ? (const void*)cache : (const void*)x,
+                                  c ? cache_bytes : x_bytes))
+                        z[u] = to_f32<T>(__ldg(zp));
+                }
+                t += tpi;
+                for (int q = 0; q < tpi; ++q)  // next tap of this lane
+                    if (++sx == p.kw) {
+                        sx = 0;
+                        if (++r == p.kh) {
+                            r = 0;
+                            ++k;
+                        }
+                    }
+            }
+        }
+    };
+    load_batch();
+
+    // stage: a thread takes (tap, ci) rows, loads each for all 16 channels at
+    // once (for each channel, consecutive threads read consecutive positions)
+    // and writes it with four 16-byte stores (consecutive threads, consecutive
+    // rows: no bank conflicts); two rows per thread per round of loads
+    const long long w_bytes = p.w_floats * (long long)sizeof(T);
+    for (int kc0 = threadIdx.x; kc0 < K; kc0 += 2 * kW16Threads) {
+        float v[2][16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int kc = kc0 + h * kW16Threads;
+#pragma unroll
+            for (int co = 0; co < 16; ++co) {
+                v[h][co] = 0.f;
+                const T* src = w + (long long)co * K + kc;
+                if (kc < K && co < p.Cout && in_bounds(p.status, src, sizeof(T), w, w_bytes))
+                    v[h][co] = to_f32<T>(__ldg(src));
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int kc = kc0 + h * kW16Threads;
+            if (kc >= K) break;
+            float4* row = reinterpret_cast<float4*>(ws + kc * kW16Stride);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                row[q] = make_float4(v[h][4 * q], v[h][4 * q + 1], v[h][4 * q + 2],
+                                     v[h][4 * q + 3]);
+        }
+    }
+    __syncthreads();
+    if (!live) return;  // whole warps leave together
+
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    for (;;) {
+#pragma unroll
+        for (int u = 0; u < kZ; ++u) {
+            if (tt[u] < 0) continue;
+            const float4* wr =
+                reinterpret_cast<const float4*>(ws + (tt[u] * p.Cin + ci) * kW16Stride);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 wv = wr[q];
+                acc[4 * q + 0] = fmaf(z[u], wv.x, acc[4 * q + 0]);
+                acc[4 * q + 1] = fmaf(z[u], wv.y, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(z[u], wv.z, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(z[u], wv.w, acc[4 * q + 3]);
+            }
+        }
+        if (t >= ntaps) break;
+        load_batch();
+    }
+    // recursive halving: after the step of offset 16 >> s a lane holds 8 >> s
+    // channels, the upper or lower half of those it held, summed with its
+    // partner's
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const int off = 16 >> s, h = 8 >> s;
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = up ? acc[i] : acc[i + h];
+            const float keep = up ? acc[i + h] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+    const int co = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                   ((lane >> 1) & 1);
+    if ((lane & 1) != 0 || co >= p.Cout) return;
+    const long long oi = ((((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo) * p.Cout + co;
+    if (!index_ok(p.status, oi, p.out_elems)) return;
+    float v = acc[0];
+    const T* bias = static_cast<const T*>(p.bias);
+    if (bias != nullptr) v += to_f32<T>(bias[co]);
+    static_cast<T*>(p.out)[oi] = from_f32<T>(v);
+}
+
 // Small calls (a few thousand (pixel, 4-channel) units, e.g. the 16-channel
 // fp32 contract call): one block per (output frame, band of band_h output
 // rows).  The block first stages, as fp32 in shared memory and with 16-byte

@@ -132,8 +132,8 @@ typedef struct ccv3d_plan_s* ccv3d_plan_t;
  * The kernel and tiling are the planner's own choice.  Environment variables
  * CCV3D_PERSIST, CCV3D_HALO, CCV3D_FUSE, CCV3D_PAIR, CCV3D_TILE_N,
  * CCV3D_STAGES, CCV3D_BOX_W, CCV3D_HALO_BK, CCV3D_SK_PAIRS, CCV3D_NO_ROT,
- * CCV3D_SIMT_SMEM, CCV3D_SIMT_TILE, CCV3D_PACED, CCV3D_FUSED_PERSIST and
- * CCV3D_FORCE_PATH=simt
+ * CCV3D_SIMT_SMEM, CCV3D_SIMT_TILE, CCV3D_SIMT_W16, CCV3D_THIN, CCV3D_W_KW,
+ * CCV3D_PACED, CCV3D_FUSED_PERSIST and CCV3D_FORCE_PATH=simt
  * override it for tests and tuning
  * sweeps, and are read only when CCV3D_TEST_OVERRIDES=1 is also set.
  *
@@ -169,8 +169,14 @@ CCV3D_API int ccv3d_plan_path(ccv3d_plan_t plan, int* tile_m, int* tile_n);
  *                    pair walking the tiles, double-buffered accumulators
  *   "tc_persistent"  persistent stream-K over all SM pairs
  *   "tc_single"      one CTA per tile
+ *   "tc_thin"        one CTA per (output row, group of output frames) for
+ *                    outputs too narrow for an MMA's N (Cout not a multiple of
+ *                    16): the temporal and column taps stacked along N, the
+ *                    column taps summed in the epilogue
  *   "simt"           FFMA, one thread per pixel and 4 output channels
  *   "simt_warp"      FFMA, one warp per pixel and 4 output channels (small calls)
+ *   "simt_warp16"    FFMA, one warp per pixel and all (<= 16) output channels,
+ *                    weights staged in shared memory (small calls, Cin | 32)
  *   "simt_smem"      FFMA, one block per band of output rows with the weights
  *                    and input rows staged in shared memory (small calls that fit)
  *   "simt_tile"      FFMA, large calls with <= 4 output channels: 8 x 128-pixel

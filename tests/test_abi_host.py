@@ -224,10 +224,18 @@ def test_quantize_validation_without_gpu():
 def test_simt_variant_choice():
     """Calls too small for one thread per (pixel, 4 channels) to fill the SMs
     run one warp per unit (the lanes split the reduction)."""
-    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
+    # Cin = 16 divides 32 and Cout = 16: one warp per pixel for all channels
+    assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp16"
     from parity_util import plan_env
+    with plan_env({"CCV3D_SIMT_W16": 0}):
+        assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_warp"
     with plan_env({"CCV3D_SIMT_SMEM": 1}):  # the shared-memory kernel is opt-in
         assert ccv3d.Plan(ccv3d.desc_for(workloads.C1)).kernel == "simt_smem"
+    # 17 output channels, or Cin = 12 (does not divide 32): 4 channels per warp
+    c17 = workloads.Conv("f32_17", 16, 17, 16, 16, T_x=3, cache_len=2, dtype="fp32")
+    assert ccv3d.Plan(ccv3d.desc_for(c17)).kernel == "simt_warp"
+    c12 = workloads.Conv("f32_12", 12, 16, 16, 16, T_x=3, cache_len=2, dtype="fp32")
+    assert ccv3d.Plan(ccv3d.desc_for(c12)).kernel == "simt_warp"
     # weights of 384 -> 384 x 27 fp32 (15.9 MB) do not fit in shared memory
     wide = workloads.Conv("f32_wide", 384, 384, 4, 4, T_x=1, cache_len=2, dtype="fp32")
     assert ccv3d.Plan(ccv3d.desc_for(wide)).kernel == "simt_warp"

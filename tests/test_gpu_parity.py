@@ -72,9 +72,10 @@ def _run_small(c, force_simt=False, env=None):
     return call, m
 
 
-@pytest.mark.parametrize("smem,kernel", [(1, "simt_smem"), (0, "simt_warp")])
-def test_config1_fp32_exact_workload(smem, kernel):
-    call, m = _run_small(workloads.C1, env={"CCV3D_SIMT_SMEM": smem})
+@pytest.mark.parametrize("smem,w16,kernel", [(1, 1, "simt_smem"), (0, 0, "simt_warp"),
+                                              (0, 1, "simt_warp16")])
+def test_config1_fp32_exact_workload(smem, w16, kernel):
+    call, m = _run_small(workloads.C1, env={"CCV3D_SIMT_SMEM": smem, "CCV3D_SIMT_W16": w16})
     assert call.plan.path["tc"] is False
     assert call.plan.kernel == kernel
     assert call.plan.stats()["simt_path"] == 1
@@ -233,7 +234,8 @@ def test_small_simt_bf16(c, smem):
     if units >= 148 * 128:
         assert call.plan.kernel == "simt"
     else:
-        assert call.plan.kernel in (("simt_smem", "simt_warp") if smem else ("simt_warp",))
+        assert call.plan.kernel in (("simt_smem", "simt_warp") if smem
+                                    else ("simt_warp", "simt_warp16"))
 
 
 @pytest.mark.parametrize("c", [
@@ -442,6 +444,8 @@ THIN = [
     Conv("n32to3_batch2_nobias", 32, 3, 10, 140, T_x=2, cache_len=2, N=2, has_bias=False),
     Conv("n32to3_biasonly", 32, 3, 10, 140, T_x=2, cache_len=0, pad_t_base=4, cache_keep=2),
     Conv("n32to3_pad3", 32, 3, 9, 140, T_x=2, cache_len=2, pad=(3, 3)),
+    # six channel blocks of 32, Cout = 8 (32 TMEM columns per frame)
+    Conv("n192to8", 192, 8, 7, 140, T_x=2, cache_len=2),
 ]
 
 
@@ -459,3 +463,26 @@ def test_small_thin_output_forced_cout16():
     c = Conv("n32to16_thin", 32, 16, 12, 140, T_x=3, cache_len=2)
     call, _ = _run_small(c, env={"CCV3D_THIN": 1})
     assert call.plan.kernel == "tc_thin", call.plan.kernel
+
+
+WARP16 = [
+    # one warp per pixel for all output channels (Cin divides 32, Cout <= 16)
+    Conv("w16_f32_c2_t3", 16, 16, 16, 16, T_x=3, cache_len=2, dtype="fp32", sigma_b=0.1),
+    Conv("w16_f32_8to5_c0", 8, 5, 13, 19, T_x=2, cache_len=0, dtype="fp32"),
+    Conv("w16_f32_32to12_c4_crop", 32, 12, 9, 11, T_x=1, cache_len=4, dtype="fp32"),
+    Conv("w16_f32_4to16_dil", 4, 16, 12, 14, T_x=2, cache_len=2, pad=(2, 2),
+         dilation=(2, 2, 2), dtype="fp32"),
+    Conv("w16_f32_16to3_s2", 16, 3, 17, 15, T_x=2, cache_len=1, stride=(2, 2), dtype="fp32",
+         has_bias=False),
+    Conv("w16_f32_2to7_3x1x1_b2", 2, 7, 10, 12, T_x=3, cache_len=2, kh=1, kw=1, pad=(0, 0),
+         N=2, dtype="fp32"),
+    Conv("w16_bf16_16to8", 16, 8, 14, 18, T_x=2, cache_len=2, sigma_b=0.1, dtype="bf16"),
+    Conv("w16_f32_biasonly", 8, 8, 10, 12, T_x=2, cache_len=0, pad_t_base=4, cache_keep=2,
+         dtype="fp32"),
+]
+
+
+@pytest.mark.parametrize("c", WARP16, ids=lambda c: c.name)
+def test_small_simt_warp16(c):
+    call, _ = _run_small(c, force_simt=True)
+    assert call.plan.kernel == "simt_warp16", call.plan.kernel
