@@ -1119,11 +1119,11 @@ ccv3d_status run_simt(ccv3d_plan_s* p, const void* x, const CacheIO& io, const v
     if (p->simt_kind == 4) {
         prm.co_groups = 1;
         prm.conv_threads = (long long)d.N * p->T_o * p->H_o * p->W_o;  // pixels
-        const long long cb = (prm.conv_threads * 32 + kW16Threads - 1) / kW16Threads;
+        const long long cb = (prm.conv_threads + kW16Pixels - 1) / kW16Pixels;
         const long long copy_bytes = (long long)prm.copy.keep * d.N * prm.copy.frame_bytes;
-        // 8 KB per copy block: two 16-byte vectors per thread, one round of loads
+        // 16 KB per copy block: two 16-byte vectors per thread, one round of loads
         const long long kb =
-            copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 8191) / 8192) : 0;
+            copy_bytes > 0 ? std::min<long long>(1184, (copy_bytes + 16383) / 16384) : 0;
         if (cb + kb > 0x7fffffffLL) return CCV3D_ERR_UNSUPPORTED;
         prm.conv_blocks = (int)cb;
         prm.copy_blocks = (int)kb;

@@ -322,21 +322,28 @@ conv_simt_warp_kernel(const __grid_constant__ SimtParams p) {
 }
 
 // Small calls whose Cin divides 32 and whose Cout <= 16 (the 16-channel fp32
-// contract call): one warp per output pixel computes every output channel.
-// A lane owns (tap offset, input channel) as in conv_simt_warp_kernel and
-// walks the taps 32 / Cin apart.  The block first stages the weights in
-// shared memory as fp32 rows [(tap, ci)][co] of kW16Stride floats (16
-// channels, zero past Cout, and 4 floats of padding so that the 16-byte reads
-// of the 8 lanes of a phase fall in distinct banks); a reduction step is then
-// one input load, four 16-byte shared loads and 16 FMAs.  The lanes' 16
-// partial sums are combined by recursive halving (each shuffle step hands the
-// partner the half of the channels it keeps): 16 shuffles leave every even
-// lane with one channel's total.  conv_threads counts pixels here.
+// contract call): two warps per output pixel compute every output channel.
+// A lane owns (tap offset, input channel): the 64 lanes of a pixel's two warps
+// take taps 64 / Cin apart.  The block first stages, in shared memory, the
+// weights as fp32 rows [(tap, ci)][co] of kW16Stride floats (16 channels,
+// zero past Cout, and 4 floats of padding so that the 16-byte reads of the 8
+// lanes of a phase fall in distinct banks) and a table of each tap's
+// (temporal tap, row offset, column offset); a reduction step is then one
+// table read, one input load, four 16-byte shared loads and 16 FMAs.  Each
+// warp combines its lanes' 16 partial sums by recursive halving (each shuffle
+// step hands the partner the half of the channels it keeps): 16 shuffles
+// leave every even lane one channel's total; the second warp of a pixel hands
+// its totals to the first through shared memory.  The first batch of input
+// loads is issued before the staging, so both wait out one round of load
+// latency together.  conv_threads counts pixels here.
 constexpr int kW16Stride = 20;
-constexpr int kW16Threads = 256;
+constexpr int kW16Threads = 512;               // 8 pixels x 2 warps
+constexpr int kW16Pixels = kW16Threads / 64;
 
 __host__ __device__ constexpr size_t simt_warp16_smem_bytes(int taps, int cin) {
-    return (size_t)taps * cin * kW16Stride * sizeof(float);
+    return (size_t)taps * cin * kW16Stride * sizeof(float)  // weights
+           + (size_t)taps * sizeof(int4)                      // tap table
+           + (size_t)kW16Pixels * 16 * sizeof(float);         // second warps' totals
 }
 
 template <typename T>
@@ -348,14 +355,18 @@ conv_simt_warp16_kernel(const __grid_constant__ SimtParams p) {
         return;
     }
     extern __shared__ float4 w16_smem[];
-    float* ws = reinterpret_cast<float*>(w16_smem);
     const T* w = static_cast<const T*>(p.w);
     const int taps2d = p.kh * p.kw;
     const int ntaps = p.taps.kt * taps2d;
     const int K = ntaps * p.Cin;  // weight rows (tap, ci)
-    // this warp's pixel (warps past the last pixel still help stage the weights)
-    const int unit = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-    const int lane = threadIdx.x & 31;
+    float* ws = reinterpret_cast<float*>(w16_smem);
+    int4* tap_tab = reinterpret_cast<int4*>(ws + (size_t)K * kW16Stride);
+    float* red = reinterpret_cast<float*>(tap_tab + ntaps);
+
+    // this warp's pixel and half (warps past the last pixel still help stage)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = warp & 1, pl = warp >> 1;  // pixel of the block
+    const int unit = (int)blockIdx.x * kW16Pixels + pl;
     const bool live = unit < p.conv_threads;
     int pix = live ? unit : 0;
     const int xo = pix % p.W_o;
@@ -382,79 +393,65 @@ conv_simt_warp16_kernel(const __grid_constant__ SimtParams p) {
                                            p.Cin);
     }
     const long long cache_bytes = p.copy.cache_bytes, x_bytes = p.copy.x_bytes;
-    const int tpi = 32 / p.Cin, ci = lane % p.Cin;
+    const int tpi = 64 / p.Cin, ci = lane % p.Cin;
     const int ybase = yo * p.s_h - p.p_h, xbase = xo * p.s_w - p.p_w;
-    int t = live ? lane / p.Cin : ntaps;
-    int k = t / taps2d, r = (t - k * taps2d) / p.kw, sx = t - k * taps2d - r * p.kw;
-    // kZ reduction steps at a time: their input loads are issued together
-    // (the first batch before the weight staging, so that both wait out one
-    // round of load latency together), then their FMAs run
-    constexpr int kZ = 16;
+    // first tap of this lane, then every tpi-th; (k, r, s) of the first ones
+    // by division here, of the rest from the table after the staging
+    int t = live ? half * (32 / p.Cin) + lane / p.Cin : ntaps;
+    constexpr int kZ = 8;
     float z[kZ];
-    int tt[kZ];
-    auto load_batch = [&]() {
-#pragma unroll
-        for (int u = 0; u < kZ; ++u) {
-            z[u] = 0.f;
-            tt[u] = -1;
-            if (t < ntaps) {
-                tt[u] = t;
-                const int yi = ybase + r * p.d_h, xi = xbase + sx * p.d_w;
-                const T* f = k == 0 ? fb[0] : (k == 1 ? fb[1] : fb[2]);
-                const bool a = k == 0 ? act[0] : (k == 1 ? act[1] : act[2]);
-                if (a && (unsigned)yi < (unsigned)p.H && (unsigned)xi < (unsigned)p.W) {
-                    const T* zp = f + (yi * p.W + xi) * p.Cin + ci;
-                    const bool c = k == 0 ? fc[0] : (k == 1 ? fc[1] : fc[2]);
-                    if (in_bounds(p.status, zp, sizeof(T),
-                                  c ? (const void*)cache : (const void*)x,
-                                  c ? cache_bytes : x_bytes))
-                        z[u] = to_f32<T>(__ldg(zp));
-                }
-                t += tpi;
-                for (int q = 0; q < tpi; ++q)  // next tap of this lane
-                    if (++sx == p.kw) {
-                        sx = 0;
-                        if (++r == p.kh) {
-                            r = 0;
-                            ++k;
-                        }
-                    }
-            }
+    auto load_step = [&](int u, int tap, int k, int dy, int dx) {
+        z[u] = 0.f;
+        const int yi = ybase + dy, xi = xbase + dx;
+        const T* f = k == 0 ? fb[0] : (k == 1 ? fb[1] : fb[2]);
+        const bool a = k == 0 ? act[0] : (k == 1 ? act[1] : act[2]);
+        if (tap < ntaps && a && (unsigned)yi < (unsigned)p.H && (unsigned)xi < (unsigned)p.W) {
+            const T* zp = f + (yi * p.W + xi) * p.Cin + ci;
+            const bool c = k == 0 ? fc[0] : (k == 1 ? fc[1] : fc[2]);
+            if (in_bounds(p.status, zp, sizeof(T), c ? (const void*)cache : (const void*)x,
+                          c ? cache_bytes : x_bytes))
+                z[u] = to_f32<T>(__ldg(zp));
         }
     };
-    load_batch();
-
-    // stage: a thread takes (tap, ci) rows, loads each for all 16 channels at
-    // once (for each channel, consecutive threads read consecutive positions)
-    // and writes it with four 16-byte stores (consecutive threads, consecutive
-    // rows: no bank conflicts); two rows per thread per round of loads
-    const long long w_bytes = p.w_floats * (long long)sizeof(T);
-    for (int kc0 = threadIdx.x; kc0 < K; kc0 += 2 * kW16Threads) {
-        float v[2][16];
+    {  // first batch: the first tap decoded by division, the next ones stepped
+        int k = t / taps2d, rs = t - k * taps2d, r = rs / p.kw, sx = rs - r * p.kw;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int kc = kc0 + h * kW16Threads;
-#pragma unroll
-            for (int co = 0; co < 16; ++co) {
-                v[h][co] = 0.f;
-                const T* src = w + (long long)co * K + kc;
-                if (kc < K && co < p.Cout && in_bounds(p.status, src, sizeof(T), w, w_bytes))
-                    v[h][co] = to_f32<T>(__ldg(src));
+        for (int u = 0; u < kZ; ++u) {
+            load_step(u, t + u * tpi, k, r * p.d_h, sx * p.d_w);
+            sx += tpi;  // advance (k, r, s) by tpi taps
+            while (sx >= p.kw) {
+                sx -= p.kw;
+                if (++r == p.kh) {
+                    r = 0;
+                    ++k;
+                }
             }
         }
+    }
+
+    // stage the weights (a thread takes a (tap, ci) row for all 16 channels:
+    // consecutive threads read consecutive positions of a channel and write
+    // consecutive rows) and the tap table
+    const long long w_bytes = p.w_floats * (long long)sizeof(T);
+    for (int kc = threadIdx.x; kc < K; kc += kW16Threads) {
+        float v[16];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int kc = kc0 + h * kW16Threads;
-            if (kc >= K) break;
-            float4* row = reinterpret_cast<float4*>(ws + kc * kW16Stride);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                row[q] = make_float4(v[h][4 * q], v[h][4 * q + 1], v[h][4 * q + 2],
-                                     v[h][4 * q + 3]);
+        for (int co = 0; co < 16; ++co) {
+            v[co] = 0.f;
+            const T* src = w + (long long)co * K + kc;
+            if (co < p.Cout && in_bounds(p.status, src, sizeof(T), w, w_bytes))
+                v[co] = to_f32<T>(__ldg(src));
         }
+        float4* row = reinterpret_cast<float4*>(ws + kc * kW16Stride);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            row[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+    for (int tp = threadIdx.x; tp < ntaps; tp += kW16Threads) {
+        const int k = tp / taps2d, rs = tp - k * taps2d, r = rs / p.kw, sx = rs - r * p.kw;
+        tap_tab[tp] = make_int4(k, r * p.d_h, sx * p.d_w, 0);
     }
     __syncthreads();
-    if (!live) return;  // whole warps leave together
 
     float acc[16];
 #pragma unroll
@@ -462,9 +459,9 @@ conv_simt_warp16_kernel(const __grid_constant__ SimtParams p) {
     for (;;) {
 #pragma unroll
         for (int u = 0; u < kZ; ++u) {
-            if (tt[u] < 0) continue;
-            const float4* wr =
-                reinterpret_cast<const float4*>(ws + (tt[u] * p.Cin + ci) * kW16Stride);
+            const int tap = t + u * tpi;
+            if (tap >= ntaps) break;  // a lane's taps increase with u
+            const float4* wr = reinterpret_cast<const float4*>(ws + (tap * p.Cin + ci) * kW16Stride);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 wv = wr[q];
@@ -474,8 +471,14 @@ conv_simt_warp16_kernel(const __grid_constant__ SimtParams p) {
                 acc[4 * q + 3] = fmaf(z[u], wv.w, acc[4 * q + 3]);
             }
         }
+        t += kZ * tpi;
         if (t >= ntaps) break;
-        load_batch();
+#pragma unroll
+        for (int u = 0; u < kZ; ++u) {  // next batch: taps from the table
+            const int tap = t + u * tpi;
+            const int4 e = tap < ntaps ? tap_tab[tap] : make_int4(0, 0, 0, 0);
+            load_step(u, tap, e.x, e.y, e.z);
+        }
     }
     // recursive halving: after the step of offset 16 >> s a lane holds 8 >> s
     // channels, the upper or lower half of those it held, summed with its
@@ -494,10 +497,12 @@ conv_simt_warp16_kernel(const __grid_constant__ SimtParams p) {
     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
     const int co = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
                    ((lane >> 1) & 1);
-    if ((lane & 1) != 0 || co >= p.Cout) return;
+    if (half == 1 && (lane & 1) == 0) red[pl * 16 + co] = acc[0];
+    __syncthreads();
+    if (!live || half == 1 || (lane & 1) != 0 || co >= p.Cout) return;
     const long long oi = ((((long long)n * p.T_o + o) * p.H_o + yo) * p.W_o + xo) * p.Cout + co;
     if (!index_ok(p.status, oi, p.out_elems)) return;
-    float v = acc[0];
+    float v = acc[0] + red[pl * 16 + co];
     const T* bias = static_cast<const T*>(p.bias);
     if (bias != nullptr) v += to_f32<T>(bias[co]);
     static_cast<T*>(p.out)[oi] = from_f32<T>(v);
