@@ -735,13 +735,18 @@ ccv3d_status encode_w_thin(CUtensorMap* m, const void* base, const ccv3d_desc& d
 // stores: boxes of (16/32/64 channels) x box_w x box_h pixels of one frame,
 // swizzled like the staging buffer; rows and channels past the tensor are
 // clipped by the hardware.
-ccv3d_status encode_out(CUtensorMap* m, void* base, const ccv3d_desc& d, const ccv3d_plan_s* p) {
+// per_warp: the box of one warp's 32 pixels of a box (the pair kernel's
+// per-warp epilogue), [kCh, min(32, box_w), max(1, 32 / box_w), 1].
+ccv3d_status encode_out(CUtensorMap* m, void* base, const ccv3d_desc& d, const ccv3d_plan_s* p,
+                        bool per_warp = false) {
     const int kch = out_block_channels(p->BN);
     const cuuint64_t dims[4] = {(cuuint64_t)d.Cout, (cuuint64_t)p->W_o, (cuuint64_t)p->H_o,
                                 (cuuint64_t)d.N * p->T_o};
     const cuuint64_t strides[3] = {(cuuint64_t)d.Cout * 2, (cuuint64_t)p->W_o * d.Cout * 2,
                                    (cuuint64_t)p->H_o * p->W_o * d.Cout * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)kch, (cuuint32_t)p->box_w, (cuuint32_t)p->box_h, 1};
+    const int bw = per_warp ? std::min(32, p->box_w) : p->box_w;
+    const int bh = per_warp ? std::max(1, 32 / p->box_w) : p->box_h;
+    const cuuint32_t box[4] = {(cuuint32_t)kch, (cuuint32_t)bw, (cuuint32_t)bh, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapSwizzle sw = kch == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : kch == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -910,6 +915,7 @@ ccv3d_status run_tc(ccv3d_plan_s* p, const void* x, const CacheIO& io, const voi
     // (the thin kernel stores with plain stores: a row of Cout < 8 channels
     // is no tensor-map stride)
     if (st == CCV3D_OK && !p->thin) st = encode_out(&prm.tmap_out, out, d, p);
+    if (st == CCV3D_OK && !p->thin) st = encode_out(&prm.tmap_out_w, out, d, p, true);
     if (st != CCV3D_OK) return st;
     prm.bias = d.has_bias ? static_cast<const uint16_t*>(bias) : nullptr;
     prm.out = static_cast<uint16_t*>(out);

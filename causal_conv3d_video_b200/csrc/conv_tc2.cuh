@@ -88,6 +88,42 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
         if (k < p.taps.kt && o >= p.taps.o_l[k] && o < p.taps.o_h[k]) ++n_active;
     const int iters = n_active * p.kh * p.kw * p.n_cb;
 
+    if (warp == 2) {
+        // An epilogue warp (idle until the accumulator is complete) arrives
+        // at the pair's rendezvous at once -- the set-up needs nothing from
+        // it -- and its lane 0 then fetches the first stages' operand boxes
+        // into L2 while thread 0 and warp 1 set up (barriers, TMEM), so that
+        // the launch's first DRAM round trip overlaps the set-up; the
+        // producer's loads of these stages then hit L2.
+        cluster_arrive();
+        if (lane == 0 && iters > 0) {
+            int act[kMaxTaps];
+            const int n_act = active_tap_list(p, o, act);
+            const int rot = (int)(((long long)pair * iters) / p.rot_div) % iters;
+            const int ybase = ty * p.box_h * p.s_h - p.p_h;
+            const int xbase = tx * p.box_w * p.s_w - p.p_w;
+            KWalk w;
+            w.set(rot, p);
+            TapSrc ts = tap_source(p, act[w.ti], n, o);
+            const int first = stages < iters ? stages : iters;
+            for (int it = 0; it < first; ++it) {
+                // (start coordinates kept inside the frame: a prefetch only
+                // warms L2, so a box shifted off the padding is as good)
+                const int xp = min(max(xbase + w.s * p.d_w, 0), p.W - 1);
+                const int yp = min(max(ybase + w.r * p.d_h, 0), p.H - 1);
+                tma_prefetch_l2_4d(ts.map, w.cb * BK, xp, yp, ts.frame);
+                const int wrow = ts.wtap + w.r * p.kw + w.s;
+                for (int j = 0; j < p.n_sub; ++j)
+                    tma_prefetch_l2_3d(&p.tmap_w, w.cb * BK, wrow,
+                                       n_tile * BN + j * BNs + (int)rank * hB);
+                if (w.next(p)) {
+                    if (w.ti == n_act) w.ti = 0;
+                    ts = tap_source(p, act[w.ti], n, o);
+                }
+            }
+        }
+        __syncwarp();
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
@@ -103,17 +139,11 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
         tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
         tmem_relinquish_pair();
     }
-    if (warp >= 2) {
-        for (int i = threadIdx.x - 64; i < BN; i += 128) {
-            const int co = n_tile * BN + i;
-            float b = 0.f;
-            if (p.bias != nullptr && co < p.Cout && index_ok(p.status, co, p.Cout))
-                b = __bfloat162float(__ushort_as_bfloat16(p.bias[co]));
-            bias_s[i] = b;
-        }
-    }
     tc_fence_before();
-    cluster_sync();  // barriers initialised in both CTAs before any remote use
+    // barriers initialised in both CTAs before any remote use (warp 2 has
+    // arrived already)
+    if (warp != 2) cluster_arrive();
+    cluster_wait();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -181,8 +211,18 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
         }
         __syncwarp();
     } else {
-        // ------------------------- new_cache slice, then this CTA's epilogue
+        // ------------------- bias, new_cache slice, then this CTA's epilogue
+        // (the bias is read here, off the set-up path, and is in shared
+        // memory long before the accumulator is complete)
         const int etid = threadIdx.x - 64;
+        for (int i = etid; i < BN; i += 128) {
+            const int co = n_tile * BN + i;
+            float b = 0.f;
+            if (p.bias != nullptr && co < p.Cout && index_ok(p.status, co, p.Cout))
+                b = __bfloat162float(__ushort_as_bfloat16(p.bias[co]));
+            bias_s[i] = b;
+        }
+        epi_bar();
         copy_new_cache(p.copy, blockIdx.x, gridDim.x, etid, 128);
 
         const bool ok = mbar_wait(smem_u32(acc_bar), 0, p.status, p.wait_limit_ns);
@@ -195,9 +235,9 @@ conv_tc2_kernel(const __grid_constant__ TcParams p) {
         const bool have_acc = iters > 0;
         const bool store = ok && ty < p.tiles_y;  // a box past the frame stores nothing
         switch (out_block_channels(BN)) {
-            case 64: epilogue_store<64>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, store); break;
-            case 32: epilogue_store<32>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, store); break;
-            default: epilogue_store<16>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, etid, q, lane, store); break;
+            case 64: epilogue_store_warp<64>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, q, lane, store); break;
+            case 32: epilogue_store_warp<32>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, q, lane, store); break;
+            default: epilogue_store_warp<16>(p, tmem_base, have_acc, bias_s, BN, smem, co0, x0, y0, frame, q, lane, store); break;
         }
     }
 

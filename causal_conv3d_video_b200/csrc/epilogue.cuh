@@ -123,4 +123,60 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, uint32_t tmem_
     }
 }
 
+// The same store, each warp on its own: warp q converts its 32 accumulator
+// rows (pixels 32q .. 32q+31 of the box, in row-major order) block by block
+// and, as soon as a block is in shared memory, its lane 0 stores that 32-pixel
+// slab with a tensor store (p.tmap_out_w).  No barrier between the warps, and
+// the stores of one block overlap the conversion of the next.
+template <int kCh>
+__device__ __forceinline__ void epilogue_store_warp(const TcParams& p, uint32_t tmem_acc,
+                                                    bool have_acc, const float* bias_s, int bn,
+                                                    uint8_t* stage, int co0, int x0, int y0,
+                                                    int frame, int q, int lane, bool do_store) {
+    constexpr int kRowB = kCh * 2;
+    const int row = q * 32 + lane;
+    const int nblk = bn / kCh;
+    const int bw = p.box_w;
+    const int sx = bw >= 32 ? x0 + (32 * q) % bw : x0;
+    const int sy = bw >= 32 ? y0 + (32 * q) / bw : y0 + q * (32 / bw);
+    // a slab that starts past the frame's edge has nothing to store
+    const bool slab = do_store && sx < p.W_o && sy < p.H_o &&
+                      index_ok(p.status, frame, (long long)p.N * p.T_o);
+    for (int b = 0; b < nblk; ++b) {
+        uint32_t v[kCh];
+#pragma unroll
+        for (int j = 0; j < kCh / 16; ++j)
+            tmem_ld_32x32b_x16(tmem_acc + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kCh + j * 16),
+                               *reinterpret_cast<uint32_t(*)[16]>(&v[j * 16]));
+        tmem_ld_wait();
+        uint8_t* blk = stage + (size_t)b * (kTileM * kRowB) + (size_t)row * kRowB;
+#pragma unroll
+        for (int c = 0; c < kCh / 8; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int ch = b * kCh + c * 8 + 2 * i;
+                const float a0 = (have_acc ? __uint_as_float(v[c * 8 + 2 * i]) : 0.f) + bias_s[ch];
+                const float a1 =
+                    (have_acc ? __uint_as_float(v[c * 8 + 2 * i + 1]) : 0.f) + bias_s[ch + 1];
+                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+                w[i] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(blk + (swizzled_chunk<kRowB>(c, row) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();  // this lane's writes -> visible to the TMA unit
+        __syncwarp();
+        if (lane == 0 && slab)
+            tma_store_4d(&p.tmap_out_w,
+                         smem_u32(stage + (size_t)b * (kTileM * kRowB) + (size_t)(q * 32) * kRowB),
+                         co0 + b * kCh, sx, sy, frame);
+    }
+    if (lane == 0 && slab) {
+        bulk_commit_group();
+        bulk_wait_group0();  // stores complete before the CTA releases the stage
+    }
+    __syncwarp();
+}
+
 }  // namespace ccv3d

@@ -87,6 +87,9 @@ struct __align__(64) TcParams {
     CUtensorMap tmap_wkw_full, tmap_wkw_half;
     int w_kw_boxes;          // 1: the two-frame kernel loads weights with the maps above
     CUtensorMap tmap_out;    // out as [N*T_o, H_o, W_o, Cout], box [kCh, box_w, box_h, 1]
+    // the same tensor, box of one warp's 32 pixels of a box:
+    // [kCh, min(32, box_w), max(1, 32 / box_w), 1] (pair kernel's epilogue)
+    CUtensorMap tmap_out_w;
     const uint16_t* bias;    // bf16 [Cout] or null
     uint16_t* out;           // bf16 [N, T_o, H_o, W_o, Cout]
     int* status;
