@@ -117,6 +117,16 @@ def test_small_tile_variants(c, env):
     _run_small(c, env=env)
 
 
+@pytest.mark.parametrize("box_w", [128, 64, 32, 16, 8])
+@pytest.mark.parametrize("c", [SMALL[3], SMALL[12], SMALL[16], SMALL[18]], ids=lambda c: c.name)
+def test_small_pair_box_shapes(c, box_w):
+    """The pair kernel on every box shape (128 output pixels as box_w x
+    128/box_w): its epilogue warps each store their own 32 pixels of the box
+    -- a row segment, or 32/box_w whole rows -- clipped at the frame edges."""
+    call, _ = _run_small(c, env={"CCV3D_BOX_W": box_w, "CCV3D_PERSIST": 0, "CCV3D_HALO": 0})
+    assert call.plan.kernel == "tc_pair", call.plan.kernel
+
+
 HALO = [
     # one 128-pixel output row per tile: the input strip is loaded once per (tap, channel block)
     Conv("h96_3x256", 96, 96, 3, 384, T_x=2, cache_len=1, sigma_b=0.1),    # 9 boxes: odd
