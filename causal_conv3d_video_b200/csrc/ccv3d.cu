@@ -820,18 +820,23 @@ Taps make_taps(const ccv3d_plan_s* p) {
 // Paced new_cache copy of the persistent kernel: for each frame the call
 // keeps, the output frame and tap that read it (the last such tap) and that
 // tap's first k-block in the frame's tiles.  Frames no tap reads stay with
-// the sliced copy.  Opt-in (CCV3D_PACED=1): measured on the decoder calls it
-// was no faster than the sliced copy, which starts at once and overlaps the
-// whole GEMM, while the paced copy of the last tiles lengthens the kernel's
-// tail.
-bool paced_copy_on() {
-    return override_env("CCV3D_PACED") != nullptr && env_int("CCV3D_PACED") > 0;
+// the sliced copy.  On by default for one output frame with a cache
+// (measured on B200: the stride-2 360x640 call 160.6 -> 156.9 us, with
+// |C| = 1 126.1 -> 119.6 us, with a ring cache 152.5 -> 146.6 us, the 3x1x1
+// 384 -> 768 call 133.9 -> 131.9 us), off otherwise: with no cache
+// (67.9 -> 71.9 us) and on the two-frame encoder calls (3x1x1 s_t = 2:
+// 146.5 -> 180.6 us) the paced copy of the last tiles lengthens the kernel's
+// tail, while the sliced copy starts at once and overlaps the whole GEMM.
+// CCV3D_PACED=0/1 overrides.
+bool paced_copy_on(const ccv3d_plan_s* p) {
+    if (override_env("CCV3D_PACED") != nullptr) return env_int("CCV3D_PACED") > 0;
+    return p->d.N * p->T_o == 1 && p->d.cache_len >= 1;
 }
 
 void plan_paced_copy(const ccv3d_plan_s* p, TcParams& prm) {
     prm.copy.paced_mask = 0u;
     const int keep = prm.copy.keep;
-    if (!p->persist || keep <= 0 || keep > kMaxPaced || !paced_copy_on()) return;
+    if (!p->persist || keep <= 0 || keep > kMaxPaced || !paced_copy_on(p)) return;
     const ccv3d_desc& d = p->d;
     const int per_tap = d.kh * d.kw * ceil_div(d.Cin, p->BK);
     for (int j = 0; j < keep; ++j) {
@@ -858,7 +863,7 @@ void plan_paced_copy_fused(const ccv3d_plan_s* p, TcParams& prm) {
     prm.copy.paced_mask = 0u;
     const int keep = prm.copy.keep;
     // (the two-CTA-per-SM form has no copy warps: it takes the sliced copy)
-    if (keep <= 0 || keep > kMaxPaced || !paced_copy_on() || p->n_acc == 1) return;
+    if (keep <= 0 || keep > kMaxPaced || !paced_copy_on(p) || p->n_acc == 1) return;
     const ccv3d_desc& d = p->d;
     for (int j = 0; j < keep; ++j) {
         const int t = p->z_len - keep + j;
