@@ -980,7 +980,8 @@ def run_reference(args, rank, world):
     smp = OracleSampler(conv)
     rate = smp.points_per_s()
     budget_s = 150.0  # whole warm-up + timed run
-    n = int(max(16, rate * budget_s / (args.steps + args.warmup)))
+    # a step samples at most as many random points as one call has outputs
+    n = int(max(16, min(smp.n_out, rate * budget_s / (args.steps + args.warmup))))
     for _ in range(args.warmup):
         smp.run(n)
     t = time.perf_counter()
@@ -998,7 +999,9 @@ def run_reference(args, rank, world):
         "config": {"workload": conv.name, "gflop_per_call": round(smp.flops / 1e9, 3),
                    "points_per_step": n},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": smp.cores,
-                         "kind": "oracle", "sample": smp.describe(n * args.steps, total)},
+                         "kind": "oracle",
+                         "sample": f"{args.steps} steps of " + smp.describe(n, total / args.steps)
+                                   + " each"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
