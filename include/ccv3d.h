@@ -131,7 +131,7 @@ typedef struct ccv3d_plan_s* ccv3d_plan_t;
  *
  * The kernel and tiling are the planner's own choice.  Environment variables
  * CCV3D_PERSIST, CCV3D_HALO, CCV3D_FUSE, CCV3D_PAIR, CCV3D_TILE_N,
- * CCV3D_STAGES, CCV3D_BOX_W, CCV3D_HALO_BK, CCV3D_SK_PAIRS, CCV3D_NO_ROT,
+ * CCV3D_STAGES, CCV3D_BOX_W, CCV3D_HALO_BK, CCV3D_SK_PAIRS, CCV3D_NO_ROT, CCV3D_ROT,
  * CCV3D_SIMT_SMEM, CCV3D_SIMT_TILE, CCV3D_SIMT_W16, CCV3D_THIN, CCV3D_W_KW,
  * CCV3D_PACED, CCV3D_FUSED_PERSIST and CCV3D_FORCE_PATH=simt
  * override it for tests and tuning
